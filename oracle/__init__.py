@@ -1,0 +1,246 @@
+"""CPU oracle for the compression-phase step of 1-bit Adam.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+``bench.py``'s CPU-baseline / reference legs may import this package.  The
+product package (``error_compensated_bit_adam_b200``) never imports it, and
+this package never imports the product.
+
+The arithmetic lives in ``onebit_oracle.c`` (plain single-threaded C99,
+``-O2 -ffp-contract=off``); this module only builds it, loads it with
+ctypes and marshals numpy arrays.  ``OracleRun`` is host-side bookkeeping
+over a list of tensors: every tensor is an independent problem (per-tensor
+scales, packing and server chunks), so a multi-tensor step is the
+per-tensor step applied to each tensor in turn.
+
+Parity status: every C function is pinned by ``tests/test_oracle_pins.py``
+(and the pins are shown to catch planted mistakes by
+``tests/test_oracle_mutants.py``); no function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import List, Optional, Sequence
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(HERE, "onebit_oracle.c")
+LIBRARY = os.path.join(HERE, "liboracle.so")
+
+CFLAGS = ["-std=c99", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
+          "-Wall", "-Wextra", "-Werror"]
+
+
+def compile_source(src: str, out: str) -> str:
+    """gcc a C source file into a shared object (atomic replace)."""
+    tmp = out + ".tmp%d" % os.getpid()
+    subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, src, "-lm"])
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile onebit_oracle.c into liboracle.so next to it."""
+    if force or not os.path.exists(LIBRARY) or os.path.getmtime(LIBRARY) < os.path.getmtime(SOURCE):
+        compile_source(SOURCE, LIBRARY)
+    return LIBRARY
+
+
+def _f32(a: np.ndarray) -> np.ndarray:
+    if a.dtype != np.float32 or not a.flags.c_contiguous:
+        raise TypeError("expected a C-contiguous float32 array")
+    return a
+
+
+def _u32(a: np.ndarray) -> np.ndarray:
+    if a.dtype != np.uint32 or not a.flags.c_contiguous:
+        raise TypeError("expected a C-contiguous uint32 array")
+    return a
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _ptr_array(arrays: Sequence[np.ndarray]):
+    arr = (ctypes.c_void_p * max(1, len(arrays)))()
+    for i, a in enumerate(arrays):
+        arr[i] = a.ctypes.data
+    return arr
+
+
+class Oracle:
+    """numpy front end of one loaded copy of the oracle library."""
+
+    def __init__(self, path: str):
+        L = ctypes.CDLL(path)
+        i64, i32, f32, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_void_p
+        L.orc_num_words.argtypes = [i64]
+        L.orc_num_words.restype = i64
+        L.orc_chunk_range.argtypes = [i64, i32, i32, ctypes.POINTER(i64), ctypes.POINTER(i64)]
+        L.orc_chunk_range.restype = None
+        L.orc_adam_warmup_step.argtypes = [i64, i32, i32, f32, f32, f32, f32, vp, vp, vp, vp]
+        L.orc_adam_warmup_step.restype = None
+        L.orc_freeze.argtypes = [i64, i32, f32, f32, vp, vp]
+        L.orc_freeze.restype = None
+        L.orc_worker_compress.argtypes = [i64, f32, vp, vp, vp, vp, vp, ctypes.POINTER(f32)]
+        L.orc_worker_compress.restype = i32
+        L.orc_server_compress.argtypes = [i64, i32, vp, vp, vp, vp, vp, vp]
+        L.orc_server_compress.restype = i32
+        L.orc_apply.argtypes = [i64, i32, f32, vp, vp, vp, vp, vp]
+        L.orc_apply.restype = None
+        self.L = L
+        self.path = path
+
+    def num_words(self, n: int) -> int:
+        return int(self.L.orc_num_words(n))
+
+    def chunk_range(self, n: int, W: int, j: int):
+        b, e = ctypes.c_int64(), ctypes.c_int64()
+        self.L.orc_chunk_range(n, W, j, ctypes.byref(b), ctypes.byref(e))
+        return int(b.value), int(e.value)
+
+    def adam_warmup_step(self, t: int, hp: dict, g: Sequence[np.ndarray], m: np.ndarray,
+                         v: np.ndarray, p: np.ndarray) -> None:
+        n = m.size
+        for a in (*g, m, v, p):
+            _f32(a)
+            assert a.size == n
+        self.L.orc_adam_warmup_step(n, len(g), t, hp["beta1"], hp["beta2"], hp["eps"], hp["lr"],
+                                    _ptr_array(g), _ptr(m), _ptr(v), _ptr(p))
+
+    def freeze(self, Tw: int, hp: dict, v: np.ndarray) -> np.ndarray:
+        d = np.empty_like(_f32(v))
+        self.L.orc_freeze(v.size, Tw, hp["beta2"], hp["eps"], _ptr(v), _ptr(d))
+        return d
+
+    def worker_compress(self, beta1: float, m: np.ndarray, g: np.ndarray, e: np.ndarray,
+                        want_x: bool = False):
+        """Returns (bits, s) or (bits, s, x); e is updated in place."""
+        n = m.size
+        for a in (m, g, e):
+            _f32(a)
+            assert a.size == n
+        bits = np.zeros(self.num_words(n), np.uint32)
+        x = np.empty(n, np.float32) if want_x else None
+        s = ctypes.c_float()
+        rc = self.L.orc_worker_compress(n, beta1, _ptr(m), _ptr(g), _ptr(e), _ptr(bits), _ptr(x),
+                                        ctypes.byref(s))
+        if rc != 0:
+            raise MemoryError("oracle worker stage out of memory")
+        return (bits, np.float32(s.value), x) if want_x else (bits, np.float32(s.value))
+
+    def server_compress(self, bits: Sequence[np.ndarray], s, e_s: np.ndarray,
+                        want_y: bool = False):
+        """Returns (sbits, s_srv[W]) or (sbits, s_srv, y); e_s is updated in place."""
+        n = e_s.size
+        W = len(bits)
+        _f32(e_s)
+        for b in bits:
+            _u32(b)
+            assert b.size == self.num_words(n)
+        s = np.ascontiguousarray(s, np.float32)
+        assert s.size == W
+        sbits = np.zeros(self.num_words(n), np.uint32)
+        s_srv = np.zeros(W, np.float32)
+        y = np.empty(n, np.float32) if want_y else None
+        rc = self.L.orc_server_compress(n, W, _ptr_array(bits), _ptr(s), _ptr(e_s), _ptr(sbits),
+                                        _ptr(s_srv), _ptr(y))
+        if rc != 0:
+            raise MemoryError("oracle server stage out of memory")
+        return (sbits, s_srv, y) if want_y else (sbits, s_srv)
+
+    def apply_update(self, lr: float, sbits: np.ndarray, s_srv, d: np.ndarray, p: np.ndarray,
+                     m: np.ndarray) -> None:
+        n = p.size
+        for a in (d, p, m):
+            _f32(a)
+            assert a.size == n
+        _u32(sbits)
+        s_srv = np.ascontiguousarray(s_srv, np.float32)
+        self.L.orc_apply(n, s_srv.size, lr, _ptr(sbits), _ptr(s_srv), _ptr(d), _ptr(p), _ptr(m))
+
+
+_default: Optional[Oracle] = None
+
+
+def default() -> Oracle:
+    """The oracle built from onebit_oracle.c (built on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+class OracleRun:
+    """The oracle's state for a list of tensors and W simulated workers.
+
+    Per tensor t: p, m, v (then d), e_w[w], e_s; after each compressed step
+    also the packed words and scales of that step.  All arrays are dense
+    float32 / uint32 numpy arrays of the tensor's own length (no padding).
+    """
+
+    def __init__(self, params: Sequence[np.ndarray], W: int, hp: dict,
+                 oracle: Optional[Oracle] = None):
+        self.o = oracle or default()
+        self.W = int(W)
+        self.hp = dict(hp)
+        self.p = [np.array(a, np.float32, copy=True).ravel() for a in params]
+        self.numel = [a.size for a in self.p]
+        self.m = [np.zeros(n, np.float32) for n in self.numel]
+        self.v = [np.zeros(n, np.float32) for n in self.numel]
+        self.d: Optional[List[np.ndarray]] = None
+        self.e_w = [[np.zeros(n, np.float32) for n in self.numel] for _ in range(self.W)]
+        self.e_s = [np.zeros(n, np.float32) for n in self.numel]
+        self.t_warmup = 0
+        self.t_compressed = 0
+        self.bits_w = None  # [w][t] words of the last step
+        self.sbits = None   # [t]
+        self.s_w = None     # [w, t]
+        self.s_srv = None   # [t, j]
+
+    @property
+    def T(self) -> int:
+        return len(self.p)
+
+    def warmup_step(self, grads: Sequence[Sequence[np.ndarray]]) -> None:
+        """grads[w][t]: worker w's gradient of tensor t."""
+        assert self.d is None, "already frozen"
+        self.t_warmup += 1
+        for t in range(self.T):
+            self.o.adam_warmup_step(self.t_warmup, self.hp, [grads[w][t] for w in range(self.W)],
+                                    self.m[t], self.v[t], self.p[t])
+
+    def freeze(self) -> None:
+        assert self.d is None and self.t_warmup >= 1
+        self.d = [self.o.freeze(self.t_warmup, self.hp, v) for v in self.v]
+        for w in range(self.W):
+            for t in range(self.T):
+                self.e_w[w][t][:] = 0
+        for t in range(self.T):
+            self.e_s[t][:] = 0
+
+    def worker_stage(self, w: int, t: int, g: np.ndarray):
+        """Worker stage of one worker on one tensor; returns (bits, s)."""
+        return self.o.worker_compress(self.hp["beta1"], self.m[t], g, self.e_w[w][t])
+
+    def compressed_step(self, grads: Sequence[Sequence[np.ndarray]]) -> None:
+        assert self.d is not None, "not frozen"
+        T, W = self.T, self.W
+        self.bits_w = [[None] * T for _ in range(W)]
+        self.s_w = np.zeros((W, T), np.float32)
+        self.sbits = [None] * T
+        self.s_srv = np.zeros((T, W), np.float32)
+        for t in range(T):
+            for w in range(W):
+                b, s = self.worker_stage(w, t, grads[w][t])
+                self.bits_w[w][t] = b
+                self.s_w[w, t] = s
+            sb, ss = self.o.server_compress([self.bits_w[w][t] for w in range(W)], self.s_w[:, t],
+                                            self.e_s[t])
+            self.sbits[t] = sb
+            self.s_srv[t] = ss
+            self.o.apply_update(self.hp["lr"], sb, ss, self.d[t], self.p[t], self.m[t])
+        self.t_compressed += 1

@@ -1,0 +1,87 @@
+"""The pins catch plausible mistakes in the oracle.
+
+Each case plants one mistake (a dropped term, a wrong sign, a wrong index,
+a transposed bit) in a copy of oracle/onebit_oracle.c, builds it with gcc
+into a temporary directory, and requires at least one pin of
+tests/oracle_pins.py to fail on it.  Mistakes are only ever planted in the
+oracle, on the CPU; none of them reads out of bounds.
+"""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+import oracle_pins
+
+# (name, text in the oracle, replacement)
+MUTANTS = [
+    ("warmup_drops_bias_correction_m", "const float mhat = m[i] / bc1;", "const float mhat = m[i];"),
+    ("warmup_eps_inside_sqrt",
+     "const float root = sqrtf(vhat);\n        const float denom = root + eps;",
+     "const float root = sqrtf(vhat + eps);\n        const float denom = root;"),
+    ("warmup_sums_instead_of_averaging", "const float gbar = acc / wf;", "const float gbar = acc;"),
+    ("warmup_variance_not_squared", "const float gsq = gbar * gbar;", "const float gsq = gbar;"),
+    ("warmup_update_wrong_sign", "p[i] = p[i] - delta;\n    }\n}\n\n/* [1BA, Abstract; Proposed",
+     "p[i] = p[i] + delta;\n    }\n}\n\n/* [1BA, Abstract; Proposed"),
+    ("freeze_drops_bias_correction",
+     "const float vhat = v[i] / bc2;\n        const float root = sqrtf(vhat);\n        d[i]",
+     "const float vhat = v[i];\n        const float root = sqrtf(vhat);\n        d[i]"),
+    ("sign_of_zero_is_minus", "return x >= 0.0f ? 1 : 0;", "return x > 0.0f ? 1 : 0;"),
+    ("scale_divides_by_n", "return (float)sqrt(sum_sq / (double)count);",
+     "return (float)(sqrt(sum_sq) / (double)count);"),
+    ("scale_is_mean_square", "return (float)sqrt(sum_sq / (double)count);",
+     "return (float)(sum_sq / (double)count);"),
+    ("worker_error_wrong_sign", "e[i] = x[i] - signed_scale(", "e[i] = x[i] + signed_scale("),
+    ("momentum_drops_old_m", "const float m_old = beta1 * m[i];\n        const float m_new = c1 * g[i];",
+     "const float m_old = 0.0f * m[i];\n        const float m_new = c1 * g[i];"),
+    ("momentum_drops_gradient",
+     "const float m_old = beta1 * m[i];\n        const float m_new = c1 * g[i];",
+     "const float m_old = beta1 * m[i];\n        const float m_new = c1 * 0.0f * g[i];"),
+    ("worker_forgets_error", "x[i] = m_w + e[i];", "x[i] = m_w;"),
+    ("server_does_not_average", "const float avg = acc / wf;", "const float avg = acc;"),
+    ("server_forgets_error", "y[i] = avg + e_s[i];", "y[i] = avg;"),
+    ("server_uses_worker0_scale", "signed_scale(get_bit(bits[w], i), s[w])",
+     "signed_scale(get_bit(bits[w], i), s[0])"),
+    ("server_reads_neighbour_bit", "signed_scale(get_bit(bits[w], i), s[w])",
+     "signed_scale(get_bit(bits[w], i ^ 1), s[w])"),
+    ("server_error_uses_chunk0_scale",
+     "e_s[i] = y[i] - signed_scale(sign_bit(y[i]), s_srv[j]);",
+     "e_s[i] = y[i] - signed_scale(sign_bit(y[i]), s_srv[0]);"),
+    ("server_error_wrong_sign", "e_s[i] = y[i] - signed_scale(", "e_s[i] = y[i] + signed_scale("),
+    ("chunks_not_word_group_aligned", "const int64_t cw = ((per + 3) / 4) * 4;",
+     "const int64_t cw = per;"),
+    ("apply_wrong_sign", "p[i] = p[i] - delta;\n            m[i] = m_hat;",
+     "p[i] = p[i] + delta;\n            m[i] = m_hat;"),
+    ("apply_keeps_old_momentum", "            m[i] = m_hat;\n", "            (void)m;\n"),
+    ("apply_uses_chunk0_scale", "signed_scale(get_bit(sbits, i), s_srv[j])",
+     "signed_scale(get_bit(sbits, i), s_srv[0])"),
+    ("apply_multiplies_by_d", "const float ratio = m_hat / d[i];", "const float ratio = m_hat * d[i];"),
+    ("packing_bit_order_reversed", "words[i >> 5] |= (uint32_t)1u << (i & 31);",
+     "words[i >> 5] |= (uint32_t)1u << (31 - (i & 31));"),
+]
+
+MUTANT_CFLAGS = [f for f in oracle.CFLAGS if f != "-Werror"]
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(oracle.SOURCE) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(name, old, new, source, tmp_path):
+    assert source.count(old) == 1, f"mutation site for {name} not unique in the oracle"
+    src = tmp_path / f"{name}.c"
+    src.write_text(source.replace(old, new))
+    lib = tmp_path / f"{name}.so"
+    subprocess.check_call(["gcc", *MUTANT_CFLAGS, "-o", str(lib), str(src), "-lm"])
+    mutant = oracle.Oracle(str(lib))
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(mutant)
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the planted mistake {name}"
