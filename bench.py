@@ -1,0 +1,386 @@
+#!/usr/bin/env python
+"""Benchmark of the compression-phase step of 1-bit Adam on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload NAME | --n N --workers W] [--adam-steps S]
+
+One step = one ob_compressed_step over the whole workload: worker stage
+(momentum, error feedback, 1-bit compression) for every simulated worker,
+server stage, gather and preconditioned update.  Default workload: the
+BERT-Large-sized flat fp32 vector, n = 335,544,320, W = 8 simulated
+workers, after 100 full-precision Adam warmup steps and the freeze.
+
+Prints one JSON line (rank 0).  value = parameters updated per second per
+simulated worker, summed over the N GPUs (each GPU runs an independent
+replica: the method's exchange lives inside one GPU's HBM).
+
+--impl reference times the CPU oracle (single-threaded C) on a bounded
+sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from error_compensated_bit_adam_b200 import _binding as B  # noqa: E402
+from error_compensated_bit_adam_b200 import workloads as WL  # noqa: E402
+
+METRIC = "params updated/s per virtual worker (W=8, 336M fp32) and HBM GB/s as % of peak"
+UNIT = "params/s per virtual worker"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0
+GRAD_SETS = 2
+
+
+# ----------------------------------------------------------------- helpers
+
+def algorithmic_bytes(n_real: int, W: int) -> dict:
+    """Bytes per step each kernel must move at minimum, per real parameter:
+    pack 4 (m) + W (4 g + 4 x_prev + 4 x) + W/8 (signs); server W/8 + 4 (y_prev)
+    + 4 (y) + 1/8; apply 1/8 + 4 (d) + 8 (p r/w) + 4 (m); scale kernels
+    ~0."""
+    pack = n_real * (4 + 12 * W + W / 8)
+    server = n_real * (W / 8 + 8 + 1 / 8)
+    apply = n_real * (1 / 8 + 4 + 8 + 4)
+    return {"ob_pack_kernel": pack, "ob_server_kernel": server, "ob_apply_kernel": apply,
+            "step": pack + server + apply}
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled while timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, interval_ms=50):
+        self.proc = None
+        self.path = None
+        self.interval_ms = interval_ms
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms", str(self.interval_ms)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        try:
+            self.proc.terminate()
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+def pick_workload(args) -> WL.Workload:
+    if args.n:
+        return WL.flat(args.n, args.workers, warmup=args.adam_steps or 2, compressed=0, seed=31,
+                       name=f"flat-n{args.n}-W{args.workers}")
+    names = dict(WL.WORKLOADS)
+    for w in WL.sweep():
+        names[w.name] = w
+    wl = names[args.workload]
+    if args.adam_steps is not None:
+        wl = WL.Workload(wl.name, wl.shapes, wl.W, args.adam_steps, wl.compressed_steps, wl.seed,
+                         wl.fan_in_scaling, wl.zero_fraction)
+    return wl
+
+
+def workload_config(wl: WL.Workload, n_pad: int, parallelism: str) -> dict:
+    return {"workload": wl.describe(), "n": wl.n, "n_padded": n_pad, "W": wl.W,
+            "tensors": wl.n_tensors, "adam_warmup_steps": wl.warmup_steps,
+            "grad_sets_cycled": GRAD_SETS,
+            "l2": f"inputs larger than L2: {4 * wl.W * n_pad / 1e9:.2f} GB of gradients per step",
+            "parallelism": parallelism}
+
+
+# ------------------------------------------------------------ oracle timing
+
+def oracle_sample_rate(W: int, n_sample: int, steps: int, warm: int = 1):
+    """Time the oracle's compressed step (single-threaded C) on a flat
+    n_sample vector with W workers; returns (params/s per worker, seconds
+    per step).  Inputs come from the shared generator, on the CPU."""
+    import oracle
+    wl = WL.flat(n_sample, W, warmup=1, compressed=steps, seed=41, name="oracle-sample")
+    offs = [0]
+    p = WL.make_params(wl, offs, n_sample).numpy()
+    scale = WL.grad_scale_vector(wl, offs, n_sample)
+    run = oracle.OracleRun([p], W, WL.HYPER)
+    g = torch.empty((W, n_sample), dtype=torch.float32)
+    WL.fill_grads(wl, 0, scale, g)
+    run.warmup_step([[g[w].numpy()] for w in range(W)])
+    run.freeze()
+    times = []
+    for k in range(warm + steps):
+        WL.fill_grads(wl, 1 + k, scale, g)
+        gl = [[g[w].numpy()] for w in range(W)]
+        t0 = time.perf_counter()
+        run.compressed_step(gl)
+        dt = time.perf_counter() - t0
+        if k >= warm:
+            times.append(dt)
+    t = sum(times) / len(times)
+    return n_sample / t, t
+
+
+def cpu_baseline(W: int, n_sample: int = 1 << 23, steps: int = 4) -> dict:
+    rate, t = oracle_sample_rate(W, n_sample, steps)
+    return {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"flat fp32 n={n_sample}, W={W}: {steps} timed oracle compressed steps "
+                      f"({t:.2f} s each) after 1 Adam step and the freeze; single-threaded C"}
+
+
+# ------------------------------------------------------------- reference arm
+
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = pick_workload(args)
+    n_sample = min(wl.n, 1 << 21)
+    rate, t = oracle_sample_rate(wl.W, n_sample, args.steps, warm=args.warmup)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": workload_config(wl, wl.n, "cpu, single thread"),
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"flat fp32 n={n_sample} of the workload's shape, W={wl.W}; "
+                                   f"{args.warmup} untimed + {args.steps} timed oracle steps"},
+        "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- b200 arm
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world <= 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_b200(args) -> None:
+    from error_compensated_bit_adam_b200.optimizer import OneBitAdam
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    wl = pick_workload(args)
+    offsets, n_pad = B.ob_layout(wl.numels)
+    params = WL.make_params(wl, offsets, n_pad, device=dev)
+    scale = WL.grad_scale_vector(wl, offsets, n_pad, device=dev)
+    opt = OneBitAdam(wl.numels, wl.W, params=params, device=dev, **WL.HYPER)
+    grads = [torch.empty((wl.W, n_pad), dtype=torch.float32, device=dev) for _ in range(GRAD_SETS)]
+
+    step = 0
+    for _ in range(wl.warmup_steps):           # full-precision Adam warmup, untimed
+        WL.fill_grads(wl, step, scale, grads[0])
+        step += 1
+        opt.warmup_step(grads[0])
+    opt.freeze()
+    for gs in grads:                           # fresh draws for the timed steps
+        WL.fill_grads(wl, step, scale, gs)
+        step += 1
+    del scale
+    for k in range(args.warmup):               # untimed compressed steps
+        opt.step(grads[k % GRAD_SETS])
+    torch.cuda.synchronize(dev)
+
+    stream = opt.stream
+    opt.profile(True)
+    opt.profile_read(reset=True)
+    sampler = ClockSampler()
+    if rank == 0:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        opt.step(grads[k % GRAD_SETS])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if rank == 0 else None
+    local_ms = t0.elapsed_time(t1)
+    prof = opt.profile_read(reset=True)
+    opt.profile(False)
+    ms = max_over_ranks(local_ms, world)
+    ms_per_step = ms / args.steps
+    launches = sum(prof[B.ob_kernel_name(k)][1] for k in range(B.OB_K_PACK, B.OB_K_APPLY + 1))
+
+    # roofline of the dominant kernel, from its own events over the timed region
+    peak = measured_peaks()
+    algo = algorithmic_bytes(wl.n, wl.W)
+    pack_ms, pack_n = prof["ob_pack_kernel"]
+    pack_avg_s = pack_ms / 1e3 / max(1, pack_n)
+    achieved = algo["ob_pack_kernel"] / pack_avg_s / 1e9
+    step_gbs = algo["step"] / (ms_per_step / 1e3) / 1e9
+    per_kernel = {}
+    for name, (kms, cnt) in prof.items():
+        if cnt:
+            entry = {"ms_avg": kms / cnt, "share": kms / max(1e-12, sum(v[0] for v in prof.values()))}
+            if name in algo:
+                entry["gbs"] = algo[name] / (kms / cnt / 1e3) / 1e9
+            per_kernel[name] = entry
+
+    # end to end: host gradients in pinned memory, copied in every step, and
+    # the step's server scales read back, through ob_compressed_step_host
+    e2e = None
+    try:
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        try:
+            host = torch.empty((wl.W, n_pad), dtype=torch.float32, pin_memory=True)
+            pinned = True
+        except RuntimeError:
+            host = torch.empty((wl.W, n_pad), dtype=torch.float32)
+            pinned = False
+        host.copy_(grads[0])
+        out = np.zeros(wl.n_tensors * wl.W, np.float32)
+        opt.step_host(host, out)                    # untimed: staging allocation
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        w0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            opt.step_host(host, out)
+        e2e_s = max_over_ranks(time.perf_counter() - w0, world) / e2e_steps
+        e2e = {"value": world * wl.n / e2e_s, "unit": UNIT,
+               "h2d_bytes_per_step": int(host.numel() * 4), "d2h_bytes_per_step": int(out.nbytes),
+               "ms_per_step": e2e_s * 1e3, "pinned": pinned, "steps": e2e_steps,
+               "call": "ob_compressed_step_host"}
+        del host
+    except Exception as exc:  # reported, never hidden
+        e2e = {"value": None, "unit": UNIT, "error": repr(exc)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl.W)
+
+    if rank == 0:
+        value = world * wl.n / (ms_per_step / 1e3)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": workload_config(wl, n_pad, "replicas" if world > 1 else "single GPU"),
+            "params_per_s_aggregate_all_workers": value * wl.W,
+            "hbm_gbs_step": step_gbs,
+            "hbm_frac_of_measured_peak_step": step_gbs / peak["hbm_gbs"],
+            "hbm_frac_of_8tbs_step": step_gbs / NOMINAL_HBM_GBS,
+            "roofline": {"bound": "hbm", "kernel": "ob_pack_kernel", "achieved": achieved,
+                         "peak": peak["hbm_gbs"], "peak_source": peak["source"], "unit": "GB/s",
+                         "frac": achieved / peak["hbm_gbs"], "traffic": args.pack_traffic,
+                         "algorithmic_bytes_per_launch": algo["ob_pack_kernel"],
+                         "avg_launch_ms": pack_avg_s * 1e3},
+            "kernels": per_kernel,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["b200", "reference"], default="b200")
+    ap.add_argument("--workload", default=WL.BERT_LARGE_FLAT_W8.name)
+    ap.add_argument("--n", type=int, default=0, help="flat vector of n elements instead")
+    ap.add_argument("--workers", type=int, default=8, help="W for --n")
+    ap.add_argument("--adam-steps", type=int, default=None, help="override warmup Adam steps")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pack-traffic", type=float, default=None,
+                    help="ncu DRAM bytes per ob_pack_kernel launch at this workload, if measured")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "b200" and not args.n:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_b200(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,235 @@
+"""ctypes binding of libonebit (include/onebit.h), one Python function per C
+entry point, with the same names.  Marshalling only: every step of the
+method runs in the library's CUDA kernels.  A non-OK status raises
+OnebitError; there is no fallback of any kind when the library is missing.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import List, Optional, Sequence, Tuple
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(HERE, "libonebit.so")
+
+OB_ABI_VERSION = 1
+OB_MAX_WORKERS = 64
+OB_TENSOR_ALIGN = 128
+
+OB_OK = 0
+OB_ERR_INVALID_ARG = 1
+OB_ERR_PHASE = 2
+OB_ERR_ALIGN = 3
+OB_ERR_WORKSPACE = 4
+OB_ERR_OOM = 5
+OB_ERR_CUDA = 6
+OB_ERR_DEVICE_TIMEOUT = 7
+
+OB_STATE_P = 0
+OB_STATE_M = 1
+OB_STATE_V = 2
+OB_STATE_D = 3
+OB_STATE_E_WORKER = 4
+OB_STATE_E_SERVER = 5
+OB_STATE_S_WORKER = 6
+OB_STATE_S_SERVER = 7
+OB_STATE_BITS_WORKER = 8
+OB_STATE_BITS_SERVER = 9
+OB_STATE_STEP = 10
+
+OB_K_WARMUP = 0
+OB_K_FREEZE = 1
+OB_K_PACK = 2
+OB_K_PACK_SCALE = 3
+OB_K_SERVER = 4
+OB_K_SERVER_SCALE = 5
+OB_K_APPLY = 6
+OB_NUM_KERNELS = 7
+
+# Every symbol include/onebit.h declares.
+EXPORTS = (
+    "ob_status_string", "ob_abi_version", "ob_layout", "ob_chunk_range", "ob_workspace_bytes",
+    "ob_create", "ob_destroy", "ob_warmup_adam_step", "ob_freeze_variance", "ob_compressed_step",
+    "ob_host_staging_bytes", "ob_compressed_step_host", "ob_read_state", "ob_write_state",
+    "ob_profile_enable", "ob_profile_read", "ob_kernel_name", "ob_test_fail_host_alloc",
+)
+
+
+class OnebitError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = int(status)
+        self.call = call
+        super().__init__(f"{call}: {status_name(status)}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libonebit.so (built in-tree).  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIBRARY):
+        raise RuntimeError(
+            f"{LIBRARY} is not built; run `python -m error_compensated_bit_adam_b200.build` "
+            "(or __graft_entry__.build()).  There is no fallback implementation.")
+    L = ctypes.CDLL(LIBRARY)
+    i32, i64, f32, vp, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+    P64 = ctypes.POINTER(i64)
+    sig = {
+        "ob_status_string": (ctypes.c_char_p, [i32]),
+        "ob_abi_version": (i32, []),
+        "ob_layout": (i32, [i32, P64, P64, P64]),
+        "ob_chunk_range": (i32, [i64, i32, i32, P64, P64]),
+        "ob_workspace_bytes": (i32, [i32, P64, i32, ctypes.POINTER(sz)]),
+        "ob_create": (i32, [i32, P64, i32, f32, f32, f32, f32, vp, vp, sz, vp, ctypes.POINTER(vp)]),
+        "ob_destroy": (None, [vp]),
+        "ob_warmup_adam_step": (i32, [vp, vp]),
+        "ob_freeze_variance": (i32, [vp]),
+        "ob_compressed_step": (i32, [vp, vp]),
+        "ob_host_staging_bytes": (i32, [vp, ctypes.POINTER(sz)]),
+        "ob_compressed_step_host": (i32, [vp, vp, vp, sz, vp]),
+        "ob_read_state": (i32, [vp, i32, i32, vp, sz]),
+        "ob_write_state": (i32, [vp, i32, i32, vp, sz]),
+        "ob_profile_enable": (i32, [vp, i32]),
+        "ob_profile_read": (i32, [vp, ctypes.POINTER(ctypes.c_double), P64, i32]),
+        "ob_kernel_name": (ctypes.c_char_p, [i32]),
+        "ob_test_fail_host_alloc": (None, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    if L.ob_abi_version() != OB_ABI_VERSION:
+        raise RuntimeError("libonebit ABI version mismatch")
+    _lib = L
+    return L
+
+
+def status_name(status: int) -> str:
+    try:
+        return lib().ob_status_string(int(status)).decode()
+    except Exception:  # the library may be what failed to load
+        return f"status {status}"
+
+
+def _check(status: int, call: str) -> None:
+    if status != OB_OK:
+        raise OnebitError(status, call)
+
+
+def _i64_array(values: Sequence[int]):
+    arr = (ctypes.c_int64 * max(1, len(values)))(*[int(v) for v in values])
+    return arr
+
+
+def _ptrs(ptrs: Sequence[int]):
+    arr = (ctypes.c_void_p * max(1, len(ptrs)))()
+    for i, p in enumerate(ptrs):
+        arr[i] = int(p)
+    return arr
+
+
+# --------------------------------------------------------------- host only
+
+def ob_status_string(status: int) -> str:
+    return lib().ob_status_string(int(status)).decode()
+
+
+def ob_abi_version() -> int:
+    return int(lib().ob_abi_version())
+
+
+def ob_layout(numel: Sequence[int]) -> Tuple[List[int], int]:
+    """Tensor offsets and n_padded of the padded layout."""
+    n = len(numel)
+    offs = (ctypes.c_int64 * max(1, n))()
+    total = ctypes.c_int64()
+    _check(lib().ob_layout(n, _i64_array(numel), offs, ctypes.byref(total)), "ob_layout")
+    return [int(offs[i]) for i in range(n)], int(total.value)
+
+
+def ob_chunk_range(numel: int, W: int, j: int) -> Tuple[int, int]:
+    b, e = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().ob_chunk_range(int(numel), int(W), int(j), ctypes.byref(b), ctypes.byref(e)),
+           "ob_chunk_range")
+    return int(b.value), int(e.value)
+
+
+def ob_workspace_bytes(numel: Sequence[int], W: int) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().ob_workspace_bytes(len(numel), _i64_array(numel), int(W), ctypes.byref(out)),
+           "ob_workspace_bytes")
+    return int(out.value)
+
+
+def ob_kernel_name(kernel_id: int) -> Optional[str]:
+    r = lib().ob_kernel_name(int(kernel_id))
+    return None if r is None else r.decode()
+
+
+def ob_test_fail_host_alloc(countdown: int) -> None:
+    lib().ob_test_fail_host_alloc(int(countdown))
+
+
+# ----------------------------------------------------------------- context
+
+def ob_create(numel: Sequence[int], W: int, beta1: float, beta2: float, eps: float, lr: float,
+              d_params: int, d_workspace: int, workspace_bytes: int, cuda_stream: int) -> int:
+    """Returns the context handle (an opaque integer)."""
+    out = ctypes.c_void_p()
+    _check(lib().ob_create(len(numel), _i64_array(numel), int(W), float(beta1), float(beta2),
+                           float(eps), float(lr), int(d_params), int(d_workspace),
+                           int(workspace_bytes), int(cuda_stream), ctypes.byref(out)), "ob_create")
+    return int(out.value)
+
+
+def ob_destroy(ctx: int) -> None:
+    lib().ob_destroy(int(ctx) if ctx else None)
+
+
+def ob_warmup_adam_step(ctx: int, d_grads: Sequence[int]) -> None:
+    _check(lib().ob_warmup_adam_step(ctx, _ptrs(d_grads)), "ob_warmup_adam_step")
+
+
+def ob_freeze_variance(ctx: int) -> None:
+    _check(lib().ob_freeze_variance(ctx), "ob_freeze_variance")
+
+
+def ob_compressed_step(ctx: int, d_grads: Sequence[int]) -> None:
+    _check(lib().ob_compressed_step(ctx, _ptrs(d_grads)), "ob_compressed_step")
+
+
+def ob_host_staging_bytes(ctx: int) -> int:
+    out = ctypes.c_size_t()
+    _check(lib().ob_host_staging_bytes(ctx, ctypes.byref(out)), "ob_host_staging_bytes")
+    return int(out.value)
+
+
+def ob_compressed_step_host(ctx: int, h_grads: Sequence[int], d_staging: int, staging_bytes: int,
+                            h_server_scales: Optional[int]) -> None:
+    _check(lib().ob_compressed_step_host(ctx, _ptrs(h_grads), int(d_staging), int(staging_bytes),
+                                         int(h_server_scales) if h_server_scales else None),
+           "ob_compressed_step_host")
+
+
+def ob_read_state(ctx: int, kind: int, index: int, host_dst: int, nbytes: int) -> None:
+    _check(lib().ob_read_state(ctx, int(kind), int(index), int(host_dst), int(nbytes)),
+           "ob_read_state")
+
+
+def ob_write_state(ctx: int, kind: int, index: int, host_src: int, nbytes: int) -> None:
+    _check(lib().ob_write_state(ctx, int(kind), int(index), int(host_src), int(nbytes)),
+           "ob_write_state")
+
+
+def ob_profile_enable(ctx: int, on: bool) -> None:
+    _check(lib().ob_profile_enable(ctx, 1 if on else 0), "ob_profile_enable")
+
+
+def ob_profile_read(ctx: int, reset: bool = False) -> Tuple[List[float], List[int]]:
+    ms = (ctypes.c_double * OB_NUM_KERNELS)()
+    n = (ctypes.c_int64 * OB_NUM_KERNELS)()
+    _check(lib().ob_profile_read(ctx, ms, n, 1 if reset else 0), "ob_profile_read")
+    return [float(v) for v in ms], [int(v) for v in n]

@@ -1,0 +1,897 @@
+// onebit.cu -- host side of libonebit: the C ABI declared in include/onebit.h.
+//
+// Owns host-side planning (padded layout, server chunks, the tile work
+// list), argument and phase validation, workspace carving, kernel launches
+// on the caller's stream, state read/write and the profiling counters.  It
+// allocates no device memory: the caller passes the workspace.
+//
+// Method: "1-bit Adam: Communication Efficient Large-Scale Training with
+// Adam's Convergence Speed" (review page), sections "Abstract" and
+// "Proposed method" ([1BA]).
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <unordered_set>
+#include <vector>
+
+#include <cuda_runtime.h>
+
+#include "../../include/onebit.h"
+#include "onebit_kernels.cuh"
+
+using onebit::Tile;
+using onebit::kTile;
+using onebit::kThreads;
+using onebit::kScaleThreads;
+
+namespace {
+
+constexpr uint64_t kMagic = 0x31424954414441ull;  // "ADATIB1"
+constexpr int64_t kMaxElements = int64_t(1) << 40;
+constexpr int64_t kDecodeStage = int64_t(1) << 20;   // elements decoded per read round
+constexpr int64_t kHostSlice = int64_t(1) << 22;     // gradient elements per worker per H2D slice
+constexpr size_t kWsAlign = 256;
+
+// ------------------------------------------------------------ test hook
+std::mutex g_alloc_mu;
+int g_fail_countdown = 0;
+
+// Called before each host allocation; throws std::bad_alloc when the test
+// hook's countdown reaches zero.
+void host_alloc_point() {
+    std::lock_guard<std::mutex> lk(g_alloc_mu);
+    if (g_fail_countdown > 0 && --g_fail_countdown == 0) throw std::bad_alloc();
+}
+
+// ------------------------------------------------------ live contexts
+std::mutex g_live_mu;
+std::unordered_set<const ob_ctx *> g_live;
+
+bool is_live(const ob_ctx *c) {
+    std::lock_guard<std::mutex> lk(g_live_mu);
+    return c && g_live.count(c) != 0;
+}
+
+// ------------------------------------------------------------ planning
+
+int64_t round_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// [1BA, Proposed method, 4]: server j of W owns sign words
+// [j*cw, min(nw, (j+1)*cw)) of a tensor, cw = roundup(ceil(nw/W), 4).
+void chunk_bounds(int64_t n, int W, int j, int64_t *b, int64_t *e) {
+    const int64_t words = (n + 31) / 32;
+    const int64_t per_server = round_up((words + W - 1) / W, 4);
+    const int64_t lo = std::min<int64_t>(words, (int64_t)j * per_server);
+    const int64_t hi = std::min<int64_t>(words, (int64_t)(j + 1) * per_server);
+    *b = std::min<int64_t>(n, 32 * lo);
+    *e = std::min<int64_t>(n, 32 * hi);
+}
+
+struct Plan {
+    int T = 0, W = 0;
+    std::vector<int64_t> numel, offset;
+    int64_t n_pad = 0;
+    std::vector<Tile> tiles;
+    std::vector<int> tensor_tile_begin;  // [T+1]
+    std::vector<int> chunk_tile_begin;   // [T*W+1]
+    std::vector<int64_t> chunk_len;      // [T*W]
+};
+
+ob_status check_list(int n_tensors, const int64_t *numel) {
+    if (n_tensors < 1 || !numel) return OB_ERR_INVALID_ARG;
+    int64_t total = 0;
+    for (int t = 0; t < n_tensors; ++t) {
+        if (numel[t] < 0 || numel[t] > kMaxElements) return OB_ERR_INVALID_ARG;
+        total += round_up(numel[t], OB_TENSOR_ALIGN);
+        if (total > kMaxElements) return OB_ERR_INVALID_ARG;
+    }
+    return OB_OK;
+}
+
+// Padded layout, server chunks and the tile work list: tiles of up to kTile
+// elements that never cross a tensor or chunk boundary, in layout order.
+ob_status make_plan(int n_tensors, const int64_t *numel, int W, bool with_tiles, Plan *pl) {
+    ob_status st = check_list(n_tensors, numel);
+    if (st != OB_OK) return st;
+    if (W < 1 || W > OB_MAX_WORKERS) return OB_ERR_INVALID_ARG;
+    host_alloc_point();
+    pl->T = n_tensors;
+    pl->W = W;
+    pl->numel.assign(numel, numel + n_tensors);
+    pl->offset.resize(n_tensors);
+    int64_t pos = 0;
+    for (int t = 0; t < n_tensors; ++t) {
+        pl->offset[t] = pos;
+        pos += round_up(numel[t], OB_TENSOR_ALIGN);
+    }
+    pl->n_pad = pos;
+    if (!with_tiles) return OB_OK;
+    host_alloc_point();
+    pl->tensor_tile_begin.assign(n_tensors + 1, 0);
+    pl->chunk_tile_begin.assign((size_t)n_tensors * W + 1, 0);
+    pl->chunk_len.assign((size_t)n_tensors * W, 0);
+    int64_t count = 0;
+    for (int t = 0; t < n_tensors; ++t) count += (numel[t] + kTile - 1) / kTile + W;
+    if (count > INT32_MAX) return OB_ERR_INVALID_ARG;
+    host_alloc_point();
+    pl->tiles.reserve((size_t)count);
+    for (int t = 0; t < n_tensors; ++t) {
+        pl->tensor_tile_begin[t] = (int)pl->tiles.size();
+        for (int j = 0; j < W; ++j) {
+            const int c = t * W + j;
+            pl->chunk_tile_begin[c] = (int)pl->tiles.size();
+            int64_t b, e;
+            chunk_bounds(numel[t], W, j, &b, &e);
+            pl->chunk_len[c] = e - b;
+            for (int64_t s = b; s < e; s += kTile) {
+                Tile tl;
+                tl.begin = pl->offset[t] + s;
+                tl.count = (int32_t)std::min<int64_t>(kTile, e - s);
+                tl.tensor = t;
+                tl.chunk = j;
+                tl.reserved = 0;
+                pl->tiles.push_back(tl);
+            }
+        }
+    }
+    pl->tensor_tile_begin[n_tensors] = (int)pl->tiles.size();
+    pl->chunk_tile_begin[(size_t)n_tensors * W] = (int)pl->tiles.size();
+    return OB_OK;
+}
+
+// Byte offsets of the workspace regions.
+struct Carve {
+    size_t m, v, x, y, bits, sbits, s_prev, s_last, sp_prev, sp_last, partial_w, partial_s, tiles,
+        tensor_tile_begin, chunk_tile_begin, numel, chunk_len, stage, total;
+};
+
+Carve carve(const Plan &pl) {
+    Carve c{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = (off + bytes + kWsAlign - 1) / kWsAlign * kWsAlign;
+        return o;
+    };
+    const size_t n = (size_t)pl.n_pad, W = (size_t)pl.W, T = (size_t)pl.T;
+    const size_t nt = pl.tiles.size();
+    c.m = take(n * 4);
+    c.v = take(n * 4);
+    c.x = take(W * n * 4);
+    c.y = take(n * 4);
+    c.bits = take(W * (n / 32) * 4);
+    c.sbits = take((n / 32) * 4);
+    c.s_prev = take(W * T * 4);
+    c.s_last = take(W * T * 4);
+    c.sp_prev = take(T * W * 4);
+    c.sp_last = take(T * W * 4);
+    c.partial_w = take(W * nt * 8);
+    c.partial_s = take(nt * 8);
+    c.tiles = take(nt * sizeof(Tile));
+    c.tensor_tile_begin = take((T + 1) * 4);
+    c.chunk_tile_begin = take((T * W + 1) * 4);
+    c.numel = take(T * 8);
+    c.chunk_len = take(T * W * 8);
+    c.stage = take((size_t)kDecodeStage * 4);
+    c.total = off;
+    return c;
+}
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// Runs of consecutive tiles whose padded span fits `limit` elements.
+struct Run {
+    int tile_lo, tile_hi;
+    int64_t elem_lo, elem_hi;
+};
+
+std::vector<Run> make_runs(const std::vector<Tile> &tiles, int64_t limit) {
+    host_alloc_point();
+    std::vector<Run> runs;
+    size_t k = 0;
+    while (k < tiles.size()) {
+        Run r;
+        r.tile_lo = (int)k;
+        r.elem_lo = tiles[k].begin;
+        r.elem_hi = tiles[k].begin + round_up(tiles[k].count, OB_TENSOR_ALIGN);
+        ++k;
+        while (k < tiles.size()) {
+            const int64_t hi = tiles[k].begin + round_up(tiles[k].count, OB_TENSOR_ALIGN);
+            if (hi - r.elem_lo > limit) break;
+            r.elem_hi = hi;
+            ++k;
+        }
+        r.tile_hi = (int)k;
+        runs.push_back(r);
+    }
+    return runs;
+}
+
+// Switches to a device for the duration of a call, then back.
+struct DeviceGuard {
+    int prev = -1;
+    bool ok = true;
+    explicit DeviceGuard(int dev) {
+        if (cudaGetDevice(&prev) != cudaSuccess) {
+            ok = false;
+            return;
+        }
+        if (prev != dev && cudaSetDevice(dev) != cudaSuccess) ok = false;
+    }
+    ~DeviceGuard() {
+        int cur;
+        if (prev >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev) cudaSetDevice(prev);
+    }
+};
+
+const char *const kKernelNames[OB_NUM_KERNELS] = {
+    "ob_warmup_kernel", "ob_freeze_kernel",       "ob_pack_kernel", "ob_pack_scale_kernel",
+    "ob_server_kernel", "ob_server_scale_kernel", "ob_apply_kernel"};
+
+}  // namespace
+
+// ------------------------------------------------------------------ ctx
+
+struct ob_ctx {
+    uint64_t magic = kMagic;
+    int device = 0;
+    Plan plan;
+    Carve cv;
+    std::vector<Run> host_runs;
+    float beta1, beta2, eps, lr, c1, c2;
+    float *params = nullptr;
+    char *ws = nullptr;
+    cudaStream_t stream = nullptr;
+    cudaStream_t copy_stream = nullptr;
+    cudaEvent_t ev_copied[2] = {nullptr, nullptr};
+    cudaEvent_t ev_consumed[2] = {nullptr, nullptr};
+    cudaEvent_t ev_start = nullptr;
+    int64_t t_warmup = 0, t_compressed = 0;
+    bool frozen = false;
+    bool broken = false;
+    // profiling
+    bool profiling = false;
+    std::vector<cudaEvent_t> event_pool;
+    std::vector<std::pair<int, std::pair<cudaEvent_t, cudaEvent_t>>> pending;
+    double kernel_ms[OB_NUM_KERNELS] = {};
+    int64_t kernel_launches[OB_NUM_KERNELS] = {};
+
+    template <class T> T *at(size_t off) const { return reinterpret_cast<T *>(ws + off); }
+    float *m() const { return at<float>(cv.m); }
+    float *v() const { return at<float>(cv.v); }
+    float *x() const { return at<float>(cv.x); }
+    float *y() const { return at<float>(cv.y); }
+    uint32_t *bits() const { return at<uint32_t>(cv.bits); }
+    uint32_t *sbits() const { return at<uint32_t>(cv.sbits); }
+    float *s_prev() const { return at<float>(cv.s_prev); }
+    float *s_last() const { return at<float>(cv.s_last); }
+    float *sp_prev() const { return at<float>(cv.sp_prev); }
+    float *sp_last() const { return at<float>(cv.sp_last); }
+    double *partial_w() const { return at<double>(cv.partial_w); }
+    double *partial_s() const { return at<double>(cv.partial_s); }
+    Tile *tiles() const { return at<Tile>(cv.tiles); }
+    int *tensor_tile_begin() const { return at<int>(cv.tensor_tile_begin); }
+    int *chunk_tile_begin() const { return at<int>(cv.chunk_tile_begin); }
+    int64_t *numel() const { return at<int64_t>(cv.numel); }
+    int64_t *chunk_len() const { return at<int64_t>(cv.chunk_len); }
+    float *stage() const { return at<float>(cv.stage); }
+    int n_tiles() const { return (int)plan.tiles.size(); }
+};
+
+namespace {
+
+ob_status fail_cuda(ob_ctx *c, cudaError_t e) {
+    if (e == cudaSuccess) return OB_OK;
+    if (c) c->broken = true;
+    return OB_ERR_CUDA;
+}
+
+ob_status check_ctx(const ob_ctx *c) {
+    if (!is_live(c) || c->magic != kMagic) return OB_ERR_INVALID_ARG;
+    if (c->broken) return OB_ERR_CUDA;
+    return OB_OK;
+}
+
+// Profiling: an event pair around one kernel, summed at ob_profile_read.
+cudaEvent_t take_event(ob_ctx *c) {
+    if (!c->event_pool.empty()) {
+        cudaEvent_t e = c->event_pool.back();
+        c->event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+struct KernelTimer {
+    ob_ctx *c;
+    int id;
+    cudaEvent_t a = nullptr, b = nullptr;
+    KernelTimer(ob_ctx *ctx, int k) : c(ctx), id(k) {
+        if (!c->profiling) return;
+        a = take_event(c);
+        b = take_event(c);
+        if (a && b) cudaEventRecord(a, c->stream);
+    }
+    void stop() {
+        if (!c->profiling || !a || !b) return;
+        cudaEventRecord(b, c->stream);
+        c->pending.push_back({id, {a, b}});
+        a = b = nullptr;
+    }
+};
+
+dim3 grid1(int n) { return dim3((unsigned)n); }
+
+ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int tile_lo, int tile_hi) {
+    if (tile_hi <= tile_lo) return OB_OK;
+    onebit::PackParams P;
+    P.tiles = c->tiles();
+    P.tile_base = tile_lo;
+    P.n_tiles = c->n_tiles();
+    P.m = c->m();
+    for (int w = 0; w < OB_MAX_WORKERS; ++w) P.g[w] = w < c->plan.W ? g[w] : nullptr;
+    P.g_offset = g_offset;
+    P.x = c->x();
+    P.bits = c->bits();
+    P.s_prev = c->s_prev();
+    P.partial = c->partial_w();
+    P.n_pad = c->plan.n_pad;
+    P.W = c->plan.W;
+    P.T = c->plan.T;
+    P.beta1 = c->beta1;
+    P.c1 = c->c1;
+    onebit::ob_pack_kernel<<<grid1(tile_hi - tile_lo), kThreads, 0, c->stream>>>(P);
+    return fail_cuda(c, cudaGetLastError());
+}
+
+// Everything of a compressed step after the worker stage's tile kernels.
+ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
+    const int T = c->plan.T, W = c->plan.W, nt = c->n_tiles();
+    pack_timer.stop();
+    {
+        KernelTimer k(c, OB_K_PACK_SCALE);
+        onebit::ob_pack_scale_kernel<<<dim3((unsigned)T, (unsigned)W), kScaleThreads, 0, c->stream>>>(
+            c->partial_w(), nt, c->tensor_tile_begin(), c->numel(), T, c->s_prev(), c->s_last());
+        k.stop();
+        ob_status st = fail_cuda(c, cudaGetLastError());
+        if (st != OB_OK) return st;
+    }
+    if (nt > 0) {
+        KernelTimer k(c, OB_K_SERVER);
+        onebit::ServerParams P;
+        P.tiles = c->tiles();
+        P.bits = c->bits();
+        P.s_w = c->s_prev();
+        P.y = c->y();
+        P.sp_prev = c->sp_prev();
+        P.sbits = c->sbits();
+        P.partial = c->partial_s();
+        P.n_pad = c->plan.n_pad;
+        P.W = W;
+        P.T = T;
+        onebit::ob_server_kernel<<<grid1(nt), kThreads, 0, c->stream>>>(P);
+        k.stop();
+        ob_status st = fail_cuda(c, cudaGetLastError());
+        if (st != OB_OK) return st;
+    }
+    {
+        KernelTimer k(c, OB_K_SERVER_SCALE);
+        onebit::ob_server_scale_kernel<<<grid1(T * W), kScaleThreads, 0, c->stream>>>(
+            c->partial_s(), c->chunk_tile_begin(), c->chunk_len(), c->sp_prev(), c->sp_last());
+        k.stop();
+        ob_status st = fail_cuda(c, cudaGetLastError());
+        if (st != OB_OK) return st;
+    }
+    if (nt > 0) {
+        KernelTimer k(c, OB_K_APPLY);
+        onebit::ApplyParams P;
+        P.tiles = c->tiles();
+        P.sbits = c->sbits();
+        P.sp = c->sp_last();
+        P.d = c->v();
+        P.p = c->params;
+        P.m = c->m();
+        P.W = W;
+        P.lr = c->lr;
+        onebit::ob_apply_kernel<<<grid1(nt), kThreads, 0, c->stream>>>(P);
+        k.stop();
+        ob_status st = fail_cuda(c, cudaGetLastError());
+        if (st != OB_OK) return st;
+    }
+    return OB_OK;
+}
+
+ob_status check_grads(const ob_ctx *c, const float *const *g) {
+    if (!g) return OB_ERR_INVALID_ARG;
+    if (c->plan.n_pad == 0) return OB_OK;  // nothing is read
+    for (int w = 0; w < c->plan.W; ++w) {
+        if (!g[w]) return OB_ERR_INVALID_ARG;
+        if (!aligned(g[w], 16)) return OB_ERR_ALIGN;
+    }
+    return OB_OK;
+}
+
+size_t state_bytes(const ob_ctx *c, int kind) {
+    const size_t n = (size_t)c->plan.n_pad, W = (size_t)c->plan.W, T = (size_t)c->plan.T;
+    switch (kind) {
+    case OB_STATE_P: case OB_STATE_M: case OB_STATE_V: case OB_STATE_D:
+    case OB_STATE_E_WORKER: case OB_STATE_E_SERVER:
+        return n * 4;
+    case OB_STATE_S_WORKER: case OB_STATE_S_SERVER:
+        return W * T * 4;
+    case OB_STATE_BITS_WORKER: case OB_STATE_BITS_SERVER:
+        return (n / 32) * 4;
+    case OB_STATE_STEP:
+        return 3 * sizeof(int64_t);
+    default:
+        return 0;
+    }
+}
+
+// Decode a lazily stored error buffer (x or y with its scales) into host
+// memory, run by run through the staging region.
+ob_status read_error(ob_ctx *c, const float *src, const float *scales, int stride_t, int stride_j,
+                     float *host) {
+    std::memset(host, 0, (size_t)c->plan.n_pad * 4);
+    std::vector<Run> runs = make_runs(c->plan.tiles, kDecodeStage);
+    for (const Run &r : runs) {
+        const int64_t span = r.elem_hi - r.elem_lo;
+        ob_status st = fail_cuda(c, cudaMemsetAsync(c->stage(), 0, (size_t)span * 4, c->stream));
+        if (st != OB_OK) return st;
+        onebit::DecodeParams P;
+        P.tiles = c->tiles();
+        P.tile_base = r.tile_lo;
+        P.x = src;
+        P.scales = scales;
+        P.stride_t = stride_t;
+        P.stride_j = stride_j;
+        P.out = c->stage();
+        P.out_base = r.elem_lo;
+        onebit::ob_decode_error_kernel<<<grid1(r.tile_hi - r.tile_lo), kThreads, 0, c->stream>>>(P);
+        st = fail_cuda(c, cudaGetLastError());
+        if (st != OB_OK) return st;
+        st = fail_cuda(c, cudaMemcpyAsync(host + r.elem_lo, c->stage(), (size_t)span * 4,
+                                          cudaMemcpyDeviceToHost, c->stream));
+        if (st != OB_OK) return st;
+        st = fail_cuda(c, cudaStreamSynchronize(c->stream));
+        if (st != OB_OK) return st;
+    }
+    return OB_OK;
+}
+
+}  // namespace
+
+// ================================================================= C ABI
+
+extern "C" {
+
+const char *ob_status_string(ob_status s) {
+    switch (s) {
+    case OB_OK: return "OB_OK";
+    case OB_ERR_INVALID_ARG: return "OB_ERR_INVALID_ARG";
+    case OB_ERR_PHASE: return "OB_ERR_PHASE";
+    case OB_ERR_ALIGN: return "OB_ERR_ALIGN";
+    case OB_ERR_WORKSPACE: return "OB_ERR_WORKSPACE";
+    case OB_ERR_OOM: return "OB_ERR_OOM";
+    case OB_ERR_CUDA: return "OB_ERR_CUDA";
+    case OB_ERR_DEVICE_TIMEOUT: return "OB_ERR_DEVICE_TIMEOUT";
+    }
+    return "OB_UNKNOWN_STATUS";
+}
+
+int ob_abi_version(void) { return OB_ABI_VERSION; }
+
+const char *ob_kernel_name(int id) {
+    return (id >= 0 && id < OB_NUM_KERNELS) ? kKernelNames[id] : nullptr;
+}
+
+void ob_test_fail_host_alloc(int countdown) {
+    std::lock_guard<std::mutex> lk(g_alloc_mu);
+    g_fail_countdown = countdown > 0 ? countdown : 0;
+}
+
+ob_status ob_layout(int n_tensors, const int64_t *numel, int64_t *tensor_offsets,
+                    int64_t *n_padded) {
+    if (!n_padded) return OB_ERR_INVALID_ARG;
+    ob_status st = check_list(n_tensors, numel);
+    if (st != OB_OK) return st;
+    int64_t pos = 0;
+    for (int t = 0; t < n_tensors; ++t) {
+        if (tensor_offsets) tensor_offsets[t] = pos;
+        pos += round_up(numel[t], OB_TENSOR_ALIGN);
+    }
+    *n_padded = pos;
+    return OB_OK;
+}
+
+ob_status ob_chunk_range(int64_t numel, int W, int j, int64_t *begin, int64_t *end) {
+    if (numel < 0 || W < 1 || W > OB_MAX_WORKERS || j < 0 || j >= W || !begin || !end)
+        return OB_ERR_INVALID_ARG;
+    chunk_bounds(numel, W, j, begin, end);
+    return OB_OK;
+}
+
+ob_status ob_workspace_bytes(int n_tensors, const int64_t *numel, int W, size_t *bytes) {
+    if (!bytes) return OB_ERR_INVALID_ARG;
+    try {
+        Plan pl;
+        ob_status st = make_plan(n_tensors, numel, W, true, &pl);
+        if (st != OB_OK) return st;
+        *bytes = carve(pl).total;
+        return OB_OK;
+    } catch (const std::bad_alloc &) {
+        return OB_ERR_OOM;
+    }
+}
+
+ob_status ob_create(int n_tensors, const int64_t *numel, int W, float beta1, float beta2,
+                    float eps, float lr, float *d_params, void *d_workspace,
+                    size_t workspace_bytes, void *cuda_stream, ob_ctx **out) {
+    if (!out) return OB_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!d_workspace) return OB_ERR_INVALID_ARG;
+    if (!(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps > 0.f) ||
+        !std::isfinite(lr) || !std::isfinite(eps))
+        return OB_ERR_INVALID_ARG;
+    if (!aligned(d_params, 16) || !aligned(d_workspace, kWsAlign)) return OB_ERR_ALIGN;
+    ob_ctx *c = nullptr;
+    try {
+        host_alloc_point();
+        c = new ob_ctx();
+        ob_status st = make_plan(n_tensors, numel, W, true, &c->plan);
+        if (st != OB_OK) {
+            delete c;
+            return st;
+        }
+        if (!d_params && c->plan.n_pad > 0) {  // NULL only for an all-empty list
+            delete c;
+            return OB_ERR_INVALID_ARG;
+        }
+        c->cv = carve(c->plan);
+        if (workspace_bytes < c->cv.total) {
+            delete c;
+            return OB_ERR_WORKSPACE;
+        }
+        c->host_runs = make_runs(c->plan.tiles, kHostSlice);
+    } catch (const std::bad_alloc &) {
+        delete c;
+        return OB_ERR_OOM;
+    }
+    c->beta1 = beta1;
+    c->beta2 = beta2;
+    c->eps = eps;
+    c->lr = lr;
+    c->c1 = 1.0f - beta1;
+    c->c2 = 1.0f - beta2;
+    c->params = d_params;
+    c->ws = static_cast<char *>(d_workspace);
+    c->stream = static_cast<cudaStream_t>(cuda_stream);
+    auto bail = [&](cudaError_t e) {
+        if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
+        for (auto &ev : c->ev_copied) if (ev) cudaEventDestroy(ev);
+        for (auto &ev : c->ev_consumed) if (ev) cudaEventDestroy(ev);
+        if (c->ev_start) cudaEventDestroy(c->ev_start);
+        delete c;
+        (void)e;
+        return OB_ERR_CUDA;
+    };
+    cudaError_t e = cudaGetDevice(&c->device);
+    if (e != cudaSuccess) return bail(e);
+    e = cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return bail(e);
+    for (int k = 0; k < 2 && e == cudaSuccess; ++k) {
+        e = cudaEventCreateWithFlags(&c->ev_copied[k], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_consumed[k], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_start, cudaEventDisableTiming);
+    if (e != cudaSuccess) return bail(e);
+    // zero the state, upload the work list
+    const Plan &pl = c->plan;
+    e = cudaMemsetAsync(c->ws, 0, c->cv.tiles, c->stream);
+    if (e == cudaSuccess && !pl.tiles.empty())
+        e = cudaMemcpyAsync(c->tiles(), pl.tiles.data(), pl.tiles.size() * sizeof(Tile),
+                            cudaMemcpyHostToDevice, c->stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(c->tensor_tile_begin(), pl.tensor_tile_begin.data(),
+                            pl.tensor_tile_begin.size() * 4, cudaMemcpyHostToDevice, c->stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(c->chunk_tile_begin(), pl.chunk_tile_begin.data(),
+                            pl.chunk_tile_begin.size() * 4, cudaMemcpyHostToDevice, c->stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(c->numel(), pl.numel.data(), pl.numel.size() * 8, cudaMemcpyHostToDevice,
+                            c->stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(c->chunk_len(), pl.chunk_len.data(), pl.chunk_len.size() * 8,
+                            cudaMemcpyHostToDevice, c->stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
+    if (e != cudaSuccess) return bail(e);
+    {
+        std::lock_guard<std::mutex> lk(g_live_mu);
+        try {
+            g_live.insert(c);
+        } catch (const std::bad_alloc &) {
+            return bail(cudaSuccess), OB_ERR_OOM;
+        }
+    }
+    *out = c;
+    return OB_OK;
+}
+
+void ob_destroy(ob_ctx *c) {
+    {
+        std::lock_guard<std::mutex> lk(g_live_mu);
+        if (!c || g_live.erase(c) == 0) return;
+    }
+    DeviceGuard dg(c->device);
+    cudaStreamSynchronize(c->stream);
+    cudaStreamSynchronize(c->copy_stream);
+    for (auto &p : c->pending) {
+        cudaEventDestroy(p.second.first);
+        cudaEventDestroy(p.second.second);
+    }
+    for (cudaEvent_t e : c->event_pool) cudaEventDestroy(e);
+    for (auto &ev : c->ev_copied) cudaEventDestroy(ev);
+    for (auto &ev : c->ev_consumed) cudaEventDestroy(ev);
+    cudaEventDestroy(c->ev_start);
+    cudaStreamDestroy(c->copy_stream);
+    c->magic = 0;
+    delete c;
+}
+
+ob_status ob_warmup_adam_step(ob_ctx *c, const float *const *d_grads) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (c->frozen) return OB_ERR_PHASE;
+    if ((st = check_grads(c, d_grads)) != OB_OK) return st;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    const int64_t t = c->t_warmup + 1;
+    onebit::WarmupParams P;
+    P.tiles = c->tiles();
+    for (int w = 0; w < OB_MAX_WORKERS; ++w) P.g[w] = w < c->plan.W ? d_grads[w] : nullptr;
+    P.m = c->m();
+    P.v = c->v();
+    P.p = c->params;
+    P.W = c->plan.W;
+    P.beta1 = c->beta1;
+    P.beta2 = c->beta2;
+    P.c1 = c->c1;
+    P.c2 = c->c2;
+    P.bc1 = (float)(1.0 - std::pow((double)c->beta1, (double)t));
+    P.bc2 = (float)(1.0 - std::pow((double)c->beta2, (double)t));
+    P.eps = c->eps;
+    P.lr = c->lr;
+    if (c->n_tiles() > 0) {
+        KernelTimer k(c, OB_K_WARMUP);
+        onebit::ob_warmup_kernel<<<grid1(c->n_tiles()), kThreads, 0, c->stream>>>(P);
+        k.stop();
+        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
+    }
+    c->t_warmup = t;
+    return OB_OK;
+}
+
+ob_status ob_freeze_variance(ob_ctx *c) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (c->frozen || c->t_warmup < 1) return OB_ERR_PHASE;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    const float bc2 = (float)(1.0 - std::pow((double)c->beta2, (double)c->t_warmup));
+    if (c->n_tiles() > 0) {
+        KernelTimer k(c, OB_K_FREEZE);
+        onebit::ob_freeze_kernel<<<grid1(c->n_tiles()), kThreads, 0, c->stream>>>(c->tiles(), c->v(),
+                                                                               bc2, c->eps);
+        k.stop();
+        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
+    }
+    // e_w = 0 and e_s = 0: zero the lazy values and their scales; clear the
+    // last step's words and scales.
+    const Carve &cv = c->cv;
+    cudaError_t e = cudaMemsetAsync(c->x(), 0, cv.bits - cv.x, c->stream);  // x, y
+    if (e == cudaSuccess) e = cudaMemsetAsync(c->bits(), 0, cv.partial_w - cv.bits, c->stream);
+    if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    c->frozen = true;
+    return OB_OK;
+}
+
+ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!c->frozen) return OB_ERR_PHASE;
+    if ((st = check_grads(c, d_grads)) != OB_OK) return st;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    KernelTimer pack(c, OB_K_PACK);
+    if ((st = launch_pack(c, d_grads, 0, 0, c->n_tiles())) != OB_OK) return st;
+    if ((st = launch_after_pack(c, pack)) != OB_OK) return st;
+    c->t_compressed += 1;
+    return OB_OK;
+}
+
+ob_status ob_host_staging_bytes(const ob_ctx *c, size_t *bytes) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!bytes) return OB_ERR_INVALID_ARG;
+    *bytes = (size_t)2 * c->plan.W * kHostSlice * sizeof(float);
+    return OB_OK;
+}
+
+ob_status ob_compressed_step_host(ob_ctx *c, const float *const *h_grads, void *d_staging,
+                                  size_t staging_bytes, float *h_server_scales) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!c->frozen) return OB_ERR_PHASE;
+    if (!h_grads || !d_staging) return OB_ERR_INVALID_ARG;
+    for (int w = 0; w < c->plan.W; ++w)
+        if (!h_grads[w]) return OB_ERR_INVALID_ARG;
+    if (!aligned(d_staging, kWsAlign)) return OB_ERR_ALIGN;
+    const int W = c->plan.W;
+    if (staging_bytes < (size_t)2 * W * kHostSlice * sizeof(float)) return OB_ERR_WORKSPACE;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    float *stage = static_cast<float *>(d_staging);
+    // The copy stream must not overwrite staging still read by earlier work.
+    cudaError_t e = cudaEventRecord(c->ev_start, c->stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(c->copy_stream, c->ev_start, 0);
+    if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    KernelTimer pack(c, OB_K_PACK);
+    const float *g[OB_MAX_WORKERS];
+    for (size_t r = 0; r < c->host_runs.size(); ++r) {
+        const Run &run = c->host_runs[r];
+        const int slot = (int)(r & 1);
+        if (r >= 2) e = cudaStreamWaitEvent(c->copy_stream, c->ev_consumed[slot], 0);
+        const size_t bytes = (size_t)(run.elem_hi - run.elem_lo) * sizeof(float);
+        for (int w = 0; w < W && e == cudaSuccess; ++w) {
+            float *dst = stage + ((size_t)slot * W + w) * kHostSlice;
+            e = cudaMemcpyAsync(dst, h_grads[w] + run.elem_lo, bytes, cudaMemcpyHostToDevice,
+                                c->copy_stream);
+            g[w] = dst;
+        }
+        if (e == cudaSuccess) e = cudaEventRecord(c->ev_copied[slot], c->copy_stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(c->stream, c->ev_copied[slot], 0);
+        if ((st = fail_cuda(c, e)) != OB_OK) return st;
+        if ((st = launch_pack(c, g, run.elem_lo, run.tile_lo, run.tile_hi)) != OB_OK) return st;
+        if ((st = fail_cuda(c, cudaEventRecord(c->ev_consumed[slot], c->stream))) != OB_OK) return st;
+    }
+    if ((st = launch_after_pack(c, pack)) != OB_OK) return st;
+    c->t_compressed += 1;
+    if (h_server_scales)
+        e = cudaMemcpyAsync(h_server_scales, c->sp_last(),
+                            (size_t)c->plan.T * W * sizeof(float), cudaMemcpyDeviceToHost, c->stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
+    return fail_cuda(c, e);
+}
+
+ob_status ob_read_state(ob_ctx *c, int kind, int index, void *host_dst, size_t bytes) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!host_dst) return OB_ERR_INVALID_ARG;
+    const size_t want = state_bytes(c, kind);
+    if (want == 0 || bytes != want) return OB_ERR_INVALID_ARG;
+    const bool indexed = kind == OB_STATE_E_WORKER || kind == OB_STATE_BITS_WORKER;
+    if (indexed ? (index < 0 || index >= c->plan.W) : index != 0) return OB_ERR_INVALID_ARG;
+    if (kind == OB_STATE_V && c->frozen) return OB_ERR_PHASE;
+    if (kind == OB_STATE_D && !c->frozen) return OB_ERR_PHASE;
+    if (kind == OB_STATE_STEP) {
+        const int64_t v[3] = {c->t_warmup, c->t_compressed, c->frozen ? 1 : 0};
+        std::memcpy(host_dst, v, sizeof(v));
+        return OB_OK;
+    }
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    if ((st = fail_cuda(c, cudaStreamSynchronize(c->stream))) != OB_OK) return st;
+    const size_t n = (size_t)c->plan.n_pad;
+    try {
+        if (kind == OB_STATE_E_WORKER)
+            return read_error(c, c->x() + (size_t)index * n, c->s_prev() + (size_t)index * c->plan.T,
+                              1, 0, static_cast<float *>(host_dst));
+        if (kind == OB_STATE_E_SERVER)
+            return read_error(c, c->y(), c->sp_prev(), c->plan.W, 1, static_cast<float *>(host_dst));
+    } catch (const std::bad_alloc &) {
+        return OB_ERR_OOM;
+    }
+    const void *src = nullptr;
+    switch (kind) {
+    case OB_STATE_P: src = c->params; break;
+    case OB_STATE_M: src = c->m(); break;
+    case OB_STATE_V: case OB_STATE_D: src = c->v(); break;
+    case OB_STATE_S_WORKER: src = c->s_last(); break;
+    case OB_STATE_S_SERVER: src = c->sp_last(); break;
+    case OB_STATE_BITS_WORKER: src = c->bits() + (size_t)index * (n / 32); break;
+    case OB_STATE_BITS_SERVER: src = c->sbits(); break;
+    default: return OB_ERR_INVALID_ARG;
+    }
+    cudaError_t e = cudaMemcpyAsync(host_dst, src, bytes, cudaMemcpyDeviceToHost, c->stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
+    return fail_cuda(c, e);
+}
+
+ob_status ob_write_state(ob_ctx *c, int kind, int index, const void *host_src, size_t bytes) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!host_src) return OB_ERR_INVALID_ARG;
+    const size_t want = state_bytes(c, kind);
+    if (want == 0 || bytes != want) return OB_ERR_INVALID_ARG;
+    const bool indexed = kind == OB_STATE_E_WORKER;
+    if (indexed ? (index < 0 || index >= c->plan.W) : index != 0) return OB_ERR_INVALID_ARG;
+    if (kind == OB_STATE_V && c->frozen) return OB_ERR_PHASE;
+    if (kind == OB_STATE_D && !c->frozen) return OB_ERR_PHASE;
+    if (kind == OB_STATE_STEP) {
+        int64_t v[3];
+        std::memcpy(v, host_src, sizeof(v));
+        if (v[0] < 0 || v[1] < 0 || (v[2] != 0 && v[2] != 1) || (v[2] == 1 && v[0] < 1) ||
+            (v[2] == 0 && v[1] != 0))
+            return OB_ERR_INVALID_ARG;
+        c->t_warmup = v[0];
+        c->t_compressed = v[1];
+        c->frozen = v[2] == 1;
+        return OB_OK;
+    }
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    const size_t n = (size_t)c->plan.n_pad;
+    void *dst = nullptr;
+    cudaError_t e = cudaSuccess;
+    switch (kind) {
+    case OB_STATE_P: dst = c->params; break;
+    case OB_STATE_M: dst = c->m(); break;
+    case OB_STATE_V: case OB_STATE_D: dst = c->v(); break;
+    case OB_STATE_E_WORKER:
+        // stored as (x, s) with s = 0, which decodes to x exactly
+        dst = c->x() + (size_t)index * n;
+        e = cudaMemsetAsync(c->s_prev() + (size_t)index * c->plan.T, 0, (size_t)c->plan.T * 4,
+                            c->stream);
+        break;
+    case OB_STATE_E_SERVER:
+        dst = c->y();
+        e = cudaMemsetAsync(c->sp_prev(), 0, (size_t)c->plan.T * c->plan.W * 4, c->stream);
+        break;
+    default:
+        return OB_ERR_INVALID_ARG;
+    }
+    if (e == cudaSuccess) e = cudaMemcpyAsync(dst, host_src, bytes, cudaMemcpyHostToDevice, c->stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
+    return fail_cuda(c, e);
+}
+
+ob_status ob_profile_enable(ob_ctx *c, int on) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    c->profiling = on != 0;
+    return OB_OK;
+}
+
+ob_status ob_profile_read(ob_ctx *c, double *ms, int64_t *launches, int reset) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    if ((st = fail_cuda(c, cudaStreamSynchronize(c->stream))) != OB_OK) return st;
+    for (auto &p : c->pending) {
+        float t = 0.f;
+        cudaError_t e = cudaEventElapsedTime(&t, p.second.first, p.second.second);
+        if (e != cudaSuccess) return fail_cuda(c, e);
+        c->kernel_ms[p.first] += t;
+        c->kernel_launches[p.first] += 1;
+        c->event_pool.push_back(p.second.first);
+        c->event_pool.push_back(p.second.second);
+    }
+    c->pending.clear();
+    for (int k = 0; k < OB_NUM_KERNELS; ++k) {
+        if (ms) ms[k] = c->kernel_ms[k];
+        if (launches) launches[k] = c->kernel_launches[k];
+        if (reset) {
+            c->kernel_ms[k] = 0;
+            c->kernel_launches[k] = 0;
+        }
+    }
+    return OB_OK;
+}
+
+}  // extern "C"

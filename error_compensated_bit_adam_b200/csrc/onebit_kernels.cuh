@@ -1,0 +1,475 @@
+// onebit_kernels.cuh -- device code of libonebit (sm_100a).
+//
+// The compression-phase step of 1-bit Adam ("1-bit Adam: Communication
+// Efficient Large-Scale Training with Adam's Convergence Speed", review
+// page, sections "Abstract" and "Proposed method") as five HBM-streaming
+// kernels over a list of 4096-element tiles:
+//
+//   ob_pack_kernel          worker stage, all W workers of a tile per CTA
+//   ob_pack_scale_kernel    worker scales per (tensor, worker)
+//   ob_server_kernel        server stage of a tile
+//   ob_server_scale_kernel  server scales per (tensor, chunk)
+//   ob_apply_kernel         gather, decode, preconditioned update
+//
+// plus the warmup Adam step, the freeze and an error decoder used when the
+// host reads state.  No step is a dense contraction, so no tensor cores:
+// every kernel is a stream of coalesced 16-byte loads and stores, bound by
+// HBM bandwidth.
+//
+// Numerics.  Every fp32 operation is written with an explicit
+// round-to-nearest intrinsic (__fmul_rn, __fadd_rn, __fsub_rn, __fdiv_rn,
+// __fsqrt_rn), so nvcc cannot contract a*b+c into an FMA, and the order of
+// operations is the method's: the results are the same IEEE binary32
+// values a plain sequential CPU evaluation gives.  Sums of squares for the
+// scales are taken in fp64 in a fixed order (per thread, warp butterfly,
+// warps in order, tiles in order), so results repeat run to run.
+//
+// Lazy error buffers.  e_w = x - sign(x) s_w needs s_w, which needs all of
+// x.  Rather than a second pass over x, the worker error is stored as the
+// pair (x, s_w) and decoded where it is next used:
+//   e_w = fl(x - sign(x) s_w)   -- the same rounding an eager pass would do.
+// The server error is stored the same way as (y, s'_j).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/onebit.h"
+
+namespace onebit {
+
+constexpr int kThreads = 256;              // threads per CTA of the tile kernels
+constexpr int kWarps = kThreads / 32;
+constexpr int kUnroll = 4;                 // float4 slots per thread per tile
+constexpr int kTile = kThreads * 4 * kUnroll;  // 4096 elements per tile
+constexpr int kScaleThreads = 256;         // threads of the scale kernels
+constexpr unsigned kFull = 0xffffffffu;
+
+// One unit of work: up to kTile consecutive elements of one tensor that all
+// belong to one server chunk.  begin is the padded-layout element offset of
+// the tile's first element (a multiple of 128); count is the number of real
+// (non-padding) elements.
+struct Tile {
+    int64_t begin;
+    int32_t count;
+    int32_t tensor;
+    int32_t chunk;
+    int32_t reserved;
+};
+static_assert(sizeof(Tile) == 24, "Tile layout");
+
+// ---------------------------------------------------------------- helpers
+
+__device__ __forceinline__ float signed_scale(bool plus, float s) { return plus ? s : -s; }
+
+// The 1-bit code: +1 for x >= 0 (so +0.0 and -0.0 give +1), else -1.
+__device__ __forceinline__ bool code_of(float x) { return x >= 0.0f; }
+
+// Error feedback stored lazily as (x, s): e = fl(x - sign(x) s).
+__device__ __forceinline__ float decode_error(float x, float s) {
+    return __fsub_rn(x, signed_scale(code_of(x), s));
+}
+
+__device__ __forceinline__ float get(const float4 &v, int k) {
+    return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
+}
+__device__ __forceinline__ void set(float4 &v, int k, float f) {
+    if (k == 0) v.x = f; else if (k == 1) v.y = f; else if (k == 2) v.z = f; else v.w = f;
+}
+
+// Streaming 16-byte accesses: every byte is touched once per step, so mark
+// the lines evict-first and keep L2 for the packed words and scales.
+__device__ __forceinline__ float4 ld_stream(const float *p) {
+    return __ldcs(reinterpret_cast<const float4 *>(p));
+}
+__device__ __forceinline__ void st_stream(float *p, const float4 &v) {
+    __stcs(reinterpret_cast<float4 *>(p), v);
+}
+
+// OR together the 4-bit groups of the 8 lanes that share one 32-bit sign
+// word.  Lane l holds elements 4l..4l+3 of the warp's 128-element slot, so
+// its nibble goes to bits 4*(l%8)..4*(l%8)+3 of word l/8.  Every lane of
+// the group ends with the whole word.
+__device__ __forceinline__ uint32_t gather_word(uint32_t nibble, int lane) {
+    uint32_t v = nibble << (4 * (lane & 7));
+    v |= __shfl_xor_sync(kFull, v, 1);
+    v |= __shfl_xor_sync(kFull, v, 2);
+    v |= __shfl_xor_sync(kFull, v, 4);
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+// Fixed-order fp64 sum over a CTA of kScaleThreads threads (result valid in
+// thread 0).
+__device__ __forceinline__ double block_sum(double v, double *smem) {
+    v = warp_sum(v);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) smem[warp] = v;
+    __syncthreads();
+    double acc = 0.0;
+    if (threadIdx.x == 0)
+        for (int k = 0; k < kScaleThreads / 32; ++k) acc += smem[k];
+    return acc;
+}
+
+// Real elements (0..4) of the float4 slot at tile offset off.
+__device__ __forceinline__ int slot_real(int count, int off) { return min(4, max(0, count - off)); }
+
+// ------------------------------------------------------------ warmup Adam
+
+struct WarmupParams {
+    const Tile *tiles;
+    const float *g[OB_MAX_WORKERS];  // worker gradients, padded layout
+    float *m, *v, *p;
+    int W;
+    float beta1, beta2, c1, c2, bc1, bc2, eps, lr;
+};
+
+// [1BA, Proposed method, 1]: one full-precision Adam step on the averaged
+// gradient, elementwise.
+__global__ void __launch_bounds__(kThreads) ob_warmup_kernel(const __grid_constant__ WarmupParams P) {
+    const Tile tile = P.tiles[blockIdx.x];
+    const float wf = (float)P.W;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * ((int)threadIdx.x + kThreads * u);
+        const int real = slot_real(tile.count, off);
+        if (real == 0) continue;
+        const int64_t i = tile.begin + off;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int w = 0; w < P.W; ++w) {
+            const float4 g = ld_stream(P.g[w] + i);
+            acc.x = __fadd_rn(acc.x, g.x);
+            acc.y = __fadd_rn(acc.y, g.y);
+            acc.z = __fadd_rn(acc.z, g.z);
+            acc.w = __fadd_rn(acc.w, g.w);
+        }
+        float4 m = ld_stream(P.m + i), v = ld_stream(P.v + i), p = ld_stream(P.p + i);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (k >= real) break;  // padding keeps its values
+            const float gbar = __fdiv_rn(get(acc, k), wf);
+            const float mk = __fadd_rn(__fmul_rn(P.beta1, get(m, k)), __fmul_rn(P.c1, gbar));
+            const float vk = __fadd_rn(__fmul_rn(P.beta2, get(v, k)),
+                                       __fmul_rn(P.c2, __fmul_rn(gbar, gbar)));
+            const float mhat = __fdiv_rn(mk, P.bc1);
+            const float vhat = __fdiv_rn(vk, P.bc2);
+            const float denom = __fadd_rn(__fsqrt_rn(vhat), P.eps);
+            const float delta = __fmul_rn(P.lr, __fdiv_rn(mhat, denom));
+            set(m, k, mk);
+            set(v, k, vk);
+            set(p, k, __fsub_rn(get(p, k), delta));
+        }
+        st_stream(P.m + i, m);
+        st_stream(P.v + i, v);
+        st_stream(P.p + i, p);
+    }
+}
+
+// ----------------------------------------------------------------- freeze
+
+// [1BA, Abstract; Proposed method, 2]: d = sqrt(v / bc2) + eps, in place.
+__global__ void __launch_bounds__(kThreads) ob_freeze_kernel(const Tile *tiles, float *v, float bc2,
+                                                             float eps) {
+    const Tile tile = tiles[blockIdx.x];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * ((int)threadIdx.x + kThreads * u);
+        const int real = slot_real(tile.count, off);
+        if (real == 0) continue;
+        float4 x = ld_stream(v + tile.begin + off);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (k < real) set(x, k, __fadd_rn(__fsqrt_rn(__fdiv_rn(get(x, k), bc2)), eps));
+        st_stream(v + tile.begin + off, x);
+    }
+}
+
+// ----------------------------------------------------------- worker stage
+
+struct PackParams {
+    const Tile *tiles;
+    int tile_base;                   // tile of blockIdx.x == 0
+    int n_tiles;                     // total tiles (row length of partial)
+    const float *m;                  // [n_pad]
+    const float *g[OB_MAX_WORKERS];  // element i of worker w at g[w][i - g_offset]
+    int64_t g_offset;
+    float *x;                        // [W][n_pad]: in x_prev (lazy e_w), out x
+    uint32_t *bits;                  // [W][n_pad/32]
+    const float *s_prev;             // [W][T]: scale that decodes x_prev
+    double *partial;                 // [W][n_tiles]: sum of x^2 per tile
+    int64_t n_pad;
+    int W, T;
+    float beta1, c1;
+};
+
+// [1BA, Proposed method, 3; Abstract]: for every worker w of one tile,
+//   m_w = beta1 m + (1-beta1) g_w,  x = m_w + e_w (e_w decoded from the
+//   stored (x_prev, s_prev)), sign bits of x, partial sum of x^2.
+// x overwrites x_prev: with this step's scale it encodes the new e_w.
+// m stays in registers across the W workers, so it is read once.
+__global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant__ PackParams P) {
+    const int tile_id = P.tile_base + (int)blockIdx.x;
+    const Tile tile = P.tiles[tile_id];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ double red[kWarps][OB_MAX_WORKERS];
+
+    float4 mv[kUnroll];
+    int real[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * (tid + kThreads * u);
+        real[u] = slot_real(tile.count, off);
+        mv[u] = real[u] > 0 ? ld_stream(P.m + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const int64_t words_per_worker = P.n_pad >> 5;
+    for (int w = 0; w < P.W; ++w) {
+        const float s_prev = P.s_prev[w * P.T + tile.tensor];
+        const float *gw = P.g[w] + (tile.begin - P.g_offset);
+        float *xw = P.x + (int64_t)w * P.n_pad + tile.begin;
+        uint32_t *bw = P.bits + (int64_t)w * words_per_worker + (tile.begin >> 5);
+        double ss = 0.0;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int off = 4 * (tid + kThreads * u);
+            uint32_t nibble = 0;
+            if (real[u] > 0) {
+                const float4 g = ld_stream(gw + off);
+                const float4 xp = ld_stream(xw + off);
+                float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    if (k < real[u]) {
+                        const float m_w = __fadd_rn(__fmul_rn(P.beta1, get(mv[u], k)),
+                                                    __fmul_rn(P.c1, get(g, k)));
+                        const float x = __fadd_rn(m_w, decode_error(get(xp, k), s_prev));
+                        ss = __fma_rn((double)x, (double)x, ss);
+                        nibble |= (uint32_t)code_of(x) << k;
+                        set(xo, k, x);
+                    }
+                }
+                st_stream(xw + off, xo);
+            }
+            const uint32_t word = gather_word(nibble, lane);
+            if ((lane & 7) == 0 && off < tile.count) bw[(tid + kThreads * u) >> 3] = word;
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) red[warp][w] = ss;
+    }
+    __syncthreads();
+    if (tid < P.W) {
+        double acc = 0.0;
+#pragma unroll
+        for (int k = 0; k < kWarps; ++k) acc += red[k][tid];
+        P.partial[(int64_t)tid * P.n_tiles + tile_id] = acc;
+    }
+}
+
+// Worker scale of (tensor t = blockIdx.x, worker w = blockIdx.y):
+// s = ||x||_2 / sqrt(numel_t) from the tile partial sums (tiles in order).
+__global__ void __launch_bounds__(kScaleThreads) ob_pack_scale_kernel(
+    const double *partial, int n_tiles, const int *tensor_tile_begin, const int64_t *numel, int T,
+    float *s_prev, float *s_last) {
+    __shared__ double smem[kScaleThreads / 32];
+    const int t = blockIdx.x, w = blockIdx.y;
+    const int lo = tensor_tile_begin[t], hi = tensor_tile_begin[t + 1];
+    const double *row = partial + (int64_t)w * n_tiles;
+    double acc = 0.0;
+    for (int k = lo + (int)threadIdx.x; k < hi; k += kScaleThreads) acc += row[k];
+    acc = block_sum(acc, smem);
+    if (threadIdx.x == 0) {
+        const int64_t n = numel[t];
+        const float s = n > 0 ? __double2float_rn(__dsqrt_rn(__ddiv_rn(acc, (double)n))) : 0.0f;
+        s_prev[w * T + t] = s;
+        s_last[w * T + t] = s;
+    }
+}
+
+// ----------------------------------------------------------- server stage
+
+struct ServerParams {
+    const Tile *tiles;
+    const uint32_t *bits;   // [W][n_pad/32] this step's worker signs
+    const float *s_w;       // [W][T] this step's worker scales
+    float *y;               // [n_pad]: in y_prev (lazy e_s), out y
+    const float *sp_prev;   // [T][W]: scale that decodes y_prev
+    uint32_t *sbits;        // [n_pad/32]
+    double *partial;        // [n_tiles]: sum of y^2 per tile
+    int64_t n_pad;
+    int W, T;
+};
+
+// [1BA, Proposed method, 3-4]: server j = tile.chunk receives every
+// worker's words for its chunk (addressed in place: the exchange is an
+// index into [W][words]) and forms
+//   y = (sum over w in order of sign_w s_w) / W + e_s,
+// with e_s decoded from (y_prev, s'_prev); then the sign bits of y and the
+// tile's partial sum of y^2.
+__global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_constant__ ServerParams P) {
+    const int tile_id = blockIdx.x;
+    const Tile tile = P.tiles[tile_id];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ double red[kWarps];
+    const int64_t words_per_worker = P.n_pad >> 5;
+    const int64_t word0 = tile.begin >> 5;
+    const int shift = 4 * (lane & 7);  // bit of this lane's first element in its word
+
+    float acc[kUnroll][4];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[u][k] = 0.0f;
+
+    for (int w = 0; w < P.W; ++w) {
+        const float s = P.s_w[w * P.T + tile.tensor];
+        const uint32_t *bw = P.bits + (int64_t)w * words_per_worker + word0;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int off = 4 * (tid + kThreads * u);
+            if (off < tile.count) {
+                const uint32_t word = __ldg(bw + ((tid + kThreads * u) >> 3)) >> shift;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    acc[u][k] = __fadd_rn(acc[u][k], signed_scale((word >> k) & 1u, s));
+            }
+        }
+    }
+
+    const float wf = (float)P.W;
+    const float sp = P.sp_prev[tile.tensor * P.W + tile.chunk];
+    double ss = 0.0;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * (tid + kThreads * u);
+        const int real = slot_real(tile.count, off);
+        uint32_t nibble = 0;
+        if (real > 0) {
+            float *yp = P.y + tile.begin + off;
+            const float4 yo = ld_stream(yp);
+            float4 yn = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                if (k < real) {
+                    const float avg = __fdiv_rn(acc[u][k], wf);
+                    const float y = __fadd_rn(avg, decode_error(get(yo, k), sp));
+                    ss = __fma_rn((double)y, (double)y, ss);
+                    nibble |= (uint32_t)code_of(y) << k;
+                    set(yn, k, y);
+                }
+            }
+            st_stream(yp, yn);
+        }
+        const uint32_t word = gather_word(nibble, lane);
+        if ((lane & 7) == 0 && off < tile.count) P.sbits[word0 + ((tid + kThreads * u) >> 3)] = word;
+    }
+    ss = warp_sum(ss);
+    if (lane == 0) red[warp] = ss;
+    __syncthreads();
+    if (tid == 0) {
+        double a = 0.0;
+#pragma unroll
+        for (int k = 0; k < kWarps; ++k) a += red[k];
+        P.partial[tile_id] = a;
+    }
+}
+
+// Server scale of chunk c = blockIdx.x (tensor c / W, server c % W):
+// s' = ||y over the chunk||_2 / sqrt(len), 0 for an empty chunk.
+__global__ void __launch_bounds__(kScaleThreads) ob_server_scale_kernel(
+    const double *partial, const int *chunk_tile_begin, const int64_t *chunk_len, float *sp_prev,
+    float *sp_last) {
+    __shared__ double smem[kScaleThreads / 32];
+    const int c = blockIdx.x;
+    const int lo = chunk_tile_begin[c], hi = chunk_tile_begin[c + 1];
+    double acc = 0.0;
+    for (int k = lo + (int)threadIdx.x; k < hi; k += kScaleThreads) acc += partial[k];
+    acc = block_sum(acc, smem);
+    if (threadIdx.x == 0) {
+        const int64_t len = chunk_len[c];
+        const float s = len > 0 ? __double2float_rn(__dsqrt_rn(__ddiv_rn(acc, (double)len))) : 0.0f;
+        sp_prev[c] = s;
+        sp_last[c] = s;
+    }
+}
+
+// ------------------------------------------------------ gather and update
+
+struct ApplyParams {
+    const Tile *tiles;
+    const uint32_t *sbits;  // [n_pad/32]
+    const float *sp;        // [T][W] this step's server scales
+    const float *d;         // [n_pad] frozen denominator
+    float *p;               // [n_pad]
+    float *m;               // [n_pad]
+    int W;
+    float lr;
+};
+
+// [1BA, Proposed method, 1-2]: every worker decodes the gathered server
+// words, m_hat = sign' s'_j, and takes a momentum SGD step preconditioned by
+// the frozen denominator: p -= lr (m_hat / d); m = m_hat.
+__global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constant__ ApplyParams P) {
+    const Tile tile = P.tiles[blockIdx.x];
+    const int tid = threadIdx.x, lane = tid & 31;
+    const float s = P.sp[tile.tensor * P.W + tile.chunk];
+    const int shift = 4 * (lane & 7);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * (tid + kThreads * u);
+        const int real = slot_real(tile.count, off);
+        if (real == 0) continue;
+        const int64_t i = tile.begin + off;
+        const uint32_t word = __ldg(P.sbits + (i >> 5)) >> shift;
+        const float4 d = ld_stream(P.d + i);
+        float4 p = ld_stream(P.p + i);
+        float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (k < real) {
+                const float m_hat = signed_scale((word >> k) & 1u, s);
+                const float delta = __fmul_rn(P.lr, __fdiv_rn(m_hat, get(d, k)));
+                set(p, k, __fsub_rn(get(p, k), delta));
+                set(m, k, m_hat);
+            }
+        }
+        st_stream(P.p + i, p);
+        st_stream(P.m + i, m);
+    }
+}
+
+// ------------------------------------------------- state decode for reads
+
+struct DecodeParams {
+    const Tile *tiles;
+    int tile_base;
+    const float *x;        // [n_pad] lazy error values (x or y)
+    const float *scales;   // scale of tile (t, j) at scales[t * stride_t + j * stride_j]
+    int stride_t, stride_j;
+    float *out;            // out[i - out_base] = decoded error
+    int64_t out_base;
+};
+
+// e = fl(x - sign(x) s) over a run of tiles (padding left untouched).
+__global__ void __launch_bounds__(kThreads) ob_decode_error_kernel(const __grid_constant__ DecodeParams P) {
+    const Tile tile = P.tiles[P.tile_base + (int)blockIdx.x];
+    const float s = P.scales[tile.tensor * P.stride_t + tile.chunk * P.stride_j];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * ((int)threadIdx.x + kThreads * u);
+        const int real = slot_real(tile.count, off);
+        if (real == 0) continue;
+        const float4 x = ld_stream(P.x + tile.begin + off);
+        float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (k < real) set(e, k, decode_error(get(x, k), s));
+        *reinterpret_cast<float4 *>(P.out + (tile.begin + off - P.out_base)) = e;
+    }
+}
+
+}  // namespace onebit

@@ -1,0 +1,238 @@
+/*
+ * onebit.h -- C ABI of libonebit: the compression-phase step of 1-bit Adam
+ * on one NVIDIA B200 (sm_100a), with W data-parallel workers simulated as W
+ * state buffers in the GPU's HBM.
+ *
+ * The method is the one on the review page "1-bit Adam: Communication
+ * Efficient Large-Scale Training with Adam's Convergence Speed" ([1BA]):
+ *   - [1BA, Proposed method, 1]: training runs full-precision Adam for a
+ *     warmup (typically 20% of the steps), then 1-bit compressed momentum
+ *     SGD for the rest;
+ *   - [1BA, Abstract; Proposed method, 2]: Adam's variance is stable after
+ *     the warmup and is frozen, becoming the fixed preconditioner;
+ *   - [1BA, Proposed method, 3]: error-compensated 1-bit compression is
+ *     applied to the momentum;
+ *   - [1BA, Proposed method, 4]: a custom compressed collective (a worker
+ *     stage and a server stage) averages the compressed momentum.
+ * The calls below follow that two-phase statement:
+ *   ob_create -> ob_warmup_adam_step* -> ob_freeze_variance ->
+ *   ob_compressed_step* (state machine enforced; OB_ERR_PHASE otherwise).
+ *
+ * Conventions shared by every call
+ *   - Every call returns an ob_status and never aborts, throws or exits.
+ *   - A "tensor list" is n_tensors >= 1 tensors of numel[t] >= 0 fp32
+ *     elements.  Each tensor is an independent problem: its own worker
+ *     scales, sign packing and server chunks.
+ *   - Padded layout: all flat per-parameter buffers (parameters, gradients,
+ *     dense state) hold the tensors back to back, tensor t starting at
+ *     element offset[t] (a multiple of OB_TENSOR_ALIGN), its numel[t]
+ *     elements followed by padding up to the next multiple of
+ *     OB_TENSOR_ALIGN.  n_padded is the total.  Padding entries are never
+ *     read into any result and never updated.  ob_layout gives offsets.
+ *   - Packed sign words (uint32): bit k of word i of tensor t is element
+ *     32*i + k of that tensor; tensor t's words start at word offset[t]/32;
+ *     bit 1 means +1 (x >= 0, so sign(0) = +1), bit 0 means -1; padding
+ *     bits are 0.
+ *   - Device pointers must be 16-byte aligned (OB_ERR_ALIGN otherwise); the
+ *     workspace 256-byte aligned.  libonebit never allocates or frees device
+ *     memory: the caller owns parameters, gradients and workspace.
+ *   - All GPU work is queued on the CUDA stream given to ob_create; the
+ *     step calls return once it is queued.  Launch errors are returned at
+ *     once; faults of queued work surface as OB_ERR_CUDA from the next call
+ *     that synchronizes (ob_read_state / ob_write_state /
+ *     ob_compressed_step_host / ob_profile_read).  After OB_ERR_CUDA a
+ *     context only accepts ob_destroy.
+ *   - A context is not thread-safe; use it from one host thread at a time.
+ *     Calls on a destroyed or unknown context return OB_ERR_INVALID_ARG.
+ */
+#ifndef ONEBIT_H
+#define ONEBIT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define OB_API __attribute__((visibility("default")))
+#else
+#define OB_API
+#endif
+
+#define OB_ABI_VERSION 1
+#define OB_MAX_WORKERS 64     /* W is 1..OB_MAX_WORKERS */
+#define OB_TENSOR_ALIGN 128   /* elements; tensor offsets are multiples of this */
+
+typedef struct ob_ctx ob_ctx; /* opaque */
+
+typedef enum ob_status {
+    OB_OK = 0,
+    OB_ERR_INVALID_ARG = 1,    /* bad count, size, index, kind or NULL pointer; unknown context */
+    OB_ERR_PHASE = 2,          /* call out of the warmup -> freeze -> compressed order */
+    OB_ERR_ALIGN = 3,          /* a device pointer is not 16-byte (workspace: 256-byte) aligned */
+    OB_ERR_WORKSPACE = 4,      /* workspace or staging buffer smaller than required */
+    OB_ERR_OOM = 5,            /* host memory allocation failed */
+    OB_ERR_CUDA = 6,           /* a CUDA call failed; the context is now unusable */
+    OB_ERR_DEVICE_TIMEOUT = 7  /* reserved: no kernel of this library waits on anything */
+} ob_status;
+
+/* Kinds of state for ob_read_state / ob_write_state. */
+typedef enum ob_state_kind {
+    OB_STATE_P = 0,           /* parameters p, float[n_padded] (the caller's buffer)           rw */
+    OB_STATE_M = 1,           /* momentum m, float[n_padded]                                    rw */
+    OB_STATE_V = 2,           /* Adam variance v, float[n_padded]; before the freeze only       rw */
+    OB_STATE_D = 3,           /* frozen denominator d = sqrt(v/bc2)+eps; after the freeze only  rw */
+    OB_STATE_E_WORKER = 4,    /* index w: worker w's error feedback e_w, float[n_padded]        rw */
+    OB_STATE_E_SERVER = 5,    /* server error feedback e_s, float[n_padded]                     rw */
+    OB_STATE_S_WORKER = 6,    /* last step's worker scales, float[W][n_tensors]                 r  */
+    OB_STATE_S_SERVER = 7,    /* last step's server chunk scales, float[n_tensors][W]           r  */
+    OB_STATE_BITS_WORKER = 8, /* index w: last step's packed worker signs, uint32[n_padded/32]  r  */
+    OB_STATE_BITS_SERVER = 9, /* last step's packed server signs, uint32[n_padded/32]           r  */
+    OB_STATE_STEP = 10        /* int64[3]: {warmup steps taken, compressed steps taken, frozen} rw */
+} ob_state_kind;
+
+/* Kernels timed by the profiling counters (ob_profile_read). */
+typedef enum ob_kernel_id {
+    OB_K_WARMUP = 0,          /* ob_warmup_adam_step */
+    OB_K_FREEZE = 1,          /* ob_freeze_variance */
+    OB_K_PACK = 2,            /* worker stage: momentum, error, signs, partial sums of squares */
+    OB_K_PACK_SCALE = 3,      /* worker scales from the partial sums */
+    OB_K_SERVER = 4,          /* server stage: average, server error, signs, partial sums */
+    OB_K_SERVER_SCALE = 5,    /* server chunk scales from the partial sums */
+    OB_K_APPLY = 6,           /* gather, decode and preconditioned update */
+    OB_NUM_KERNELS = 7
+} ob_kernel_id;
+
+/* Name of a status code (static string; never NULL). */
+OB_API const char *ob_status_string(ob_status status);
+
+/* OB_ABI_VERSION of the loaded library. */
+OB_API int ob_abi_version(void);
+
+/* Padded layout of a tensor list (host only, no GPU needed).
+ * numel: n_tensors counts (>= 0).  tensor_offsets (out, may be NULL):
+ * n_tensors element offsets.  n_padded (out): total padded elements.
+ * OB_ERR_INVALID_ARG for n_tensors < 1, a negative count, NULL numel or
+ * n_padded, or a total above 2^40 elements. */
+OB_API ob_status ob_layout(int n_tensors, const int64_t *numel, int64_t *tensor_offsets,
+                    int64_t *n_padded);
+
+/* Server j's chunk of a tensor of numel elements split among W servers
+ * (host only).  [1BA, Proposed method, 4]: with nw = ceil(numel/32) sign
+ * words, each server owns cw = roundup(ceil(nw/W), 4) words; server j owns
+ * elements [min(numel, 32*j*cw), min(numel, 32*(j+1)*cw)).  Chunks start on
+ * 128-element boundaries, so no sign word or 16-byte word group is split;
+ * trailing servers may own nothing.  OB_ERR_INVALID_ARG for numel < 0, W
+ * outside 1..OB_MAX_WORKERS, j outside 0..W-1 or NULL outputs. */
+OB_API ob_status ob_chunk_range(int64_t numel, int W, int j, int64_t *begin, int64_t *end);
+
+/* Bytes of device workspace ob_create needs for this tensor list and W
+ * (host only).  The workspace holds every piece of optimizer state except
+ * the parameters: m, v/d, the W worker error buffers, the server error,
+ * packed signs, scales, per-tile partial sums and the tile work list. */
+OB_API ob_status ob_workspace_bytes(int n_tensors, const int64_t *numel, int W, size_t *bytes);
+
+/* Create a context.  numel: as for ob_layout (copied).  W: simulated
+ * workers, 1..OB_MAX_WORKERS.  beta1, beta2 in [0, 1), eps > 0, lr: Adam
+ * hyperparameters (the same lr drives the compressed phase).  d_params:
+ * device float[n_padded] in the padded layout, caller-owned, updated in
+ * place by the step calls (NULL allowed only when n_padded is 0).  d_workspace: device buffer of workspace_bytes
+ * >= ob_workspace_bytes(...), 256-byte aligned, caller-owned, not touched
+ * by the caller while the context lives.  cuda_stream: cudaStream_t (NULL =
+ * legacy default stream) on the current device; every call of this
+ * context queues its work there.  The call uploads the work list and
+ * zeroes the state, then waits for the stream.  *out receives the context.
+ * Errors: OB_ERR_INVALID_ARG, OB_ERR_ALIGN, OB_ERR_WORKSPACE, OB_ERR_OOM,
+ * OB_ERR_CUDA. */
+OB_API ob_status ob_create(int n_tensors, const int64_t *numel, int W, float beta1, float beta2,
+                    float eps, float lr, float *d_params, void *d_workspace,
+                    size_t workspace_bytes, void *cuda_stream, ob_ctx **out);
+
+/* Destroy a context (NULL and unknown pointers are ignored).  Waits for the
+ * context's stream; frees only host-side objects. */
+OB_API void ob_destroy(ob_ctx *ctx);
+
+/* One full-precision Adam step on the averaged gradient
+ * [1BA, Proposed method, 1].  d_grads: host array of W device pointers,
+ * each a float[n_padded] gradient in the padded layout (read only).  With
+ * t the new step count, bc1 = 1 - beta1^t, bc2 = 1 - beta2^t:
+ *   gbar = (g_0 + ... + g_{W-1}) / W,  m = beta1 m + (1-beta1) gbar,
+ *   v = beta2 v + (1-beta2) gbar^2,    p -= lr (m/bc1) / (sqrt(v/bc2) + eps).
+ * Pointers may be NULL when n_padded is 0.  OB_ERR_PHASE after the freeze. */
+OB_API ob_status ob_warmup_adam_step(ob_ctx *ctx, const float *const *d_grads);
+
+/* Freeze the variance [1BA, Abstract; Proposed method, 2]: d = sqrt(v /
+ * bc2(Tw)) + eps replaces v (Tw = warmup steps taken), every worker and
+ * server error is set to 0, and m is kept.  OB_ERR_PHASE if no warmup step
+ * was taken or the variance is already frozen. */
+OB_API ob_status ob_freeze_variance(ob_ctx *ctx);
+
+/* One compression-phase step [1BA, Proposed method, 1-4], all on the GPU:
+ *   worker stage, per worker w and tensor t:
+ *     m_w = beta1 m + (1-beta1) g_w;  x = m_w + e_w;
+ *     s_w = ||x||_2 / sqrt(numel_t);  signs of x packed 32 per word;
+ *     e_w = x - sign(x) s_w;
+ *   server stage, per tensor t and server chunk j:
+ *     y = (sum over w in order of sign_w s_w) / W + e_s;
+ *     s'_j = ||y over chunk j||_2 / sqrt(len_j) (0 for an empty chunk);
+ *     signs of y packed;  e_s = y - sign(y) s'_j;
+ *   gather and update:  m_hat = sign(y) s'_j;  p -= lr (m_hat / d);
+ *     m = m_hat for every worker.
+ * d_grads: as for ob_warmup_adam_step.  OB_ERR_PHASE before the freeze. */
+OB_API ob_status ob_compressed_step(ob_ctx *ctx, const float *const *d_grads);
+
+/* Bytes of device staging ob_compressed_step_host needs (host only). */
+OB_API ob_status ob_host_staging_bytes(const ob_ctx *ctx, size_t *bytes);
+
+/* The compression-phase step with the gradients in HOST memory.  h_grads:
+ * host array of W host pointers, each float[n_padded] in the padded layout
+ * (page-locked memory lets the copies overlap the worker stage).  The
+ * gradients are copied to the GPU in slices through d_staging (device,
+ * caller-owned, >= ob_host_staging_bytes, 256-byte aligned) on a second
+ * stream, overlapping the worker stage of earlier slices; the rest of the
+ * step is ob_compressed_step's.  h_server_scales (may be NULL) receives the
+ * step's server chunk scales, float[n_tensors][W].  The call returns when
+ * the step is complete on the GPU.  Errors as ob_compressed_step, plus
+ * OB_ERR_WORKSPACE for a small staging buffer. */
+OB_API ob_status ob_compressed_step_host(ob_ctx *ctx, const float *const *h_grads, void *d_staging,
+                                  size_t staging_bytes, float *h_server_scales);
+
+/* Copy one piece of state to host memory.  kind: ob_state_kind.  index:
+ * the worker for OB_STATE_E_WORKER / OB_STATE_BITS_WORKER, else 0.  bytes:
+ * must equal the size listed with the kind.  Waits for the stream first.
+ * Error buffers are decoded on the GPU (padding entries read as 0).
+ * OB_ERR_PHASE for V after / D before the freeze. */
+OB_API ob_status ob_read_state(ob_ctx *ctx, int kind, int index, void *host_dst, size_t bytes);
+
+/* Overwrite one piece of state from host memory (resume from a checkpoint,
+ * or re-sync with another implementation).  Same arguments as
+ * ob_read_state; the kinds marked r above are read only
+ * (OB_ERR_INVALID_ARG).  OB_STATE_STEP takes {t_warmup >= 0,
+ * t_compressed >= 0, frozen in {0,1}} with frozen requiring t_warmup >= 1.
+ * Waits for the copy to finish. */
+OB_API ob_status ob_write_state(ob_ctx *ctx, int kind, int index, const void *host_src, size_t bytes);
+
+/* Turn per-kernel timing on or off.  While on, every step records CUDA
+ * events between its kernels on the context's stream. */
+OB_API ob_status ob_profile_enable(ob_ctx *ctx, int on);
+
+/* Wait for the stream and return, per ob_kernel_id, the summed event time
+ * in milliseconds (ms, may be NULL) and the number of launches (launches,
+ * may be NULL) since profiling was enabled or last reset; reset != 0 clears
+ * the counters afterwards.  Arrays have OB_NUM_KERNELS entries. */
+OB_API ob_status ob_profile_read(ob_ctx *ctx, double *ms, int64_t *launches, int reset);
+
+/* Name of a kernel id, or NULL for an unknown id. */
+OB_API const char *ob_kernel_name(int kernel_id);
+
+/* Test hook: make the countdown-th host allocation from now on fail with
+ * OB_ERR_OOM (countdown <= 0 disarms).  Host memory only. */
+OB_API void ob_test_fail_host_alloc(int countdown);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ONEBIT_H */
