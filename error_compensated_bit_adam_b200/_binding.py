@@ -37,6 +37,8 @@ OB_STATE_BITS_WORKER = 8
 OB_STATE_BITS_SERVER = 9
 OB_STATE_STEP = 10
 
+OB_STATIC_MAX_ELEMENTS = 1 << 26
+
 OB_K_WARMUP = 0
 OB_K_FREEZE = 1
 OB_K_PACK = 2
@@ -52,6 +54,7 @@ EXPORTS = (
     "ob_create", "ob_destroy", "ob_warmup_adam_step", "ob_freeze_variance", "ob_compressed_step",
     "ob_host_staging_bytes", "ob_compressed_step_host", "ob_read_state", "ob_write_state",
     "ob_profile_enable", "ob_profile_read", "ob_kernel_name", "ob_test_fail_host_alloc",
+    "ob_onebit_compress_static",
 )
 
 
@@ -96,6 +99,7 @@ def lib() -> ctypes.CDLL:
         "ob_profile_read": (i32, [vp, ctypes.POINTER(ctypes.c_double), P64, i32]),
         "ob_kernel_name": (ctypes.c_char_p, [i32]),
         "ob_test_fail_host_alloc": (None, [i32]),
+        "ob_onebit_compress_static": (i32, [vp, i64, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -233,3 +237,15 @@ def ob_profile_read(ctx: int, reset: bool = False) -> Tuple[List[float], List[in
     n = (ctypes.c_int64 * OB_NUM_KERNELS)()
     _check(lib().ob_profile_read(ctx, ms, n, 1 if reset else 0), "ob_profile_read")
     return [float(v) for v in ms], [int(v) for v in n]
+
+
+# ------------------------------------------------------ allocation-free call
+
+def ob_onebit_compress_static(d_x: int, n: int, d_bits: int, d_error: int, d_scale: int,
+                              cuda_stream: int) -> None:
+    """1-bit compression of one device vector with the library's static
+    scratch: for callers that cannot allocate device memory."""
+    _check(lib().ob_onebit_compress_static(int(d_x) or None, int(n), int(d_bits) or None,
+                                           int(d_error) or None, int(d_scale) or None,
+                                           int(cuda_stream) or None),
+           "ob_onebit_compress_static")

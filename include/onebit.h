@@ -231,6 +231,36 @@ OB_API const char *ob_kernel_name(int kernel_id);
  * OB_ERR_OOM (countdown <= 0 disarms).  Host memory only. */
 OB_API void ob_test_fail_host_alloc(int countdown);
 
+/* --------------------------------------------------------------------
+ * A compressor that allocates nothing.
+ *
+ * Some callers cannot allocate device memory: a plugin inside a host
+ * framework whose caching allocator has already reserved the GPU's memory
+ * (a direct cudaMalloc there fails or fragments the pool), or a
+ * latency-critical loop that cannot afford cudaMalloc's implicit device
+ * synchronization.  For them this entry point needs no workspace at all:
+ * the caller passes only inputs and outputs, and the scratch (one fp64
+ * partial sum per 4096 elements) is a static device array of the library,
+ * sized for OB_STATIC_MAX_ELEMENTS elements (128 KiB), which every GPU
+ * that loads the library holds until the process exits.  The paper has no
+ * counterpart to this call; it is the worker stage's compressor of
+ * ob_compressed_step applied to a given x:
+ *   s = ||x||_2 / sqrt(n);  bits: 1 where x >= 0;  e = x - sign(x) s.
+ * d_x: device float[n] (16-byte aligned, no padding needed).  d_bits:
+ * device uint32[ceil(n/32)] (bits past n are 0).  d_error: device float[n]
+ * (16-byte aligned; may not alias d_x).  d_scale: device float[1].  All
+ * work is queued on cuda_stream; the call does no cudaMalloc, cudaFree or
+ * other allocating call.  The first call on a device looks up the scratch
+ * array's device address (with that device current); make that first call
+ * before any stream capture.  Every call shares the one scratch array and
+ * overwrites the part it reads, so calls that overlap on the GPU (on
+ * different streams) race; serialize them.  n above OB_STATIC_MAX_ELEMENTS
+ * returns OB_ERR_WORKSPACE; bad pointers OB_ERR_INVALID_ARG / OB_ERR_ALIGN;
+ * a failed lookup or launch OB_ERR_CUDA. */
+#define OB_STATIC_MAX_ELEMENTS ((int64_t)1 << 26)
+OB_API ob_status ob_onebit_compress_static(const float *d_x, int64_t n, uint32_t *d_bits,
+                                           float *d_error, float *d_scale, void *cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -23,7 +23,6 @@ def declared_symbols():
 
 def test_library_exports_every_declared_symbol():
     names = declared_symbols()
-    assert len(names) == 18
     L = B.lib()
     for name in names:
         assert hasattr(L, name), name
