@@ -251,6 +251,9 @@ struct ob_ctx {
     cudaEvent_t ev_start = nullptr;
     int64_t t_warmup = 0, t_compressed = 0;
     bool frozen = false;
+    // m is held densely in the m region (after create / warmup / a write),
+    // or, after a compressed step, only as the server words and scales.
+    bool m_dense = true;
     bool broken = false;
     // profiling
     bool profiling = false;
@@ -334,6 +337,9 @@ ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int ti
     P.tile_base = tile_lo;
     P.n_tiles = c->n_tiles();
     P.m = c->m();
+    P.m_bits = c->sbits();
+    P.m_scale = c->sp_last();
+    P.m_dense = c->m_dense ? 1 : 0;
     for (int w = 0; w < OB_MAX_WORKERS; ++w) P.g[w] = w < c->plan.W ? g[w] : nullptr;
     P.g_offset = g_offset;
     P.x = c->x();
@@ -345,7 +351,7 @@ ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int ti
     P.T = c->plan.T;
     P.beta1 = c->beta1;
     P.c1 = c->c1;
-    onebit::ob_pack_kernel<<<grid1(tile_hi - tile_lo), kThreads, 0, c->stream>>>(P);
+    onebit::ob_pack_kernel<<<grid1(tile_hi - tile_lo), kThreads, onebit::kPackSmemBytes, c->stream>>>(P);
     return fail_cuda(c, cudaGetLastError());
 }
 
@@ -374,7 +380,10 @@ ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
         P.n_pad = c->plan.n_pad;
         P.W = W;
         P.T = T;
-        onebit::ob_server_kernel<<<grid1(nt), kThreads, 0, c->stream>>>(P);
+        P.w_pow2 = (W & (W - 1)) == 0;
+        P.inv_w = 1.0f / (float)W;  // exact for a power of two
+        const size_t smem = (size_t)W * onebit::kTileWords * sizeof(uint32_t);
+        onebit::ob_server_kernel<<<grid1(nt), kThreads, smem, c->stream>>>(P);
         k.stop();
         ob_status st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
@@ -395,7 +404,7 @@ ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
         P.sp = c->sp_last();
         P.d = c->v();
         P.p = c->params;
-        P.m = c->m();
+        P.m = nullptr;  // m stays as (sbits, sp_last); see ob_ctx::m_dense
         P.W = W;
         P.lr = c->lr;
         onebit::ob_apply_kernel<<<grid1(nt), kThreads, 0, c->stream>>>(P);
@@ -433,26 +442,17 @@ size_t state_bytes(const ob_ctx *c, int kind) {
     }
 }
 
-// Decode a lazily stored error buffer (x or y with its scales) into host
-// memory, run by run through the staging region.
-ob_status read_error(ob_ctx *c, const float *src, const float *scales, int stride_t, int stride_j,
-                     float *host) {
+// Decode a lazily stored buffer into host memory, run by run through the
+// staging region.  launch(run, out, out_base) queues the decoder of one run.
+template <class Launch>
+ob_status read_decoded(ob_ctx *c, float *host, Launch launch) {
     std::memset(host, 0, (size_t)c->plan.n_pad * 4);
     std::vector<Run> runs = make_runs(c->plan.tiles, kDecodeStage);
     for (const Run &r : runs) {
         const int64_t span = r.elem_hi - r.elem_lo;
         ob_status st = fail_cuda(c, cudaMemsetAsync(c->stage(), 0, (size_t)span * 4, c->stream));
         if (st != OB_OK) return st;
-        onebit::DecodeParams P;
-        P.tiles = c->tiles();
-        P.tile_base = r.tile_lo;
-        P.x = src;
-        P.scales = scales;
-        P.stride_t = stride_t;
-        P.stride_j = stride_j;
-        P.out = c->stage();
-        P.out_base = r.elem_lo;
-        onebit::ob_decode_error_kernel<<<grid1(r.tile_hi - r.tile_lo), kThreads, 0, c->stream>>>(P);
+        launch(r, c->stage(), r.elem_lo);
         st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
         st = fail_cuda(c, cudaMemcpyAsync(host + r.elem_lo, c->stage(), (size_t)span * 4,
@@ -461,6 +461,42 @@ ob_status read_error(ob_ctx *c, const float *src, const float *scales, int strid
         st = fail_cuda(c, cudaStreamSynchronize(c->stream));
         if (st != OB_OK) return st;
     }
+    return OB_OK;
+}
+
+// Error buffer (x or y with its scales): e = fl(x - sign(x) s).
+ob_status read_error(ob_ctx *c, const float *src, const float *scales, int stride_t, int stride_j,
+                     float *host) {
+    return read_decoded(c, host, [&](const Run &r, float *out, int64_t base) {
+        onebit::DecodeParams P;
+        P.tiles = c->tiles();
+        P.tile_base = r.tile_lo;
+        P.x = src;
+        P.scales = scales;
+        P.stride_t = stride_t;
+        P.stride_j = stride_j;
+        P.out = out;
+        P.out_base = base;
+        onebit::ob_decode_error_kernel<<<grid1(r.tile_hi - r.tile_lo), kThreads, 0, c->stream>>>(P);
+    });
+}
+
+// Momentum held as server words and scales: m = sign' s'_j.
+void launch_decode_momentum(ob_ctx *c, int tile_lo, int tile_hi, float *out, int64_t base) {
+    onebit::ob_decode_momentum_kernel<<<grid1(tile_hi - tile_lo), kThreads, 0, c->stream>>>(
+        c->tiles(), tile_lo, c->sbits(), c->sp_last(), c->plan.W, out, base);
+}
+
+// Rebuild the dense momentum in its own region (before a consumer that
+// needs it dense: the warmup step).
+ob_status materialize_momentum(ob_ctx *c) {
+    if (c->m_dense) return OB_OK;
+    if (c->n_tiles() > 0) {
+        launch_decode_momentum(c, 0, c->n_tiles(), c->m(), 0);
+        ob_status st = fail_cuda(c, cudaGetLastError());
+        if (st != OB_OK) return st;
+    }
+    c->m_dense = true;
     return OB_OK;
 }
 
@@ -582,6 +618,9 @@ ob_status ob_create(int n_tensors, const int64_t *numel, int W, float beta1, flo
     };
     cudaError_t e = cudaGetDevice(&c->device);
     if (e != cudaSuccess) return bail(e);
+    e = cudaFuncSetAttribute(onebit::ob_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             onebit::kPackSmemBytes);
+    if (e != cudaSuccess) return bail(e);
     e = cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking);
     if (e != cudaSuccess) return bail(e);
     for (int k = 0; k < 2 && e == cudaSuccess; ++k) {
@@ -650,6 +689,7 @@ ob_status ob_warmup_adam_step(ob_ctx *c, const float *const *d_grads) {
     if ((st = check_grads(c, d_grads)) != OB_OK) return st;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    if ((st = materialize_momentum(c)) != OB_OK) return st;
     const int64_t t = c->t_warmup + 1;
     onebit::WarmupParams P;
     P.tiles = c->tiles();
@@ -710,6 +750,7 @@ ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
     KernelTimer pack(c, OB_K_PACK);
     if ((st = launch_pack(c, d_grads, 0, 0, c->n_tiles())) != OB_OK) return st;
     if ((st = launch_after_pack(c, pack)) != OB_OK) return st;
+    c->m_dense = false;
     c->t_compressed += 1;
     return OB_OK;
 }
@@ -760,6 +801,7 @@ ob_status ob_compressed_step_host(ob_ctx *c, const float *const *h_grads, void *
         if ((st = fail_cuda(c, cudaEventRecord(c->ev_consumed[slot], c->stream))) != OB_OK) return st;
     }
     if ((st = launch_after_pack(c, pack)) != OB_OK) return st;
+    c->m_dense = false;
     c->t_compressed += 1;
     if (h_server_scales)
         e = cudaMemcpyAsync(h_server_scales, c->sp_last(),
@@ -793,6 +835,11 @@ ob_status ob_read_state(ob_ctx *c, int kind, int index, void *host_dst, size_t b
                               1, 0, static_cast<float *>(host_dst));
         if (kind == OB_STATE_E_SERVER)
             return read_error(c, c->y(), c->sp_prev(), c->plan.W, 1, static_cast<float *>(host_dst));
+        if (kind == OB_STATE_M && !c->m_dense)
+            return read_decoded(c, static_cast<float *>(host_dst),
+                                [&](const Run &r, float *out, int64_t base) {
+                                    launch_decode_momentum(c, r.tile_lo, r.tile_hi, out, base);
+                                });
     } catch (const std::bad_alloc &) {
         return OB_ERR_OOM;
     }
@@ -840,7 +887,7 @@ ob_status ob_write_state(ob_ctx *c, int kind, int index, const void *host_src, s
     cudaError_t e = cudaSuccess;
     switch (kind) {
     case OB_STATE_P: dst = c->params; break;
-    case OB_STATE_M: dst = c->m(); break;
+    case OB_STATE_M: dst = c->m(); c->m_dense = true; break;
     case OB_STATE_V: case OB_STATE_D: dst = c->v(); break;
     case OB_STATE_E_WORKER:
         // stored as (x, s) with s = 0, which decodes to x exactly

@@ -43,6 +43,8 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kUnroll = 4;                 // float4 slots per thread per tile
 constexpr int kTile = kThreads * 4 * kUnroll;  // 4096 elements per tile
 constexpr int kScaleThreads = 256;         // threads of the scale kernels
+constexpr int kPackStages = 2;             // workers in flight in the worker-stage pipeline
+constexpr int kPackSmemBytes = kPackStages * 2 * kUnroll * kThreads * 16;  // 64 KiB: 3 CTAs per SM
 constexpr unsigned kFull = 0xffffffffu;
 
 // One unit of work: up to kTile consecutive elements of one tensor that all
@@ -70,6 +72,13 @@ __device__ __forceinline__ float decode_error(float x, float s) {
     return __fsub_rn(x, signed_scale(code_of(x), s));
 }
 
+// +-s as a float, from a sign word: bit b of `word` set -> +s, clear -> -s.
+// s >= 0, so only the sign bit changes: (~word << (31 - b)) keeps the
+// inverted bit in bit 31.
+__device__ __forceinline__ float signed_from_bit(uint32_t word, int b, uint32_t s_bits) {
+    return __uint_as_float(((~word << (31 - b)) & 0x80000000u) | s_bits);
+}
+
 __device__ __forceinline__ float get(const float4 &v, int k) {
     return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
 }
@@ -84,6 +93,26 @@ __device__ __forceinline__ float4 ld_stream(const float *p) {
 }
 __device__ __forceinline__ void st_stream(float *p, const float4 &v) {
     __stcs(reinterpret_cast<float4 *>(p), v);
+}
+
+// Asynchronous 16-byte global -> shared copies (sm_80+ LDGSTS), with an L2
+// evict-first policy: the CTA queues the next workers' inputs while it
+// computes on the current one.  Completion is awaited per thread with
+// cp.async.wait_group (a hardware wait, no polling).
+__device__ __forceinline__ uint64_t evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, uint64_t pol) {
+    const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem),
+                 "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
 // OR together the 4-bit groups of the 8 lanes that share one 32-bit sign
@@ -196,7 +225,10 @@ struct PackParams {
     const Tile *tiles;
     int tile_base;                   // tile of blockIdx.x == 0
     int n_tiles;                     // total tiles (row length of partial)
-    const float *m;                  // [n_pad]
+    const float *m;                  // [n_pad] dense momentum (when m_dense)
+    const uint32_t *m_bits;          // [n_pad/32] last step's server signs (when !m_dense)
+    const float *m_scale;            // [T][W] last step's server scales (when !m_dense)
+    int m_dense;
     const float *g[OB_MAX_WORKERS];  // element i of worker w at g[w][i - g_offset]
     int64_t g_offset;
     float *x;                        // [W][n_pad]: in x_prev (lazy e_w), out x
@@ -212,7 +244,10 @@ struct PackParams {
 //   m_w = beta1 m + (1-beta1) g_w,  x = m_w + e_w (e_w decoded from the
 //   stored (x_prev, s_prev)), sign bits of x, partial sum of x^2.
 // x overwrites x_prev: with this step's scale it encodes the new e_w.
-// m stays in registers across the W workers, so it is read once.
+// m stays in registers across the W workers, so it is read once.  After a
+// compressed step m is exactly last step's decoded server momentum
+// sign' s'_j, so it is rebuilt from the server words (1/8 byte per
+// parameter) instead of read as fp32 (4 bytes).
 __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant__ PackParams P) {
     const int tile_id = P.tile_base + (int)blockIdx.x;
     const Tile tile = P.tiles[tile_id];
@@ -221,26 +256,70 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
 
     float4 mv[kUnroll];
     int real[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-        const int off = 4 * (tid + kThreads * u);
-        real[u] = slot_real(tile.count, off);
-        mv[u] = real[u] > 0 ? ld_stream(P.m + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    const int64_t words_per_worker = P.n_pad >> 5;
-    for (int w = 0; w < P.W; ++w) {
-        const float s_prev = P.s_prev[w * P.T + tile.tensor];
-        const float *gw = P.g[w] + (tile.begin - P.g_offset);
-        float *xw = P.x + (int64_t)w * P.n_pad + tile.begin;
-        uint32_t *bw = P.bits + (int64_t)w * words_per_worker + (tile.begin >> 5);
-        double ss = 0.0;
+    if (P.m_dense) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int off = 4 * (tid + kThreads * u);
+            real[u] = slot_real(tile.count, off);
+            mv[u] = real[u] > 0 ? ld_stream(P.m + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    } else {
+        const uint32_t sb = __float_as_uint(P.m_scale[tile.tensor * P.W + tile.chunk]);
+        const int shift = 4 * (lane & 7);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int off = 4 * (tid + kThreads * u);
+            real[u] = slot_real(tile.count, off);
+            mv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (real[u] > 0) {
+                const uint32_t word = __ldg(P.m_bits + ((tile.begin + off) >> 5));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) set(mv[u], k, signed_from_bit(word, shift + k, sb));
+            }
+        }
+    }
+    const int64_t words_per_worker = P.n_pad >> 5;
+    // Pipeline over the workers: the gradient and x_prev slots of worker
+    // w + kPackStages - 1 are copied into shared memory (cp.async) while
+    // worker w is computed, so HBM stays busy whatever the arithmetic's
+    // latency.  Each thread reads back only the slots it copied itself, so
+    // its own wait_group is the only synchronisation needed.
+    extern __shared__ float4 pipe[];  // [kPackStages][2 (g, x_prev)][kUnroll][kThreads]
+    const uint64_t pol = evict_first_policy();
+    auto issue = [&](int w) {
+        if (w < P.W) {
+            const int st = w % kPackStages;
+            const float *gw = P.g[w] + (tile.begin - P.g_offset);
+            const float *xw = P.x + (int64_t)w * P.n_pad + tile.begin;
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                if (real[u] > 0) {
+                    const int off = 4 * (tid + kThreads * u);
+                    cp_async16(&pipe[((st * 2 + 0) * kUnroll + u) * kThreads + tid], gw + off, pol);
+                    cp_async16(&pipe[((st * 2 + 1) * kUnroll + u) * kThreads + tid], xw + off, pol);
+                }
+            }
+        }
+        cp_async_commit();  // one group per worker, empty past the last
+    };
+#pragma unroll
+    for (int k = 0; k < kPackStages - 1; ++k) issue(k);
+    for (int w = 0; w < P.W; ++w) {
+        issue(w + kPackStages - 1);
+        cp_async_wait<kPackStages - 1>();  // worker w's group has landed
+        const int st = w % kPackStages;
+        const float s_prev = P.s_prev[w * P.T + tile.tensor];
+        float *xw = P.x + (int64_t)w * P.n_pad + tile.begin;
+        uint32_t *bw = P.bits + (int64_t)w * words_per_worker + (tile.begin >> 5);
+        double ss[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int off = 4 * (tid + kThreads * u);
+            ss[u] = 0.0;
             uint32_t nibble = 0;
             if (real[u] > 0) {
-                const float4 g = ld_stream(gw + off);
-                const float4 xp = ld_stream(xw + off);
+                const float4 g = pipe[((st * 2 + 0) * kUnroll + u) * kThreads + tid];
+                const float4 xp = pipe[((st * 2 + 1) * kUnroll + u) * kThreads + tid];
                 float4 xo = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
@@ -248,7 +327,7 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
                         const float m_w = __fadd_rn(__fmul_rn(P.beta1, get(mv[u], k)),
                                                     __fmul_rn(P.c1, get(g, k)));
                         const float x = __fadd_rn(m_w, decode_error(get(xp, k), s_prev));
-                        ss = __fma_rn((double)x, (double)x, ss);
+                        ss[u] = __fma_rn((double)x, (double)x, ss[u]);
                         nibble |= (uint32_t)code_of(x) << k;
                         set(xo, k, x);
                     }
@@ -258,8 +337,11 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
             const uint32_t word = gather_word(nibble, lane);
             if ((lane & 7) == 0 && off < tile.count) bw[(tid + kThreads * u) >> 3] = word;
         }
-        ss = warp_sum(ss);
-        if (lane == 0) red[warp][w] = ss;
+        double t = 0.0;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) t += ss[u];
+        t = warp_sum(t);
+        if (lane == 0) red[warp][w] = t;
     }
     __syncthreads();
     if (tid < P.W) {
@@ -292,6 +374,8 @@ __global__ void __launch_bounds__(kScaleThreads) ob_pack_scale_kernel(
 
 // ----------------------------------------------------------- server stage
 
+constexpr int kTileWords = kTile / 32;  // sign words of one worker in a full tile
+
 struct ServerParams {
     const Tile *tiles;
     const uint32_t *bits;   // [W][n_pad/32] this step's worker signs
@@ -302,6 +386,8 @@ struct ServerParams {
     double *partial;        // [n_tiles]: sum of y^2 per tile
     int64_t n_pad;
     int W, T;
+    float inv_w;            // 1/W when W is a power of two (then acc*inv_w == acc/W exactly)
+    int w_pow2;
 };
 
 // [1BA, Proposed method, 3-4]: server j = tile.chunk receives every
@@ -309,34 +395,55 @@ struct ServerParams {
 // index into [W][words]) and forms
 //   y = (sum over w in order of sign_w s_w) / W + e_s,
 // with e_s decoded from (y_prev, s'_prev); then the sign bits of y and the
-// tile's partial sum of y^2.
+// tile's partial sum of y^2.  The W workers' words of the tile are first
+// staged in shared memory with one 16-byte load per thread, so the W-long
+// sequential sum never waits on global memory.
 __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_constant__ ServerParams P) {
+    extern __shared__ uint4 staged[];  // [W][kTileWords / 4]
+    __shared__ double red[kWarps];
+    __shared__ uint32_t scale_bits[OB_MAX_WORKERS];
     const int tile_id = blockIdx.x;
     const Tile tile = P.tiles[tile_id];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __shared__ double red[kWarps];
     const int64_t words_per_worker = P.n_pad >> 5;
     const int64_t word0 = tile.begin >> 5;
-    const int shift = 4 * (lane & 7);  // bit of this lane's first element in its word
+    const int groups = (((tile.count + 31) >> 5) + 3) >> 2;  // 16-byte word groups with real elements
 
+    for (int idx = tid; idx < P.W * (kTileWords / 4); idx += kThreads) {
+        const int w = idx / (kTileWords / 4), q = idx % (kTileWords / 4);
+        if (q < groups)
+            staged[idx] = __ldcs(reinterpret_cast<const uint4 *>(P.bits + w * words_per_worker + word0) + q);
+    }
+    if (tid < P.W) scale_bits[tid] = __float_as_uint(P.s_w[tid * P.T + tile.tensor]);
+
+    float4 yo[kUnroll];
+    int real[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * (tid + kThreads * u);
+        real[u] = slot_real(tile.count, off);
+        yo[u] = real[u] > 0 ? ld_stream(P.y + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+
+    const uint32_t *words = reinterpret_cast<const uint32_t *>(staged);
+    const int shift = 4 * (lane & 7);  // bit of this lane's first element in its word
     float acc[kUnroll][4];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u)
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc[u][k] = 0.0f;
-
     for (int w = 0; w < P.W; ++w) {
-        const float s = P.s_w[w * P.T + tile.tensor];
-        const uint32_t *bw = P.bits + (int64_t)w * words_per_worker + word0;
+        const uint32_t sb = scale_bits[w];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int off = 4 * (tid + kThreads * u);
-            if (off < tile.count) {
-                const uint32_t word = __ldg(bw + ((tid + kThreads * u) >> 3)) >> shift;
+            // this lane's 4 bits, inverted, at bits 0..3: element k's sign
+            // bit is then (inv << (31 - k)) & 0x80000000 (a constant shift)
+            const uint32_t inv = ~(words[w * kTileWords + ((tid + kThreads * u) >> 3)] >> shift);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    acc[u][k] = __fadd_rn(acc[u][k], signed_scale((word >> k) & 1u, s));
-            }
+            for (int k = 0; k < 4; ++k)
+                acc[u][k] = __fadd_rn(acc[u][k],
+                                      __uint_as_float(((inv << (31 - k)) & 0x80000000u) | sb));
         }
     }
 
@@ -346,23 +453,20 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
         const int off = 4 * (tid + kThreads * u);
-        const int real = slot_real(tile.count, off);
         uint32_t nibble = 0;
-        if (real > 0) {
-            float *yp = P.y + tile.begin + off;
-            const float4 yo = ld_stream(yp);
+        if (real[u] > 0) {
             float4 yn = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                if (k < real) {
-                    const float avg = __fdiv_rn(acc[u][k], wf);
-                    const float y = __fadd_rn(avg, decode_error(get(yo, k), sp));
+                if (k < real[u]) {
+                    const float avg = P.w_pow2 ? __fmul_rn(acc[u][k], P.inv_w) : __fdiv_rn(acc[u][k], wf);
+                    const float y = __fadd_rn(avg, decode_error(get(yo[u], k), sp));
                     ss = __fma_rn((double)y, (double)y, ss);
                     nibble |= (uint32_t)code_of(y) << k;
                     set(yn, k, y);
                 }
             }
-            st_stream(yp, yn);
+            st_stream(P.y + tile.begin + off, yn);
         }
         const uint32_t word = gather_word(nibble, lane);
         if ((lane & 7) == 0 && off < tile.count) P.sbits[word0 + ((tid + kThreads * u) >> 3)] = word;
@@ -405,18 +509,19 @@ struct ApplyParams {
     const float *sp;        // [T][W] this step's server scales
     const float *d;         // [n_pad] frozen denominator
     float *p;               // [n_pad]
-    float *m;               // [n_pad]
+    float *m;               // [n_pad] dense momentum, or NULL to keep it as (sbits, sp)
     int W;
     float lr;
 };
 
 // [1BA, Proposed method, 1-2]: every worker decodes the gathered server
 // words, m_hat = sign' s'_j, and takes a momentum SGD step preconditioned by
-// the frozen denominator: p -= lr (m_hat / d); m = m_hat.
+// the frozen denominator: p -= lr (m_hat / d); m = m_hat (m is left as the
+// words and scales themselves unless a dense copy is asked for).
 __global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constant__ ApplyParams P) {
     const Tile tile = P.tiles[blockIdx.x];
     const int tid = threadIdx.x, lane = tid & 31;
-    const float s = P.sp[tile.tensor * P.W + tile.chunk];
+    const uint32_t sb = __float_as_uint(P.sp[tile.tensor * P.W + tile.chunk]);
     const int shift = 4 * (lane & 7);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -424,25 +529,47 @@ __global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constan
         const int real = slot_real(tile.count, off);
         if (real == 0) continue;
         const int64_t i = tile.begin + off;
-        const uint32_t word = __ldg(P.sbits + (i >> 5)) >> shift;
+        const uint32_t inv = ~(__ldg(P.sbits + (i >> 5)) >> shift);
         const float4 d = ld_stream(P.d + i);
         float4 p = ld_stream(P.p + i);
         float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             if (k < real) {
-                const float m_hat = signed_scale((word >> k) & 1u, s);
+                const float m_hat = __uint_as_float(((inv << (31 - k)) & 0x80000000u) | sb);
                 const float delta = __fmul_rn(P.lr, __fdiv_rn(m_hat, get(d, k)));
                 set(p, k, __fsub_rn(get(p, k), delta));
                 set(m, k, m_hat);
             }
         }
         st_stream(P.p + i, p);
-        st_stream(P.m + i, m);
+        if (P.m) st_stream(P.m + i, m);
     }
 }
 
 // ------------------------------------------------- state decode for reads
+
+// m = sign' s'_j from the server words, into out[i - out_base], over a run
+// of tiles (padding left untouched).
+__global__ void __launch_bounds__(kThreads) ob_decode_momentum_kernel(
+    const Tile *tiles, int tile_base, const uint32_t *sbits, const float *sp, int W, float *out,
+    int64_t out_base) {
+    const Tile tile = tiles[tile_base + (int)blockIdx.x];
+    const uint32_t sb = __float_as_uint(sp[tile.tensor * W + tile.chunk]);
+    const int shift = 4 * (threadIdx.x & 7);
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * ((int)threadIdx.x + kThreads * u);
+        const int real = slot_real(tile.count, off);
+        if (real == 0) continue;
+        const uint32_t word = sbits[(tile.begin + off) >> 5];
+        float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (k < real) set(m, k, signed_from_bit(word, shift + k, sb));
+        *reinterpret_cast<float4 *>(out + (tile.begin + off - out_base)) = m;
+    }
+}
 
 struct DecodeParams {
     const Tile *tiles;
