@@ -78,7 +78,30 @@ struct Plan {
     std::vector<int> tensor_tile_begin;  // [T+1]
     std::vector<int> chunk_tile_begin;   // [T*W+1]
     std::vector<int64_t> chunk_len;      // [T*W]
+    // segmented scale reductions: first segment slot of each range, the
+    // total number of slots, and the most segments of any range
+    std::vector<int> tensor_seg_base, chunk_seg_base;
+    int tensor_segs = 0, chunk_segs = 0, tensor_max_seg = 1, chunk_max_seg = 1;
 };
+
+int scale_segments(int tiles) {
+    return tiles <= onebit::kScaleSegTiles ? 1
+                                           : (tiles + onebit::kScaleSegTiles - 1) / onebit::kScaleSegTiles;
+}
+
+void plan_segments(const std::vector<int> &range_begin, std::vector<int> *base, int *total, int *most) {
+    const size_t R = range_begin.size() - 1;
+    base->assign(R, 0);
+    int pos = 0;
+    *most = 1;
+    for (size_t r = 0; r < R; ++r) {
+        const int nseg = scale_segments(range_begin[r + 1] - range_begin[r]);
+        (*base)[r] = pos;
+        pos += nseg;
+        *most = std::max(*most, nseg);
+    }
+    *total = pos;
+}
 
 ob_status check_list(int n_tensors, const int64_t *numel) {
     if (n_tensors < 1 || !numel) return OB_ERR_INVALID_ARG;
@@ -139,13 +162,17 @@ ob_status make_plan(int n_tensors, const int64_t *numel, int W, bool with_tiles,
     }
     pl->tensor_tile_begin[n_tensors] = (int)pl->tiles.size();
     pl->chunk_tile_begin[(size_t)n_tensors * W] = (int)pl->tiles.size();
+    host_alloc_point();
+    plan_segments(pl->tensor_tile_begin, &pl->tensor_seg_base, &pl->tensor_segs, &pl->tensor_max_seg);
+    plan_segments(pl->chunk_tile_begin, &pl->chunk_seg_base, &pl->chunk_segs, &pl->chunk_max_seg);
     return OB_OK;
 }
 
 // Byte offsets of the workspace regions.
 struct Carve {
-    size_t m, v, x, y, bits, sbits, s_prev, s_last, sp_prev, sp_last, partial_w, partial_s, tiles,
-        tensor_tile_begin, chunk_tile_begin, numel, chunk_len, stage, total;
+    size_t m, v, x, y, bits, sbits, s_prev, s_last, sp_prev, sp_last, partial_w, partial_s,
+        counters_w, counters_s, seg_w, seg_s, tiles, tensor_tile_begin, chunk_tile_begin, numel,
+        chunk_len, tensor_seg_base, chunk_seg_base, stage, total;
 };
 
 Carve carve(const Plan &pl) {
@@ -170,11 +197,17 @@ Carve carve(const Plan &pl) {
     c.sp_last = take(T * W * 4);
     c.partial_w = take(W * nt * 8);
     c.partial_s = take(nt * 8);
+    c.counters_w = take(T * W * 4);
+    c.counters_s = take(T * W * 4);
+    c.seg_w = take((size_t)pl.tensor_segs * W * 8);
+    c.seg_s = take((size_t)pl.chunk_segs * 8);
     c.tiles = take(nt * sizeof(Tile));
     c.tensor_tile_begin = take((T + 1) * 4);
     c.chunk_tile_begin = take((T * W + 1) * 4);
     c.numel = take(T * 8);
     c.chunk_len = take(T * W * 8);
+    c.tensor_seg_base = take(T * 4);
+    c.chunk_seg_base = take(T * W * 4);
     c.stage = take((size_t)kDecodeStage * 4);
     c.total = off;
     return c;
@@ -228,8 +261,8 @@ struct DeviceGuard {
 };
 
 const char *const kKernelNames[OB_NUM_KERNELS] = {
-    "ob_warmup_kernel", "ob_freeze_kernel",       "ob_pack_kernel", "ob_pack_scale_kernel",
-    "ob_server_kernel", "ob_server_scale_kernel", "ob_apply_kernel"};
+    "ob_warmup_kernel", "ob_freeze_kernel",       "ob_pack_kernel", "ob_scale_kernel:worker",
+    "ob_server_kernel", "ob_scale_kernel:server", "ob_apply_kernel"};
 
 }  // namespace
 
@@ -280,6 +313,12 @@ struct ob_ctx {
     int *chunk_tile_begin() const { return at<int>(cv.chunk_tile_begin); }
     int64_t *numel() const { return at<int64_t>(cv.numel); }
     int64_t *chunk_len() const { return at<int64_t>(cv.chunk_len); }
+    unsigned *counters_w() const { return at<unsigned>(cv.counters_w); }
+    unsigned *counters_s() const { return at<unsigned>(cv.counters_s); }
+    double *seg_w() const { return at<double>(cv.seg_w); }
+    double *seg_s() const { return at<double>(cv.seg_s); }
+    int *tensor_seg_base() const { return at<int>(cv.tensor_seg_base); }
+    int *chunk_seg_base() const { return at<int>(cv.chunk_seg_base); }
     float *stage() const { return at<float>(cv.stage); }
     int n_tiles() const { return (int)plan.tiles.size(); }
 };
@@ -361,8 +400,22 @@ ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
     pack_timer.stop();
     {
         KernelTimer k(c, OB_K_PACK_SCALE);
-        onebit::ob_pack_scale_kernel<<<dim3((unsigned)T, (unsigned)W), kScaleThreads, 0, c->stream>>>(
-            c->partial_w(), nt, c->tensor_tile_begin(), c->numel(), T, c->s_prev(), c->s_last());
+        onebit::ScaleParams P;
+        P.partial = c->partial_w();
+        P.n_tiles = nt;
+        P.range_begin = c->tensor_tile_begin();
+        P.seg_base = c->tensor_seg_base();
+        P.count = c->numel();
+        P.seg = c->seg_w();
+        P.counter = c->counters_w();
+        P.out_prev = c->s_prev();
+        P.out_last = c->s_last();
+        P.rows = W;
+        P.R = T;
+        P.out_stride_r = 1;
+        P.out_stride_row = T;
+        onebit::ob_scale_kernel<<<dim3((unsigned)T, (unsigned)W, (unsigned)c->plan.tensor_max_seg),
+                                  kScaleThreads, 0, c->stream>>>(P);
         k.stop();
         ob_status st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
@@ -390,8 +443,22 @@ ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
     }
     {
         KernelTimer k(c, OB_K_SERVER_SCALE);
-        onebit::ob_server_scale_kernel<<<grid1(T * W), kScaleThreads, 0, c->stream>>>(
-            c->partial_s(), c->chunk_tile_begin(), c->chunk_len(), c->sp_prev(), c->sp_last());
+        onebit::ScaleParams P;
+        P.partial = c->partial_s();
+        P.n_tiles = nt;
+        P.range_begin = c->chunk_tile_begin();
+        P.seg_base = c->chunk_seg_base();
+        P.count = c->chunk_len();
+        P.seg = c->seg_s();
+        P.counter = c->counters_s();
+        P.out_prev = c->sp_prev();
+        P.out_last = c->sp_last();
+        P.rows = 1;
+        P.R = T * W;
+        P.out_stride_r = 1;
+        P.out_stride_row = 0;
+        onebit::ob_scale_kernel<<<dim3((unsigned)(T * W), 1u, (unsigned)c->plan.chunk_max_seg),
+                                  kScaleThreads, 0, c->stream>>>(P);
         k.stop();
         ob_status st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
@@ -647,6 +714,12 @@ ob_status ob_create(int n_tensors, const int64_t *numel, int W, float beta1, flo
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(c->chunk_len(), pl.chunk_len.data(), pl.chunk_len.size() * 8,
                             cudaMemcpyHostToDevice, c->stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(c->tensor_seg_base(), pl.tensor_seg_base.data(),
+                            pl.tensor_seg_base.size() * 4, cudaMemcpyHostToDevice, c->stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(c->chunk_seg_base(), pl.chunk_seg_base.data(),
+                            pl.chunk_seg_base.size() * 4, cudaMemcpyHostToDevice, c->stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
     if (e != cudaSuccess) return bail(e);
     {

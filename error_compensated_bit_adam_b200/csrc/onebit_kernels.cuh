@@ -6,9 +6,9 @@
 // kernels over a list of 4096-element tiles:
 //
 //   ob_pack_kernel          worker stage, all W workers of a tile per CTA
-//   ob_pack_scale_kernel    worker scales per (tensor, worker)
+//   ob_scale_kernel         worker scales per (tensor, worker)
 //   ob_server_kernel        server stage of a tile
-//   ob_server_scale_kernel  server scales per (tensor, chunk)
+//   ob_scale_kernel         server scales per (tensor, chunk)
 //   ob_apply_kernel         gather, decode, preconditioned update
 //
 // plus the warmup Adam step, the freeze and an error decoder used when the
@@ -59,6 +59,8 @@ struct Tile {
     int32_t reserved;
 };
 static_assert(sizeof(Tile) == 24, "Tile layout");
+static_assert(kWarps * kUnroll * 128 == kTile, "warp spans cover a tile");
+static_assert(kUnroll * 4 <= 32, "a warp's sign words fit one store");
 
 // ---------------------------------------------------------------- helpers
 
@@ -125,6 +127,27 @@ __device__ __forceinline__ uint32_t gather_word(uint32_t nibble, int lane) {
     v |= __shfl_xor_sync(kFull, v, 2);
     v |= __shfl_xor_sync(kFull, v, 4);
     return v;
+}
+
+// Element offset, within a tile, of slot u of a thread when each warp owns a
+// contiguous span of kUnroll * 128 elements: warp `warp`'s slot u covers
+// [512 warp + 128 u, +128), lane l holding elements 4l..4l+3 of it.  The
+// warp's sign words for the span are then 4 * kUnroll consecutive words.
+__device__ __forceinline__ int span_off(int warp, int lane, int u) {
+    return (kUnroll * 128) * warp + 128 * u + 4 * lane;
+}
+
+// After gather_word for every slot, lanes 0, 8, 16, 24 hold words 4u..4u+3
+// of slot u.  Bring word L of the warp's 4 * kUnroll to lane L so the warp
+// stores all of them with one 64-byte, sector-aligned write.
+__device__ __forceinline__ uint32_t collect_words(const uint32_t (&word)[kUnroll], int lane) {
+    uint32_t mine = 0;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const uint32_t v = __shfl_sync(kFull, word[u], 8 * (lane & 3));
+        if ((lane >> 2) == u) mine = v;
+    }
+    return mine;
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -259,7 +282,7 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
     if (P.m_dense) {
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int off = 4 * (tid + kThreads * u);
+            const int off = span_off(warp, lane, u);
             real[u] = slot_real(tile.count, off);
             mv[u] = real[u] > 0 ? ld_stream(P.m + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
@@ -268,7 +291,7 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
         const int shift = 4 * (lane & 7);
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int off = 4 * (tid + kThreads * u);
+            const int off = span_off(warp, lane, u);
             real[u] = slot_real(tile.count, off);
             mv[u] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (real[u] > 0) {
@@ -294,7 +317,7 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 if (real[u] > 0) {
-                    const int off = 4 * (tid + kThreads * u);
+                    const int off = span_off(warp, lane, u);
                     cp_async16(&pipe[((st * 2 + 0) * kUnroll + u) * kThreads + tid], gw + off, pol);
                     cp_async16(&pipe[((st * 2 + 1) * kUnroll + u) * kThreads + tid], xw + off, pol);
                 }
@@ -312,9 +335,10 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
         float *xw = P.x + (int64_t)w * P.n_pad + tile.begin;
         uint32_t *bw = P.bits + (int64_t)w * words_per_worker + (tile.begin >> 5);
         double ss[kUnroll];
+        uint32_t words[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            const int off = 4 * (tid + kThreads * u);
+            const int off = span_off(warp, lane, u);
             ss[u] = 0.0;
             uint32_t nibble = 0;
             if (real[u] > 0) {
@@ -334,9 +358,11 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
                 }
                 st_stream(xw + off, xo);
             }
-            const uint32_t word = gather_word(nibble, lane);
-            if ((lane & 7) == 0 && off < tile.count) bw[(tid + kThreads * u) >> 3] = word;
+            words[u] = gather_word(nibble, lane);
         }
+        const uint32_t mine = collect_words(words, lane);
+        if (lane < 4 * kUnroll && (kUnroll * 128) * warp + 32 * lane < tile.count)
+            bw[4 * kUnroll * warp + lane] = mine;
         double t = 0.0;
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) t += ss[u];
@@ -352,23 +378,101 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
     }
 }
 
-// Worker scale of (tensor t = blockIdx.x, worker w = blockIdx.y):
-// s = ||x||_2 / sqrt(numel_t) from the tile partial sums (tiles in order).
-__global__ void __launch_bounds__(kScaleThreads) ob_pack_scale_kernel(
-    const double *partial, int n_tiles, const int *tensor_tile_begin, const int64_t *numel, int T,
-    float *s_prev, float *s_last) {
+// ------------------------------------------------------------- scales
+//
+// A scale is sqrt(S / count) with S the sum of the per-tile partial sums of
+// one range of tiles (a tensor for the worker scales, a server chunk for
+// the server scales).  A range is cut into segments of kScaleSegTiles
+// tiles; one CTA sums one segment, and the CTA that finishes last for the
+// range sums the segment results in segment order.  The order of every
+// addition is fixed by the layout, so the scales repeat run to run.  The
+// last CTA is found with a per-range counter (thread fence, then atomic
+// increment; it resets the counter), so nothing ever waits.
+
+constexpr int kScaleSegTiles = 2048;
+
+__device__ __forceinline__ double segment_sum(const double *v, int lo, int hi, double *smem) {
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    int k = lo + (int)threadIdx.x;
+    for (; k + 3 * kScaleThreads < hi; k += 4 * kScaleThreads) {
+        a0 += __ldcg(v + k);
+        a1 += __ldcg(v + k + kScaleThreads);
+        a2 += __ldcg(v + k + 2 * kScaleThreads);
+        a3 += __ldcg(v + k + 3 * kScaleThreads);
+    }
+    for (; k < hi; k += kScaleThreads) a0 += __ldcg(v + k);
+    return block_sum((a0 + a1) + (a2 + a3), smem);
+}
+
+// One segment of range r; returns (in thread 0, with *done = true) the
+// range's total when this CTA is the last of the range's nseg CTAs.
+__device__ __forceinline__ bool range_sum(const double *v, int lo, int hi, int seg, int nseg,
+                                          double *seg_out, unsigned *counter, double *total) {
     __shared__ double smem[kScaleThreads / 32];
-    const int t = blockIdx.x, w = blockIdx.y;
-    const int lo = tensor_tile_begin[t], hi = tensor_tile_begin[t + 1];
-    const double *row = partial + (int64_t)w * n_tiles;
-    double acc = 0.0;
-    for (int k = lo + (int)threadIdx.x; k < hi; k += kScaleThreads) acc += row[k];
-    acc = block_sum(acc, smem);
+    __shared__ bool last;
+    const int a = lo + seg * kScaleSegTiles;
+    const int b = min(hi, a + kScaleSegTiles);
+    const double part = segment_sum(v, a, b, smem);
+    if (nseg == 1) {
+        *total = part;
+        return true;
+    }
     if (threadIdx.x == 0) {
-        const int64_t n = numel[t];
-        const float s = n > 0 ? __double2float_rn(__dsqrt_rn(__ddiv_rn(acc, (double)n))) : 0.0f;
-        s_prev[w * T + t] = s;
-        s_last[w * T + t] = s;
+        seg_out[seg] = part;
+        __threadfence();
+        last = atomicAdd(counter, 1u) == (unsigned)(nseg - 1);
+    }
+    __syncthreads();
+    if (!last) return false;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        double acc = 0.0;
+        for (int k = 0; k < nseg; ++k) acc += __ldcg(seg_out + k);
+        *counter = 0u;
+        *total = acc;
+    }
+    return true;
+}
+
+__device__ __forceinline__ int num_segments(int tiles) {
+    return tiles <= kScaleSegTiles ? 1 : (tiles + kScaleSegTiles - 1) / kScaleSegTiles;
+}
+
+__device__ __forceinline__ float rms(double sum_sq, int64_t count) {
+    return count > 0 ? __double2float_rn(__dsqrt_rn(__ddiv_rn(sum_sq, (double)count))) : 0.0f;
+}
+
+struct ScaleParams {
+    const double *partial;     // per-tile sums
+    int n_tiles;               // row length of partial (worker scales: one row per worker)
+    const int *range_begin;    // [R+1] tile ranges
+    const int *seg_base;       // [R] first segment slot of each range
+    const int64_t *count;      // [R] elements of each range
+    double *seg;               // segment results, [segments][rows]
+    unsigned *counter;         // [R][rows], zero between launches
+    float *out_prev, *out_last;
+    int rows;                  // workers (worker scales) or 1 (server scales)
+    int R;
+    int out_stride_r, out_stride_row;  // out[r * stride_r + row * stride_row]
+};
+
+// Grid (R, rows, segments): worker scales use ranges = tensors and one row
+// per worker; server scales use ranges = (tensor, chunk) and one row.
+__global__ void __launch_bounds__(kScaleThreads) ob_scale_kernel(const __grid_constant__ ScaleParams P) {
+    const int r = blockIdx.x, row = blockIdx.y, seg = blockIdx.z;
+    const int lo = P.range_begin[r], hi = P.range_begin[r + 1];
+    const int nseg = num_segments(hi - lo);
+    if (seg >= nseg) return;
+    double total = 0.0;
+    const double *v = P.partial + (int64_t)row * P.n_tiles;
+    double *seg_out = P.seg + ((int64_t)P.seg_base[r] * P.rows + (int64_t)row * nseg);
+    if (!range_sum(v, lo, hi, seg, nseg, seg_out, P.counter + (int64_t)r * P.rows + row, &total))
+        return;
+    if (threadIdx.x == 0) {
+        const float s = rms(total, P.count[r]);
+        const int64_t o = (int64_t)r * P.out_stride_r + (int64_t)row * P.out_stride_row;
+        P.out_prev[o] = s;
+        P.out_last[o] = s;
     }
 }
 
@@ -420,7 +524,7 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
     int real[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-        const int off = 4 * (tid + kThreads * u);
+        const int off = span_off(warp, lane, u);
         real[u] = slot_real(tile.count, off);
         yo[u] = real[u] > 0 ? ld_stream(P.y + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -439,7 +543,7 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
         for (int u = 0; u < kUnroll; ++u) {
             // this lane's 4 bits, inverted, at bits 0..3: element k's sign
             // bit is then (inv << (31 - k)) & 0x80000000 (a constant shift)
-            const uint32_t inv = ~(words[w * kTileWords + ((tid + kThreads * u) >> 3)] >> shift);
+            const uint32_t inv = ~(words[w * kTileWords + (span_off(warp, lane, u) >> 5)] >> shift);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
                 acc[u][k] = __fadd_rn(acc[u][k],
@@ -449,11 +553,13 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
 
     const float wf = (float)P.W;
     const float sp = P.sp_prev[tile.tensor * P.W + tile.chunk];
-    double ss = 0.0;
+    double ss[kUnroll];
+    uint32_t out_words[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-        const int off = 4 * (tid + kThreads * u);
+        const int off = span_off(warp, lane, u);
         uint32_t nibble = 0;
+        ss[u] = 0.0;
         if (real[u] > 0) {
             float4 yn = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -461,43 +567,29 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
                 if (k < real[u]) {
                     const float avg = P.w_pow2 ? __fmul_rn(acc[u][k], P.inv_w) : __fdiv_rn(acc[u][k], wf);
                     const float y = __fadd_rn(avg, decode_error(get(yo[u], k), sp));
-                    ss = __fma_rn((double)y, (double)y, ss);
+                    ss[u] = __fma_rn((double)y, (double)y, ss[u]);
                     nibble |= (uint32_t)code_of(y) << k;
                     set(yn, k, y);
                 }
             }
             st_stream(P.y + tile.begin + off, yn);
         }
-        const uint32_t word = gather_word(nibble, lane);
-        if ((lane & 7) == 0 && off < tile.count) P.sbits[word0 + ((tid + kThreads * u) >> 3)] = word;
+        out_words[u] = gather_word(nibble, lane);
     }
-    ss = warp_sum(ss);
-    if (lane == 0) red[warp] = ss;
+    const uint32_t mine = collect_words(out_words, lane);
+    if (lane < 4 * kUnroll && (kUnroll * 128) * warp + 32 * lane < tile.count)
+        P.sbits[word0 + 4 * kUnroll * warp + lane] = mine;
+    double t = 0.0;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) t += ss[u];
+    t = warp_sum(t);
+    if (lane == 0) red[warp] = t;
     __syncthreads();
     if (tid == 0) {
         double a = 0.0;
 #pragma unroll
         for (int k = 0; k < kWarps; ++k) a += red[k];
         P.partial[tile_id] = a;
-    }
-}
-
-// Server scale of chunk c = blockIdx.x (tensor c / W, server c % W):
-// s' = ||y over the chunk||_2 / sqrt(len), 0 for an empty chunk.
-__global__ void __launch_bounds__(kScaleThreads) ob_server_scale_kernel(
-    const double *partial, const int *chunk_tile_begin, const int64_t *chunk_len, float *sp_prev,
-    float *sp_last) {
-    __shared__ double smem[kScaleThreads / 32];
-    const int c = blockIdx.x;
-    const int lo = chunk_tile_begin[c], hi = chunk_tile_begin[c + 1];
-    double acc = 0.0;
-    for (int k = lo + (int)threadIdx.x; k < hi; k += kScaleThreads) acc += partial[k];
-    acc = block_sum(acc, smem);
-    if (threadIdx.x == 0) {
-        const int64_t len = chunk_len[c];
-        const float s = len > 0 ? __double2float_rn(__dsqrt_rn(__ddiv_rn(acc, (double)len))) : 0.0f;
-        sp_prev[c] = s;
-        sp_last[c] = s;
     }
 }
 

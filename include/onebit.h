@@ -98,9 +98,9 @@ typedef enum ob_kernel_id {
     OB_K_WARMUP = 0,          /* ob_warmup_adam_step */
     OB_K_FREEZE = 1,          /* ob_freeze_variance */
     OB_K_PACK = 2,            /* worker stage: momentum, error, signs, partial sums of squares */
-    OB_K_PACK_SCALE = 3,      /* worker scales from the partial sums */
+    OB_K_PACK_SCALE = 3,      /* worker scales from the partial sums (ob_scale_kernel) */
     OB_K_SERVER = 4,          /* server stage: average, server error, signs, partial sums */
-    OB_K_SERVER_SCALE = 5,    /* server chunk scales from the partial sums */
+    OB_K_SERVER_SCALE = 5,    /* server chunk scales from the partial sums (ob_scale_kernel) */
     OB_K_APPLY = 6,           /* gather, decode and preconditioned update */
     OB_NUM_KERNELS = 7
 } ob_kernel_id;

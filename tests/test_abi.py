@@ -37,8 +37,8 @@ def test_abi_version_and_status_strings():
         assert B.ob_status_string(code) == name
     assert B.ob_status_string(99) == "OB_UNKNOWN_STATUS"
     assert [B.ob_kernel_name(k) for k in range(B.OB_NUM_KERNELS)] == [
-        "ob_warmup_kernel", "ob_freeze_kernel", "ob_pack_kernel", "ob_pack_scale_kernel",
-        "ob_server_kernel", "ob_server_scale_kernel", "ob_apply_kernel"]
+        "ob_warmup_kernel", "ob_freeze_kernel", "ob_pack_kernel", "ob_scale_kernel:worker",
+        "ob_server_kernel", "ob_scale_kernel:server", "ob_apply_kernel"]
     assert B.ob_kernel_name(B.OB_NUM_KERNELS) is None
 
 

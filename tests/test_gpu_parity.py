@@ -36,6 +36,8 @@ CASES = {
     "flat-ragged-tail-W3": WL.flat(100_003, 3, 3, 5, seed=23),
     "flat-W5": WL.flat(40_000, 5, 2, 4, seed=24),
     "flat-W1": WL.flat(70_001, 1, 2, 4, seed=25),
+    # > 2048 tiles per tensor and per server chunk: multi-segment scale sums
+    "flat-multi-segment-W2": WL.flat((1 << 24) + 12_345, 2, 1, 2, seed=29),
 }
 
 
@@ -226,8 +228,8 @@ def test_profiling_counters():
         pr.compressed_step()
     prof = pr.gpu.profile_read(reset=True)
     assert prof["ob_warmup_kernel"][1] == 1 and prof["ob_freeze_kernel"][1] == 1
-    for k in ("ob_pack_kernel", "ob_pack_scale_kernel", "ob_server_kernel",
-              "ob_server_scale_kernel", "ob_apply_kernel"):
+    for k in ("ob_pack_kernel", "ob_scale_kernel:worker", "ob_server_kernel",
+              "ob_scale_kernel:server", "ob_apply_kernel"):
         assert prof[k][1] == 3 and prof[k][0] > 0, k
     assert all(v == (0.0, 0) for v in pr.gpu.profile_read().values())
     pr.close()
