@@ -180,10 +180,19 @@ class OracleRun:
     Per tensor t: p, m, v (then d), e_w[w], e_s; after each compressed step
     also the packed words and scales of that step.  All arrays are dense
     float32 / uint32 numpy arrays of the tensor's own length (no padding).
+
+    threads > 1 runs independent oracle calls concurrently (ctypes releases
+    the GIL): the worker stage of every (tensor, worker), the server stage
+    and update of every tensor, and slices of the elementwise warmup and
+    freeze.  Each call is still the plain single-threaded C function, so
+    the results do not depend on `threads`.
     """
 
+    SLICE = 1 << 22  # elements per warmup/freeze call when threaded
+
     def __init__(self, params: Sequence[np.ndarray], W: int, hp: dict,
-                 oracle: Optional[Oracle] = None):
+                 oracle: Optional[Oracle] = None, threads: int = 1):
+        self.threads = max(1, int(threads))
         self.o = oracle or default()
         self.W = int(W)
         self.hp = dict(hp)
@@ -205,17 +214,42 @@ class OracleRun:
     def T(self) -> int:
         return len(self.p)
 
+    def _run(self, jobs):
+        """Run independent zero-argument callables, concurrently if threaded."""
+        if self.threads == 1:
+            for j in jobs:
+                j()
+            return
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(self.threads) as ex:
+            for f in [ex.submit(j) for j in jobs]:
+                f.result()
+
+    def _slices(self, n: int):
+        step = self.SLICE if self.threads > 1 else max(1, n)
+        return [(a, min(n, a + step)) for a in range(0, n, step)] or [(0, 0)]
+
     def warmup_step(self, grads: Sequence[Sequence[np.ndarray]]) -> None:
         """grads[w][t]: worker w's gradient of tensor t."""
         assert self.d is None, "already frozen"
         self.t_warmup += 1
+        t_step = self.t_warmup
+        jobs = []
         for t in range(self.T):
-            self.o.adam_warmup_step(self.t_warmup, self.hp, [grads[w][t] for w in range(self.W)],
-                                    self.m[t], self.v[t], self.p[t])
+            for a, b in self._slices(self.numel[t]):
+                jobs.append(lambda t=t, a=a, b=b: self.o.adam_warmup_step(
+                    t_step, self.hp, [grads[w][t][a:b] for w in range(self.W)],
+                    self.m[t][a:b], self.v[t][a:b], self.p[t][a:b]))
+        self._run(jobs)
 
     def freeze(self) -> None:
         assert self.d is None and self.t_warmup >= 1
-        self.d = [self.o.freeze(self.t_warmup, self.hp, v) for v in self.v]
+        self.d = [np.empty_like(v) for v in self.v]
+
+        def job(t, a, b):
+            self.d[t][a:b] = self.o.freeze(self.t_warmup, self.hp, self.v[t][a:b])
+        self._run([lambda t=t, a=a, b=b: job(t, a, b)
+                   for t in range(self.T) for a, b in self._slices(self.numel[t])])
         for w in range(self.W):
             for t in range(self.T):
                 self.e_w[w][t][:] = 0
@@ -233,14 +267,19 @@ class OracleRun:
         self.s_w = np.zeros((W, T), np.float32)
         self.sbits = [None] * T
         self.s_srv = np.zeros((T, W), np.float32)
-        for t in range(T):
-            for w in range(W):
-                b, s = self.worker_stage(w, t, grads[w][t])
-                self.bits_w[w][t] = b
-                self.s_w[w, t] = s
+
+        def worker_job(t, w):
+            b, s = self.worker_stage(w, t, grads[w][t])
+            self.bits_w[w][t] = b
+            self.s_w[w, t] = s
+
+        def server_job(t):
             sb, ss = self.o.server_compress([self.bits_w[w][t] for w in range(W)], self.s_w[:, t],
                                             self.e_s[t])
             self.sbits[t] = sb
             self.s_srv[t] = ss
             self.o.apply_update(self.hp["lr"], sb, ss, self.d[t], self.p[t], self.m[t])
+
+        self._run([lambda t=t, w=w: worker_job(t, w) for t in range(T) for w in range(W)])
+        self._run([lambda t=t: server_job(t) for t in range(T)])
         self.t_compressed += 1

@@ -40,7 +40,7 @@ def words_of(flat_words: np.ndarray, offsets, numels):
 class Pair:
     """A GPU context and an oracle run over the same workload."""
 
-    def __init__(self, wl: WL.Workload, device="cuda"):
+    def __init__(self, wl: WL.Workload, device="cuda", threads: int = 1):
         self.wl = wl
         self.W = wl.W
         self.numels = wl.numels
@@ -50,7 +50,8 @@ class Pair:
         self.scale = WL.grad_scale_vector(wl, self.offsets, self.n_pad, device=self.dev)
         self.gpu = OneBitAdam(self.numels, wl.W, params=params.clone(), **WL.HYPER)
         self.orc = oracle.OracleRun(WL.split(params.cpu().numpy(), self.offsets, self.numels), wl.W,
-                                    WL.HYPER)
+                                    WL.HYPER, threads=threads)
+        del params
         self.grads = torch.empty((wl.W, self.n_pad), dtype=torch.float32, device=self.dev)
         self.step_index = 0
 
@@ -159,13 +160,13 @@ class Pair:
 
 
 def run_schedule(wl: WL.Workload, synced: bool, warmup: Optional[int] = None,
-                 compressed: Optional[int] = None):
+                 compressed: Optional[int] = None, threads: int = 1):
     """Warmup (checked bit for bit every step), freeze (bit for bit), then
     compressed steps: re-synced from the oracle before each step, or left to
     run free.  Returns (pair, list of per-step 'scales exact' flags)."""
     warmup = wl.warmup_steps if warmup is None else warmup
     compressed = wl.compressed_steps if compressed is None else compressed
-    pr = Pair(wl)
+    pr = Pair(wl, threads=threads)
     for _ in range(warmup):
         pr.warmup_step()
         pr.check_warmup_exact()
