@@ -88,13 +88,23 @@ __device__ __forceinline__ void set(float4 &v, int k, float f) {
     if (k == 0) v.x = f; else if (k == 1) v.y = f; else if (k == 2) v.z = f; else v.w = f;
 }
 
-// Streaming 16-byte accesses: every byte is touched once per step, so mark
-// the lines evict-first and keep L2 for the packed words and scales.
+// Streaming 16-byte accesses: every byte is touched once per step, so the
+// lines are marked evict-first (.cs), keeping L2 for the packed words and
+// scales.  The load is a plain (non-volatile, no memory clobber) asm, so the
+// compiler may issue a thread's later loads before its earlier stores; that
+// is correct because no kernel here loads an address after the same thread
+// stored to it (each element is read, then written once, the store
+// depending on the load).
 __device__ __forceinline__ float4 ld_stream(const float *p) {
-    return __ldcs(reinterpret_cast<const float4 *>(p));
+    float4 v;
+    asm("ld.global.cs.v4.f32 {%0, %1, %2, %3}, [%4];"
+        : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+        : "l"(p));
+    return v;
 }
 __device__ __forceinline__ void st_stream(float *p, const float4 &v) {
-    __stcs(reinterpret_cast<float4 *>(p), v);
+    asm volatile("st.global.cs.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w));
 }
 
 // Asynchronous 16-byte global -> shared copies (sm_80+ LDGSTS), with an L2
