@@ -65,6 +65,29 @@ def algorithmic_bytes(n_real: int, W: int) -> dict:
             "step": pack + server + apply, "model": n_real * (12 * W + W / 4 + 28.25)}
 
 
+def kernel_source_sha256() -> str:
+    import hashlib
+    path = os.path.join(ROOT, "error_compensated_bit_adam_b200", "csrc", "onebit_kernels.cuh")
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def measured_traffic(kernel: str, n: int, W: int):
+    """DRAM bytes per launch of `kernel` from the ncu capture recorded in
+    profiles/ncu_traffic.json, scaled to n parameters; None when no capture
+    exists for this W or the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    entry = rec.get("kernels", {}).get(kernel)
+    if not entry or rec.get("kernels_sha256") != kernel_source_sha256() or entry.get("W") != W:
+        return None
+    return entry["dram_bytes_per_param"] * n
+
+
 def measured_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -350,7 +373,8 @@ def run_b200(args) -> None:
             "hbm_frac_of_8tbs_effective_dense_model": model_gbs / NOMINAL_HBM_GBS,
             "roofline": {"bound": "hbm", "kernel": "ob_pack_kernel", "achieved": achieved,
                          "peak": peak["hbm_gbs"], "peak_source": peak["source"], "unit": "GB/s",
-                         "frac": achieved / peak["hbm_gbs"], "traffic": args.pack_traffic,
+                         "frac": achieved / peak["hbm_gbs"],
+                         "traffic": measured_traffic("ob_pack_kernel", wl.n, wl.W),
                          "algorithmic_bytes_per_launch": algo["ob_pack_kernel"],
                          "avg_launch_ms": pack_avg_s * 1e3},
             "kernels": per_kernel,
@@ -379,8 +403,6 @@ def main(argv=None):
     ap.add_argument("--adam-steps", type=int, default=None, help="override warmup Adam steps")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--pack-traffic", type=float, default=None,
-                    help="ncu DRAM bytes per ob_pack_kernel launch at this workload, if measured")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "b200" and not args.n:
         ap.error("--warmup must be >= 3")
