@@ -244,6 +244,13 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def replica_throughput(n_per_replica: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job parameters updated per second per simulated worker: every
+    rank updates its own replica of n parameters each step, and the step
+    time is the slowest rank's."""
+    return world * n_per_replica / (ms_per_step_max / 1e3)
+
+
 def barrier(world: int) -> None:
     if world > 1:
         import torch.distributed as dist
@@ -359,7 +366,7 @@ def run_b200(args) -> None:
         cpu = cpu_baseline(wl.W)
 
     if rank == 0:
-        value = world * wl.n / (ms_per_step / 1e3)
+        value = replica_throughput(wl.n, world, ms_per_step)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
