@@ -504,39 +504,39 @@ struct ServerParams {
     int w_pow2;
 };
 
+// Two independent IEEE round-to-nearest additions in one instruction
+// (packed fp32 pair, sm_100a): (a0, a1) += (b0, b1), each lane exactly
+// __fadd_rn.
+__device__ __forceinline__ void add2_rn(float &a0, float &a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb;\n\tmov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+        "add.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(b0), "f"(b1));
+}
+
 // [1BA, Proposed method, 3-4]: server j = tile.chunk receives every
 // worker's words for its chunk (addressed in place: the exchange is an
 // index into [W][words]) and forms
 //   y = (sum over w in order of sign_w s_w) / W + e_s,
 // with e_s decoded from (y_prev, s'_prev); then the sign bits of y and the
-// tile's partial sum of y^2.  The W workers' words of the tile are first
-// staged in shared memory with one 16-byte load per thread, so the W-long
-// sequential sum never waits on global memory.
-__global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_constant__ ServerParams P) {
-    extern __shared__ uint4 staged[];  // [W][kTileWords / 4]
-    __shared__ double red[kWarps];
-    __shared__ uint32_t scale_bits[OB_MAX_WORKERS];
-    const int tile_id = blockIdx.x;
-    const Tile tile = P.tiles[tile_id];
+// tile's partial sum of y^2.  The tile's W word rows are staged in shared
+// memory with one 16-byte load per thread, so the W-long sequential sum
+// never waits on global memory.  FULL tiles (all 4096 elements real, the
+// rule) skip every per-element bound check.
+template <bool FULL>
+__device__ __forceinline__ void server_tile(const ServerParams &P, const Tile &tile, int tile_id,
+                                            const uint4 *staged, const uint32_t *scale_bits,
+                                            double *red) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t words_per_worker = P.n_pad >> 5;
     const int64_t word0 = tile.begin >> 5;
-    const int groups = (((tile.count + 31) >> 5) + 3) >> 2;  // 16-byte word groups with real elements
-
-    for (int idx = tid; idx < P.W * (kTileWords / 4); idx += kThreads) {
-        const int w = idx / (kTileWords / 4), q = idx % (kTileWords / 4);
-        if (q < groups)
-            staged[idx] = __ldcs(reinterpret_cast<const uint4 *>(P.bits + w * words_per_worker + word0) + q);
-    }
-    if (tid < P.W) scale_bits[tid] = __float_as_uint(P.s_w[tid * P.T + tile.tensor]);
 
     float4 yo[kUnroll];
     int real[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
         const int off = span_off(warp, lane, u);
-        real[u] = slot_real(tile.count, off);
-        yo[u] = real[u] > 0 ? ld_stream(P.y + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+        real[u] = FULL ? 4 : slot_real(tile.count, off);
+        yo[u] = (FULL || real[u] > 0) ? ld_stream(P.y + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     __syncthreads();
 
@@ -547,6 +547,7 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
     for (int u = 0; u < kUnroll; ++u)
 #pragma unroll
         for (int k = 0; k < 4; ++k) acc[u][k] = 0.0f;
+#pragma unroll 4
     for (int w = 0; w < P.W; ++w) {
         const uint32_t sb = scale_bits[w];
 #pragma unroll
@@ -554,10 +555,12 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
             // this lane's 4 bits, inverted, at bits 0..3: element k's sign
             // bit is then (inv << (31 - k)) & 0x80000000 (a constant shift)
             const uint32_t inv = ~(words[w * kTileWords + (span_off(warp, lane, u) >> 5)] >> shift);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                acc[u][k] = __fadd_rn(acc[u][k],
-                                      __uint_as_float(((inv << (31 - k)) & 0x80000000u) | sb));
+            const float v0 = __uint_as_float(((inv << 31) & 0x80000000u) | sb);
+            const float v1 = __uint_as_float(((inv << 30) & 0x80000000u) | sb);
+            const float v2 = __uint_as_float(((inv << 29) & 0x80000000u) | sb);
+            const float v3 = __uint_as_float(((inv << 28) & 0x80000000u) | sb);
+            add2_rn(acc[u][0], acc[u][1], v0, v1);
+            add2_rn(acc[u][2], acc[u][3], v2, v3);
         }
     }
 
@@ -570,11 +573,11 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
         const int off = span_off(warp, lane, u);
         uint32_t nibble = 0;
         ss[u] = 0.0;
-        if (real[u] > 0) {
+        if (FULL || real[u] > 0) {
             float4 yn = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                if (k < real[u]) {
+                if (FULL || k < real[u]) {
                     const float avg = P.w_pow2 ? __fmul_rn(acc[u][k], P.inv_w) : __fdiv_rn(acc[u][k], wf);
                     const float y = __fadd_rn(avg, decode_error(get(yo[u], k), sp));
                     ss[u] = __fma_rn((double)y, (double)y, ss[u]);
@@ -587,7 +590,7 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
         out_words[u] = gather_word(nibble, lane);
     }
     const uint32_t mine = collect_words(out_words, lane);
-    if (lane < 4 * kUnroll && (kUnroll * 128) * warp + 32 * lane < tile.count)
+    if (lane < 4 * kUnroll && (FULL || (kUnroll * 128) * warp + 32 * lane < tile.count))
         P.sbits[word0 + 4 * kUnroll * warp + lane] = mine;
     double t = 0.0;
 #pragma unroll
@@ -601,6 +604,29 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
         for (int k = 0; k < kWarps; ++k) a += red[k];
         P.partial[tile_id] = a;
     }
+}
+
+__global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_constant__ ServerParams P) {
+    extern __shared__ uint4 staged[];  // [W][kTileWords / 4]
+    __shared__ double red[kWarps];
+    __shared__ uint32_t scale_bits[OB_MAX_WORKERS];
+    const int tile_id = blockIdx.x;
+    const Tile tile = P.tiles[tile_id];
+    const int tid = threadIdx.x;
+    const int64_t words_per_worker = P.n_pad >> 5;
+    const int64_t word0 = tile.begin >> 5;
+    const int groups = (((tile.count + 31) >> 5) + 3) >> 2;  // 16-byte word groups with real elements
+
+    for (int idx = tid; idx < P.W * (kTileWords / 4); idx += kThreads) {
+        const int w = idx / (kTileWords / 4), q = idx % (kTileWords / 4);
+        if (q < groups)
+            staged[idx] = __ldcs(reinterpret_cast<const uint4 *>(P.bits + w * words_per_worker + word0) + q);
+    }
+    if (tid < P.W) scale_bits[tid] = __float_as_uint(P.s_w[tid * P.T + tile.tensor]);
+    if (tile.count == kTile)
+        server_tile<true>(P, tile, tile_id, staged, scale_bits, red);
+    else
+        server_tile<false>(P, tile, tile_id, staged, scale_bits, red);
 }
 
 // ------------------------------------------------------ gather and update
@@ -620,16 +646,16 @@ struct ApplyParams {
 // words, m_hat = sign' s'_j, and takes a momentum SGD step preconditioned by
 // the frozen denominator: p -= lr (m_hat / d); m = m_hat (m is left as the
 // words and scales themselves unless a dense copy is asked for).
-__global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constant__ ApplyParams P) {
-    const Tile tile = P.tiles[blockIdx.x];
+template <bool FULL>
+__device__ __forceinline__ void apply_tile(const ApplyParams &P, const Tile &tile) {
     const int tid = threadIdx.x, lane = tid & 31;
     const uint32_t sb = __float_as_uint(P.sp[tile.tensor * P.W + tile.chunk]);
     const int shift = 4 * (lane & 7);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
         const int off = 4 * (tid + kThreads * u);
-        const int real = slot_real(tile.count, off);
-        if (real == 0) continue;
+        const int real = FULL ? 4 : slot_real(tile.count, off);
+        if (!FULL && real == 0) continue;
         const int64_t i = tile.begin + off;
         const uint32_t inv = ~(__ldg(P.sbits + (i >> 5)) >> shift);
         const float4 d = ld_stream(P.d + i);
@@ -637,7 +663,7 @@ __global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constan
         float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            if (k < real) {
+            if (FULL || k < real) {
                 const float m_hat = __uint_as_float(((inv << (31 - k)) & 0x80000000u) | sb);
                 const float delta = __fmul_rn(P.lr, __fdiv_rn(m_hat, get(d, k)));
                 set(p, k, __fsub_rn(get(p, k), delta));
@@ -647,6 +673,14 @@ __global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constan
         st_stream(P.p + i, p);
         if (P.m) st_stream(P.m + i, m);
     }
+}
+
+__global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constant__ ApplyParams P) {
+    const Tile tile = P.tiles[blockIdx.x];
+    if (tile.count == kTile)
+        apply_tile<true>(P, tile);
+    else
+        apply_tile<false>(P, tile);
 }
 
 // ------------------------------------------------- state decode for reads
