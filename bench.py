@@ -65,27 +65,29 @@ def algorithmic_bytes(n_real: int, W: int) -> dict:
             "step": pack + server + apply, "model": n_real * (12 * W + W / 4 + 28.25)}
 
 
-def kernel_source_sha256() -> str:
+def kernel_sources_sha256(files) -> str:
     import hashlib
-    path = os.path.join(ROOT, "error_compensated_bit_adam_b200", "csrc", "onebit_kernels.cuh")
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "error_compensated_bit_adam_b200", "csrc", "kernels", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
 def measured_traffic(kernel: str, n: int, W: int):
     """DRAM bytes per launch of `kernel` from the ncu capture recorded in
     profiles/ncu_traffic.json, scaled to n parameters; None when no capture
-    exists for this W or the kernels changed since it was taken."""
+    exists for this W or the kernel's sources changed since it was taken."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
+        entry = rec["kernels"][kernel]
+        if entry["W"] != W or kernel_sources_sha256(entry["sources"]) != entry["sources_sha256"]:
+            return None
+        return entry["dram_bytes_per_param"] * n
     except Exception:
         return None
-    entry = rec.get("kernels", {}).get(kernel)
-    if not entry or rec.get("kernels_sha256") != kernel_source_sha256() or entry.get("W") != W:
-        return None
-    return entry["dram_bytes_per_param"] * n
 
 
 def measured_peaks() -> dict:

@@ -16,7 +16,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 SOURCES = [os.path.join(CSRC, "onebit.cu")]
-DEPENDS = SOURCES + [os.path.join(CSRC, "onebit_kernels.cuh"), os.path.join(ROOT, "include", "onebit.h")]
+DEPENDS = SOURCES + [os.path.join(CSRC, "onebit_kernels.cuh"), os.path.join(ROOT, "include", "onebit.h")] + [
+    os.path.join(CSRC, "kernels", f) for f in sorted(os.listdir(os.path.join(CSRC, "kernels")))]
 LIBRARY = os.path.join(HERE, "libonebit.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

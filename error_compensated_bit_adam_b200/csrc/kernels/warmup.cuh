@@ -1,0 +1,80 @@
+// kernels/warmup.cuh -- Warmup Adam step and the variance freeze.
+//
+// Part of libonebit (sm_100a); see onebit_kernels.cuh for the overview.
+#pragma once
+
+#include "common.cuh"
+
+namespace onebit {
+
+// ------------------------------------------------------------ warmup Adam
+
+struct WarmupParams {
+    const Tile *tiles;
+    const float *g[OB_MAX_WORKERS];  // worker gradients, padded layout
+    float *m, *v, *p;
+    int W;
+    float beta1, beta2, c1, c2, bc1, bc2, eps, lr;
+};
+
+// [1BA, Proposed method, 1]: one full-precision Adam step on the averaged
+// gradient, elementwise.
+__global__ void __launch_bounds__(kThreads) ob_warmup_kernel(const __grid_constant__ WarmupParams P) {
+    const Tile tile = P.tiles[blockIdx.x];
+    const float wf = (float)P.W;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * ((int)threadIdx.x + kThreads * u);
+        const int real = slot_real(tile.count, off);
+        if (real == 0) continue;
+        const int64_t i = tile.begin + off;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int w = 0; w < P.W; ++w) {
+            const float4 g = ld_stream(P.g[w] + i);
+            acc.x = __fadd_rn(acc.x, g.x);
+            acc.y = __fadd_rn(acc.y, g.y);
+            acc.z = __fadd_rn(acc.z, g.z);
+            acc.w = __fadd_rn(acc.w, g.w);
+        }
+        float4 m = ld_stream(P.m + i), v = ld_stream(P.v + i), p = ld_stream(P.p + i);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (k >= real) break;  // padding keeps its values
+            const float gbar = __fdiv_rn(get(acc, k), wf);
+            const float mk = __fadd_rn(__fmul_rn(P.beta1, get(m, k)), __fmul_rn(P.c1, gbar));
+            const float vk = __fadd_rn(__fmul_rn(P.beta2, get(v, k)),
+                                       __fmul_rn(P.c2, __fmul_rn(gbar, gbar)));
+            const float mhat = __fdiv_rn(mk, P.bc1);
+            const float vhat = __fdiv_rn(vk, P.bc2);
+            const float denom = __fadd_rn(__fsqrt_rn(vhat), P.eps);
+            const float delta = __fmul_rn(P.lr, __fdiv_rn(mhat, denom));
+            set(m, k, mk);
+            set(v, k, vk);
+            set(p, k, __fsub_rn(get(p, k), delta));
+        }
+        st_stream(P.m + i, m);
+        st_stream(P.v + i, v);
+        st_stream(P.p + i, p);
+    }
+}
+
+// ----------------------------------------------------------------- freeze
+
+// [1BA, Abstract; Proposed method, 2]: d = sqrt(v / bc2) + eps, in place.
+__global__ void __launch_bounds__(kThreads) ob_freeze_kernel(const Tile *tiles, float *v, float bc2,
+                                                             float eps) {
+    const Tile tile = tiles[blockIdx.x];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * ((int)threadIdx.x + kThreads * u);
+        const int real = slot_real(tile.count, off);
+        if (real == 0) continue;
+        float4 x = ld_stream(v + tile.begin + off);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            if (k < real) set(x, k, __fadd_rn(__fsqrt_rn(__fdiv_rn(get(x, k), bc2)), eps));
+        st_stream(v + tile.begin + off, x);
+    }
+}
+
+}  // namespace onebit
