@@ -168,10 +168,10 @@ def pick_workload(args) -> WL.Workload:
     return wl
 
 
-def workload_config(wl: WL.Workload, n_pad: int, parallelism: str) -> dict:
+def workload_config(wl: WL.Workload, n_pad: int, parallelism: str, grad_sets: int = GRAD_SETS) -> dict:
     return {"workload": wl.describe(), "n": wl.n, "n_padded": n_pad, "W": wl.W,
             "tensors": wl.n_tensors, "adam_warmup_steps": wl.warmup_steps,
-            "grad_sets_cycled": GRAD_SETS,
+            "grad_sets_cycled": grad_sets,
             "l2": f"inputs larger than L2: {4 * wl.W * n_pad / 1e9:.2f} GB of gradients per step",
             "parallelism": parallelism}
 
@@ -259,6 +259,35 @@ def barrier(world: int) -> None:
         dist.barrier()
 
 
+def measure_e2e(opt, wl, n_pad, dev_grads, args, world, dev) -> dict:
+    """The step through the public host-buffer call: every step copies W
+    gradient vectors from pinned host memory to the GPU (overlapped with the
+    worker stage) and reads the step's server scales back."""
+    try:
+        e2e_steps = max(1, min(args.steps, args.e2e_steps))
+        try:
+            host = torch.empty((wl.W, n_pad), dtype=torch.float32, pin_memory=True)
+            pinned = True
+        except RuntimeError:
+            host = torch.empty((wl.W, n_pad), dtype=torch.float32)
+            pinned = False
+        host.copy_(dev_grads)
+        out = np.zeros(wl.n_tensors * wl.W, np.float32)
+        opt.step_host(host, out)                    # untimed: staging allocation
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        w0 = time.perf_counter()
+        for _ in range(e2e_steps):
+            opt.step_host(host, out)
+        e2e_s = max_over_ranks(time.perf_counter() - w0, world) / e2e_steps
+        return {"value": world * wl.n / e2e_s, "unit": UNIT,
+                "h2d_bytes_per_step": int(host.numel() * 4), "d2h_bytes_per_step": int(out.nbytes),
+                "ms_per_step": e2e_s * 1e3, "pinned": pinned, "steps": e2e_steps,
+                "call": "ob_compressed_step_host"}
+    except Exception as exc:  # reported, never hidden
+        return {"value": None, "unit": UNIT, "error": repr(exc)}
+
+
 def run_b200(args) -> None:
     from error_compensated_bit_adam_b200.optimizer import OneBitAdam
 
@@ -280,7 +309,10 @@ def run_b200(args) -> None:
     params = WL.make_params(wl, offsets, n_pad, device=dev)
     scale = WL.grad_scale_vector(wl, offsets, n_pad, device=dev)
     opt = OneBitAdam(wl.numels, wl.W, params=params, device=dev, **WL.HYPER)
-    grads = [torch.empty((wl.W, n_pad), dtype=torch.float32, device=dev) for _ in range(GRAD_SETS)]
+    set_bytes = 4 * wl.W * n_pad
+    free_bytes = torch.cuda.mem_get_info(dev)[0]
+    n_sets = GRAD_SETS if free_bytes > GRAD_SETS * set_bytes + 2 * 4 * n_pad + (1 << 30) else 1
+    grads = [torch.empty((wl.W, n_pad), dtype=torch.float32, device=dev) for _ in range(n_sets)]
 
     step = 0
     for _ in range(wl.warmup_steps):           # full-precision Adam warmup, untimed
@@ -293,7 +325,7 @@ def run_b200(args) -> None:
         step += 1
     del scale
     for k in range(args.warmup):               # untimed compressed steps
-        opt.step(grads[k % GRAD_SETS])
+        opt.step(grads[k % n_sets])
     torch.cuda.synchronize(dev)
 
     stream = opt.stream
@@ -307,7 +339,7 @@ def run_b200(args) -> None:
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for k in range(args.steps):
-        opt.step(grads[k % GRAD_SETS])
+        opt.step(grads[k % n_sets])
     t1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
@@ -337,31 +369,8 @@ def run_b200(args) -> None:
 
     # end to end: host gradients in pinned memory, copied in every step, and
     # the step's server scales read back, through ob_compressed_step_host
-    e2e = None
-    try:
-        e2e_steps = max(1, min(args.steps, args.e2e_steps))
-        try:
-            host = torch.empty((wl.W, n_pad), dtype=torch.float32, pin_memory=True)
-            pinned = True
-        except RuntimeError:
-            host = torch.empty((wl.W, n_pad), dtype=torch.float32)
-            pinned = False
-        host.copy_(grads[0])
-        out = np.zeros(wl.n_tensors * wl.W, np.float32)
-        opt.step_host(host, out)                    # untimed: staging allocation
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        w0 = time.perf_counter()
-        for _ in range(e2e_steps):
-            opt.step_host(host, out)
-        e2e_s = max_over_ranks(time.perf_counter() - w0, world) / e2e_steps
-        e2e = {"value": world * wl.n / e2e_s, "unit": UNIT,
-               "h2d_bytes_per_step": int(host.numel() * 4), "d2h_bytes_per_step": int(out.nbytes),
-               "ms_per_step": e2e_s * 1e3, "pinned": pinned, "steps": e2e_steps,
-               "call": "ob_compressed_step_host"}
-        del host
-    except Exception as exc:  # reported, never hidden
-        e2e = {"value": None, "unit": UNIT, "error": repr(exc)}
+    e2e = ({"value": None, "unit": UNIT, "skipped": "--no-e2e"} if args.no_e2e
+           else measure_e2e(opt, wl, n_pad, grads[0], args, world, dev))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -373,7 +382,7 @@ def run_b200(args) -> None:
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(wl, n_pad, "replicas" if world > 1 else "single GPU"),
+            "config": workload_config(wl, n_pad, "replicas" if world > 1 else "single GPU", n_sets),
             "params_per_s_aggregate_all_workers": value * wl.W,
             "hbm_gbs_step": step_gbs,
             "hbm_frac_of_measured_peak_step": step_gbs / peak["hbm_gbs"],
@@ -412,6 +421,7 @@ def main(argv=None):
     ap.add_argument("--adam-steps", type=int, default=None, help="override warmup Adam steps")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-gradient end-to-end leg")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "b200" and not args.n:
         ap.error("--warmup must be >= 3")
