@@ -40,17 +40,18 @@ def words_of(flat_words: np.ndarray, offsets, numels):
 class Pair:
     """A GPU context and an oracle run over the same workload."""
 
-    def __init__(self, wl: WL.Workload, device="cuda", threads: int = 1):
+    def __init__(self, wl: WL.Workload, device="cuda", threads: int = 1, hp: Optional[dict] = None):
         self.wl = wl
+        self.hp = dict(hp or WL.HYPER)
         self.W = wl.W
         self.numels = wl.numels
         self.offsets, self.n_pad = B.ob_layout(self.numels)
         self.dev = torch.device(device)
         params = WL.make_params(wl, self.offsets, self.n_pad, device=self.dev)
         self.scale = WL.grad_scale_vector(wl, self.offsets, self.n_pad, device=self.dev)
-        self.gpu = OneBitAdam(self.numels, wl.W, params=params.clone(), **WL.HYPER)
+        self.gpu = OneBitAdam(self.numels, wl.W, params=params.clone(), **self.hp)
         self.orc = oracle.OracleRun(WL.split(params.cpu().numpy(), self.offsets, self.numels), wl.W,
-                                    WL.HYPER, threads=threads)
+                                    self.hp, threads=threads)
         del params
         self.grads = torch.empty((wl.W, self.n_pad), dtype=torch.float32, device=self.dev)
         self.step_index = 0
@@ -160,13 +161,13 @@ class Pair:
 
 
 def run_schedule(wl: WL.Workload, synced: bool, warmup: Optional[int] = None,
-                 compressed: Optional[int] = None, threads: int = 1):
+                 compressed: Optional[int] = None, threads: int = 1, hp: Optional[dict] = None):
     """Warmup (checked bit for bit every step), freeze (bit for bit), then
     compressed steps: re-synced from the oracle before each step, or left to
     run free.  Returns (pair, list of per-step 'scales exact' flags)."""
     warmup = wl.warmup_steps if warmup is None else warmup
     compressed = wl.compressed_steps if compressed is None else compressed
-    pr = Pair(wl, threads=threads)
+    pr = Pair(wl, threads=threads, hp=hp)
     for _ in range(warmup):
         pr.warmup_step()
         pr.check_warmup_exact()

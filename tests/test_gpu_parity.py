@@ -233,3 +233,60 @@ def test_profiling_counters():
         assert prof[k][1] == 3 and prof[k][0] > 0, k
     assert all(v == (0.0, 0) for v in pr.gpu.profile_read().values())
     pr.close()
+
+
+@pytest.mark.parametrize("hp", [dict(beta1=0.95, beta2=0.98, eps=1e-6, lr=3e-3),
+                                dict(beta1=0.5, beta2=0.9, eps=1e-4, lr=0.05)],
+                         ids=["b0.95-b0.98", "b0.5-b0.9"])
+def test_other_hyperparameters(hp):
+    wl = small_ragged(W=4, count=40)
+    pr, flags = run_schedule(wl, synced=True, hp=hp)
+    pr.close()
+    pr, flags = run_schedule(wl, synced=False, hp=hp)
+    try:
+        assert pr.params_rel_l2() <= PARAM_TOL
+    finally:
+        pr.close()
+
+
+def test_bucketed_contexts_on_two_streams_match_sequential():
+    """Two parameter buckets, each its own context on its own stream (the
+    way a trainer overlaps optimizer steps with backward), stepping
+    concurrently, end bit-identical to the same buckets stepped one after
+    the other."""
+    buckets = [small_ragged(W=4, count=30), WL.flat(300_001, 4, 2, 3, seed=31)]
+    dev = torch.device("cuda")
+
+    def run(concurrent):
+        streams = [torch.cuda.Stream() for _ in buckets]
+        opts, grads = [], []
+        for wl, st in zip(buckets, streams):
+            offs, n_pad = B.ob_layout(wl.numels)
+            params = WL.make_params(wl, offs, n_pad, device=dev)
+            scale = WL.grad_scale_vector(wl, offs, n_pad, device=dev)
+            g = torch.empty((wl.W, n_pad), device=dev)
+            WL.fill_grads(wl, 0, scale, g)
+            torch.cuda.synchronize()
+            opts.append(OneBitAdam(wl.numels, wl.W, params=params, stream=st, **WL.HYPER))
+            grads.append(g)
+        for o, g in zip(opts, grads):
+            o.warmup_step(g)
+            o.freeze()
+        for _ in range(4):
+            if concurrent:
+                for o, g in zip(opts, grads):
+                    o.step(g)          # queued on different streams, no sync in between
+            else:
+                for o, g in zip(opts, grads):
+                    o.step(g)
+                    torch.cuda.synchronize()
+        torch.cuda.synchronize()
+        out = [(o.read(B.OB_STATE_P), o.read(B.OB_STATE_BITS_SERVER), o.read(B.OB_STATE_E_WORKER, 1))
+               for o in opts]
+        for o in opts:
+            o.close()
+        return out
+
+    for a, b in zip(run(True), run(False)):
+        for x, y in zip(a, b):
+            assert np.array_equal(x.view(np.uint8), y.view(np.uint8))
