@@ -54,7 +54,7 @@ EXPORTS = (
     "ob_create", "ob_destroy", "ob_warmup_adam_step", "ob_freeze_variance", "ob_compressed_step",
     "ob_host_staging_bytes", "ob_compressed_step_host", "ob_read_state", "ob_write_state",
     "ob_profile_enable", "ob_profile_read", "ob_kernel_name", "ob_test_fail_host_alloc",
-    "ob_onebit_compress_static",
+    "ob_onebit_compress_static", "ob_set_lr", "ob_graph_enable",
 )
 
 
@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
         "ob_kernel_name": (ctypes.c_char_p, [i32]),
         "ob_test_fail_host_alloc": (None, [i32]),
         "ob_onebit_compress_static": (i32, [vp, i64, vp, vp, vp, vp]),
+        "ob_set_lr": (i32, [vp, f32]),
+        "ob_graph_enable": (i32, [vp, i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -226,6 +228,14 @@ def ob_read_state(ctx: int, kind: int, index: int, host_dst: int, nbytes: int) -
 def ob_write_state(ctx: int, kind: int, index: int, host_src: int, nbytes: int) -> None:
     _check(lib().ob_write_state(ctx, int(kind), int(index), int(host_src), int(nbytes)),
            "ob_write_state")
+
+
+def ob_set_lr(ctx: int, lr: float) -> None:
+    _check(lib().ob_set_lr(ctx, float(lr)), "ob_set_lr")
+
+
+def ob_graph_enable(ctx: int, on: bool) -> None:
+    _check(lib().ob_graph_enable(ctx, 1 if on else 0), "ob_graph_enable")
 
 
 def ob_profile_enable(ctx: int, on: bool) -> None:

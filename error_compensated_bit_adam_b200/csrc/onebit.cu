@@ -268,6 +268,16 @@ const char *const kKernelNames[OB_NUM_KERNELS] = {
 
 // ------------------------------------------------------------------ ctx
 
+// A compressed step recorded as a CUDA graph (graph mode).
+struct StepGraph {
+    bool built = false;
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    cudaGraphNode_t pack_node = nullptr, apply_node = nullptr;
+    onebit::PackParams pack{};   // parameters last written into the nodes
+    onebit::ApplyParams apply{};
+};
+
 struct ob_ctx {
     uint64_t magic = kMagic;
     int device = 0;
@@ -287,6 +297,8 @@ struct ob_ctx {
     // m is held densely in the m region (after create / warmup / a write),
     // or, after a compressed step, only as the server words and scales.
     bool m_dense = true;
+    bool use_graph = false;
+    StepGraph graph;
     bool broken = false;
     // profiling
     bool profiling = false;
@@ -369,9 +381,15 @@ struct KernelTimer {
 
 dim3 grid1(int n) { return dim3((unsigned)n); }
 
-ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int tile_lo, int tile_hi) {
-    if (tile_hi <= tile_lo) return OB_OK;
-    onebit::PackParams P;
+// ---------------------------------------------------------------- launches
+//
+// The five kernels of a compressed step, each with its parameters built by
+// one function, so direct launches and the CUDA-graph nodes of graph mode
+// are the same launches.
+
+onebit::PackParams pack_params(const ob_ctx *c, const float *const *g, int64_t g_offset,
+                               int tile_lo) {
+    onebit::PackParams P{};  // zeroed, padding too: compared bytewise in graph mode
     P.tiles = c->tiles();
     P.tile_base = tile_lo;
     P.n_tiles = c->n_tiles();
@@ -390,96 +408,232 @@ ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int ti
     P.T = c->plan.T;
     P.beta1 = c->beta1;
     P.c1 = c->c1;
-    onebit::ob_pack_kernel<<<grid1(tile_hi - tile_lo), kThreads, onebit::kPackSmemBytes, c->stream>>>(P);
+    return P;
+}
+
+onebit::ScaleParams worker_scale_params(const ob_ctx *c) {
+    onebit::ScaleParams P{};  // zeroed, padding too: compared bytewise in graph mode
+    P.partial = c->partial_w();
+    P.n_tiles = c->n_tiles();
+    P.range_begin = c->tensor_tile_begin();
+    P.seg_base = c->tensor_seg_base();
+    P.count = c->numel();
+    P.seg = c->seg_w();
+    P.counter = c->counters_w();
+    P.out_prev = c->s_prev();
+    P.out_last = c->s_last();
+    P.rows = c->plan.W;
+    P.R = c->plan.T;
+    P.out_stride_r = 1;
+    P.out_stride_row = c->plan.T;
+    return P;
+}
+
+onebit::ServerParams server_params(const ob_ctx *c) {
+    const int W = c->plan.W;
+    onebit::ServerParams P{};  // zeroed, padding too: compared bytewise in graph mode
+    P.tiles = c->tiles();
+    P.bits = c->bits();
+    P.s_w = c->s_prev();
+    P.y = c->y();
+    P.sp_prev = c->sp_prev();
+    P.sbits = c->sbits();
+    P.partial = c->partial_s();
+    P.n_pad = c->plan.n_pad;
+    P.W = W;
+    P.T = c->plan.T;
+    P.w_pow2 = (W & (W - 1)) == 0;
+    P.inv_w = 1.0f / (float)W;  // exact for a power of two
+    return P;
+}
+
+onebit::ScaleParams server_scale_params(const ob_ctx *c) {
+    onebit::ScaleParams P{};  // zeroed, padding too: compared bytewise in graph mode
+    P.partial = c->partial_s();
+    P.n_tiles = c->n_tiles();
+    P.range_begin = c->chunk_tile_begin();
+    P.seg_base = c->chunk_seg_base();
+    P.count = c->chunk_len();
+    P.seg = c->seg_s();
+    P.counter = c->counters_s();
+    P.out_prev = c->sp_prev();
+    P.out_last = c->sp_last();
+    P.rows = 1;
+    P.R = c->plan.T * c->plan.W;
+    P.out_stride_r = 1;
+    P.out_stride_row = 0;
+    return P;
+}
+
+onebit::ApplyParams apply_params(const ob_ctx *c) {
+    onebit::ApplyParams P{};  // zeroed, padding too: compared bytewise in graph mode
+    P.tiles = c->tiles();
+    P.sbits = c->sbits();
+    P.sp = c->sp_last();
+    P.d = c->v();
+    P.p = c->params;
+    P.m = nullptr;  // m stays as (sbits, sp_last); see ob_ctx::m_dense
+    P.W = c->plan.W;
+    P.lr = c->lr;
+    return P;
+}
+
+// Launch geometry of each kernel: grid, block, dynamic shared memory.
+struct Geometry {
+    dim3 grid, block;
+    size_t smem;
+};
+Geometry pack_geometry(int tiles) { return {grid1(tiles), dim3(kThreads), (size_t)onebit::kPackSmemBytes}; }
+Geometry worker_scale_geometry(const ob_ctx *c) {
+    return {dim3((unsigned)c->plan.T, (unsigned)c->plan.W, (unsigned)c->plan.tensor_max_seg),
+            dim3(kScaleThreads), 0};
+}
+Geometry server_geometry(const ob_ctx *c) {
+    return {grid1(c->n_tiles()), dim3(kThreads),
+            (size_t)c->plan.W * onebit::kTileWords * sizeof(uint32_t)};
+}
+Geometry server_scale_geometry(const ob_ctx *c) {
+    return {dim3((unsigned)(c->plan.T * c->plan.W), 1u, (unsigned)c->plan.chunk_max_seg),
+            dim3(kScaleThreads), 0};
+}
+Geometry apply_geometry(const ob_ctx *c) { return {grid1(c->n_tiles()), dim3(kThreads), 0}; }
+
+ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int tile_lo, int tile_hi) {
+    if (tile_hi <= tile_lo) return OB_OK;
+    const onebit::PackParams P = pack_params(c, g, g_offset, tile_lo);
+    const Geometry G = pack_geometry(tile_hi - tile_lo);
+    onebit::ob_pack_kernel<<<G.grid, G.block, G.smem, c->stream>>>(P);
     return fail_cuda(c, cudaGetLastError());
 }
 
 // Everything of a compressed step after the worker stage's tile kernels.
 ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
-    const int T = c->plan.T, W = c->plan.W, nt = c->n_tiles();
+    const int nt = c->n_tiles();
     pack_timer.stop();
     {
         KernelTimer k(c, OB_K_PACK_SCALE);
-        onebit::ScaleParams P;
-        P.partial = c->partial_w();
-        P.n_tiles = nt;
-        P.range_begin = c->tensor_tile_begin();
-        P.seg_base = c->tensor_seg_base();
-        P.count = c->numel();
-        P.seg = c->seg_w();
-        P.counter = c->counters_w();
-        P.out_prev = c->s_prev();
-        P.out_last = c->s_last();
-        P.rows = W;
-        P.R = T;
-        P.out_stride_r = 1;
-        P.out_stride_row = T;
-        onebit::ob_scale_kernel<<<dim3((unsigned)T, (unsigned)W, (unsigned)c->plan.tensor_max_seg),
-                                  kScaleThreads, 0, c->stream>>>(P);
+        const Geometry G = worker_scale_geometry(c);
+        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(worker_scale_params(c));
         k.stop();
         ob_status st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
     }
     if (nt > 0) {
         KernelTimer k(c, OB_K_SERVER);
-        onebit::ServerParams P;
-        P.tiles = c->tiles();
-        P.bits = c->bits();
-        P.s_w = c->s_prev();
-        P.y = c->y();
-        P.sp_prev = c->sp_prev();
-        P.sbits = c->sbits();
-        P.partial = c->partial_s();
-        P.n_pad = c->plan.n_pad;
-        P.W = W;
-        P.T = T;
-        P.w_pow2 = (W & (W - 1)) == 0;
-        P.inv_w = 1.0f / (float)W;  // exact for a power of two
-        const size_t smem = (size_t)W * onebit::kTileWords * sizeof(uint32_t);
-        onebit::ob_server_kernel<<<grid1(nt), kThreads, smem, c->stream>>>(P);
+        const Geometry G = server_geometry(c);
+        onebit::ob_server_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_params(c));
         k.stop();
         ob_status st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
     }
     {
         KernelTimer k(c, OB_K_SERVER_SCALE);
-        onebit::ScaleParams P;
-        P.partial = c->partial_s();
-        P.n_tiles = nt;
-        P.range_begin = c->chunk_tile_begin();
-        P.seg_base = c->chunk_seg_base();
-        P.count = c->chunk_len();
-        P.seg = c->seg_s();
-        P.counter = c->counters_s();
-        P.out_prev = c->sp_prev();
-        P.out_last = c->sp_last();
-        P.rows = 1;
-        P.R = T * W;
-        P.out_stride_r = 1;
-        P.out_stride_row = 0;
-        onebit::ob_scale_kernel<<<dim3((unsigned)(T * W), 1u, (unsigned)c->plan.chunk_max_seg),
-                                  kScaleThreads, 0, c->stream>>>(P);
+        const Geometry G = server_scale_geometry(c);
+        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_scale_params(c));
         k.stop();
         ob_status st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
     }
     if (nt > 0) {
         KernelTimer k(c, OB_K_APPLY);
-        onebit::ApplyParams P;
-        P.tiles = c->tiles();
-        P.sbits = c->sbits();
-        P.sp = c->sp_last();
-        P.d = c->v();
-        P.p = c->params;
-        P.m = nullptr;  // m stays as (sbits, sp_last); see ob_ctx::m_dense
-        P.W = W;
-        P.lr = c->lr;
-        onebit::ob_apply_kernel<<<grid1(nt), kThreads, 0, c->stream>>>(P);
+        const Geometry G = apply_geometry(c);
+        onebit::ob_apply_kernel<<<G.grid, G.block, G.smem, c->stream>>>(apply_params(c));
         k.stop();
         ob_status st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
     }
     return OB_OK;
+}
+
+// ------------------------------------------------------------- graph mode
+//
+// The step's kernels as one CUDA graph: a chain of kernel nodes built once
+// (lazily), replayed with one launch.  Parameters that change between
+// steps (gradient pointers, dense or lazy momentum, the learning rate) are
+// written into the instantiated graph's nodes before the replay.
+
+template <class Params>
+cudaKernelNodeParams node_params(void *func, const Geometry &G, Params *P, void **args) {
+    cudaKernelNodeParams kp{};
+    kp.func = func;
+    kp.gridDim = G.grid;
+    kp.blockDim = G.block;
+    kp.sharedMemBytes = (unsigned)G.smem;
+    args[0] = P;
+    kp.kernelParams = args;
+    kp.extra = nullptr;
+    return kp;
+}
+
+void destroy_graph(ob_ctx *c);
+
+ob_status build_graph(ob_ctx *c, const float *const *g) {
+    StepGraph &sg = c->graph;
+    cudaError_t e = cudaGraphCreate(&sg.graph, 0);
+    cudaGraphNode_t prev = nullptr;
+    auto add = [&](void *func, const Geometry &G, auto *P, cudaGraphNode_t *out) {
+        if (e != cudaSuccess) return;
+        void *args[1];
+        const cudaKernelNodeParams kp = node_params(func, G, P, args);
+        e = cudaGraphAddKernelNode(out, sg.graph, prev ? &prev : nullptr, prev ? 1 : 0, &kp);
+        if (e == cudaSuccess) prev = *out;
+    };
+    const int nt = c->n_tiles();
+    sg.pack = pack_params(c, g, 0, 0);
+    sg.apply = apply_params(c);
+    onebit::ScaleParams ws = worker_scale_params(c), ss = server_scale_params(c);
+    onebit::ServerParams sv = server_params(c);
+    cudaGraphNode_t n_ws, n_sv, n_ss;
+    if (nt > 0) add((void *)onebit::ob_pack_kernel, pack_geometry(nt), &sg.pack, &sg.pack_node);
+    add((void *)onebit::ob_scale_kernel, worker_scale_geometry(c), &ws, &n_ws);
+    if (nt > 0) add((void *)onebit::ob_server_kernel, server_geometry(c), &sv, &n_sv);
+    add((void *)onebit::ob_scale_kernel, server_scale_geometry(c), &ss, &n_ss);
+    if (nt > 0) add((void *)onebit::ob_apply_kernel, apply_geometry(c), &sg.apply, &sg.apply_node);
+    if (e == cudaSuccess) e = cudaGraphInstantiate(&sg.exec, sg.graph, 0);
+    if (e != cudaSuccess) {
+        destroy_graph(c);
+        return fail_cuda(c, e);
+    }
+    sg.built = true;
+    return OB_OK;
+}
+
+void destroy_graph(ob_ctx *c) {
+    StepGraph &sg = c->graph;
+    if (sg.exec) cudaGraphExecDestroy(sg.exec);
+    if (sg.graph) cudaGraphDestroy(sg.graph);
+    sg = StepGraph{};
+}
+
+// One compressed step through the graph.
+ob_status graph_step(ob_ctx *c, const float *const *g) {
+    StepGraph &sg = c->graph;
+    if (!sg.built) {
+        ob_status st = build_graph(c, g);
+        if (st != OB_OK) return st;
+    }
+    const int nt = c->n_tiles();
+    cudaError_t e = cudaSuccess;
+    if (nt > 0) {
+        onebit::PackParams P = pack_params(c, g, 0, 0);
+        if (std::memcmp(&P, &sg.pack, sizeof P) != 0) {
+            sg.pack = P;
+            void *args[1];
+            const cudaKernelNodeParams kp =
+                node_params((void *)onebit::ob_pack_kernel, pack_geometry(nt), &sg.pack, args);
+            e = cudaGraphExecKernelNodeSetParams(sg.exec, sg.pack_node, &kp);
+        }
+        onebit::ApplyParams A = apply_params(c);
+        if (e == cudaSuccess && std::memcmp(&A, &sg.apply, sizeof A) != 0) {
+            sg.apply = A;
+            void *args[1];
+            const cudaKernelNodeParams kp =
+                node_params((void *)onebit::ob_apply_kernel, apply_geometry(c), &sg.apply, args);
+            e = cudaGraphExecKernelNodeSetParams(sg.exec, sg.apply_node, &kp);
+        }
+    }
+    if (e == cudaSuccess) e = cudaGraphLaunch(sg.exec, c->stream);
+    return fail_cuda(c, e);
 }
 
 ob_status check_grads(const ob_ctx *c, const float *const *g) {
@@ -751,6 +905,7 @@ void ob_destroy(ob_ctx *c) {
     for (auto &ev : c->ev_consumed) cudaEventDestroy(ev);
     cudaEventDestroy(c->ev_start);
     cudaStreamDestroy(c->copy_stream);
+    destroy_graph(c);
     c->magic = 0;
     delete c;
 }
@@ -820,11 +975,30 @@ ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
     if ((st = check_grads(c, d_grads)) != OB_OK) return st;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
-    KernelTimer pack(c, OB_K_PACK);
-    if ((st = launch_pack(c, d_grads, 0, 0, c->n_tiles())) != OB_OK) return st;
-    if ((st = launch_after_pack(c, pack)) != OB_OK) return st;
+    if (c->use_graph && !c->profiling) {
+        if ((st = graph_step(c, d_grads)) != OB_OK) return st;
+    } else {
+        KernelTimer pack(c, OB_K_PACK);
+        if ((st = launch_pack(c, d_grads, 0, 0, c->n_tiles())) != OB_OK) return st;
+        if ((st = launch_after_pack(c, pack)) != OB_OK) return st;
+    }
     c->m_dense = false;
     c->t_compressed += 1;
+    return OB_OK;
+}
+
+ob_status ob_graph_enable(ob_ctx *c, int on) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    c->use_graph = on != 0;
+    return OB_OK;
+}
+
+ob_status ob_set_lr(ob_ctx *c, float lr) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!std::isfinite(lr)) return OB_ERR_INVALID_ARG;
+    c->lr = lr;
     return OB_OK;
 }
 

@@ -121,6 +121,13 @@ class OneBitAdam:
         arr = np.ascontiguousarray(value, _STATE_DTYPE[kind]).reshape(self._shape(kind))
         B.ob_write_state(self.ctx, kind, index, arr.ctypes.data, arr.nbytes)
 
+    def set_lr(self, lr: float) -> None:
+        B.ob_set_lr(self.ctx, lr)
+
+    def graph(self, on: bool = True) -> None:
+        """Replay the compressed step as one CUDA graph (small tensor lists)."""
+        B.ob_graph_enable(self.ctx, on)
+
     def profile(self, on: bool = True) -> None:
         B.ob_profile_enable(self.ctx, on)
 

@@ -214,6 +214,21 @@ OB_API ob_status ob_read_state(ob_ctx *ctx, int kind, int index, void *host_dst,
  * Waits for the copy to finish. */
 OB_API ob_status ob_write_state(ob_ctx *ctx, int kind, int index, const void *host_src, size_t bytes);
 
+/* Set the learning rate used by the following warmup and compressed steps
+ * (learning-rate schedules).  OB_ERR_INVALID_ARG for a non-finite lr. */
+OB_API ob_status ob_set_lr(ob_ctx *ctx, float lr);
+
+/* Graph mode on or off (default off).  While on (and profiling is off),
+ * ob_compressed_step replays the step's five kernels as one CUDA graph,
+ * built at the first such call: one launch instead of five, which matters
+ * for small tensor lists where each kernel runs a few microseconds.
+ * Changed gradient pointers, the dense/lazy state of m and the learning
+ * rate are written into the graph before each replay; the results are
+ * those of the ordinary launches.  ob_compressed_step_host never uses the
+ * graph.  The first call in graph mode must not be made while the stream is
+ * being captured. */
+OB_API ob_status ob_graph_enable(ob_ctx *ctx, int on);
+
 /* Turn per-kernel timing on or off.  While on, every step records CUDA
  * events between its kernels on the context's stream. */
 OB_API ob_status ob_profile_enable(ob_ctx *ctx, int on);

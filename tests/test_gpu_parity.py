@@ -290,3 +290,38 @@ def test_bucketed_contexts_on_two_streams_match_sequential():
     for a, b in zip(run(True), run(False)):
         for x, y in zip(a, b):
             assert np.array_equal(x.view(np.uint8), y.view(np.uint8))
+
+
+def test_graph_mode_matches_direct_launches():
+    """Graph mode replays the same five kernels: with gradient buffers that
+    alternate between steps, the dense -> lazy momentum switch and a
+    learning-rate change, it ends bit-identical to direct launches."""
+    wl = small_ragged(W=4, count=50)
+    runs = []
+    for graph in (False, True):
+        pr = Pair(wl)
+        other = torch.empty_like(pr.grads)
+        for _ in range(2):
+            pr.warmup_step()
+        pr.freeze()
+        pr.gpu.graph(graph)
+        for k in range(6):
+            pr.next_grads()
+            g = pr.grads if k % 2 == 0 else other.copy_(pr.grads)
+            if k == 3:
+                pr.gpu.set_lr(3e-4)
+            pr.gpu.step(g)
+        runs.append([pr.gpu.read(kd) for kd in (B.OB_STATE_P, B.OB_STATE_M, B.OB_STATE_E_SERVER,
+                                                B.OB_STATE_BITS_SERVER, B.OB_STATE_S_WORKER)]
+                    + [pr.gpu.read(B.OB_STATE_E_WORKER, w) for w in range(wl.W)])
+        pr.close()
+    for a, b in zip(*runs):
+        assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
+
+
+def test_set_lr_rejects_non_finite():
+    opt = OneBitAdam([100], 2, **WL.HYPER)
+    with pytest.raises(B.OnebitError) as ei:
+        opt.set_lr(float("nan"))
+    assert ei.value.status == B.OB_ERR_INVALID_ARG
+    opt.close()
