@@ -58,6 +58,19 @@ EXPORTS = (
 )
 
 
+__all__ = [name for name in EXPORTS] + [
+    "OnebitError", "lib", "status_name", "LIBRARY",
+    "OB_ABI_VERSION", "OB_MAX_WORKERS", "OB_TENSOR_ALIGN", "OB_STATIC_MAX_ELEMENTS",
+    "OB_OK", "OB_ERR_INVALID_ARG", "OB_ERR_PHASE", "OB_ERR_ALIGN", "OB_ERR_WORKSPACE",
+    "OB_ERR_OOM", "OB_ERR_CUDA", "OB_ERR_DEVICE_TIMEOUT",
+    "OB_STATE_P", "OB_STATE_M", "OB_STATE_V", "OB_STATE_D", "OB_STATE_E_WORKER",
+    "OB_STATE_E_SERVER", "OB_STATE_S_WORKER", "OB_STATE_S_SERVER", "OB_STATE_BITS_WORKER",
+    "OB_STATE_BITS_SERVER", "OB_STATE_STEP",
+    "OB_K_WARMUP", "OB_K_FREEZE", "OB_K_PACK", "OB_K_PACK_SCALE", "OB_K_SERVER",
+    "OB_K_SERVER_SCALE", "OB_K_APPLY", "OB_NUM_KERNELS",
+]
+
+
 class OnebitError(RuntimeError):
     def __init__(self, status: int, call: str):
         self.status = int(status)

@@ -369,7 +369,13 @@ struct KernelTimer {
         if (!c->profiling) return;
         a = take_event(c);
         b = take_event(c);
-        if (a && b) cudaEventRecord(a, c->stream);
+        if (a && b) {
+            cudaEventRecord(a, c->stream);
+        } else {  // no timing for this launch; keep whichever event was made
+            if (a) c->event_pool.push_back(a);
+            if (b) c->event_pool.push_back(b);
+            a = b = nullptr;
+        }
     }
     void stop() {
         if (!c->profiling || !a || !b) return;
@@ -828,28 +834,28 @@ ob_status ob_create(int n_tensors, const int64_t *numel, int W, float beta1, flo
     c->params = d_params;
     c->ws = static_cast<char *>(d_workspace);
     c->stream = static_cast<cudaStream_t>(cuda_stream);
-    auto bail = [&](cudaError_t e) {
+    // Release what was created so far and report `status`.
+    auto bail = [&](ob_status status) {
         if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
         for (auto &ev : c->ev_copied) if (ev) cudaEventDestroy(ev);
         for (auto &ev : c->ev_consumed) if (ev) cudaEventDestroy(ev);
         if (c->ev_start) cudaEventDestroy(c->ev_start);
         delete c;
-        (void)e;
-        return OB_ERR_CUDA;
+        return status;
     };
     cudaError_t e = cudaGetDevice(&c->device);
-    if (e != cudaSuccess) return bail(e);
+    if (e != cudaSuccess) return bail(OB_ERR_CUDA);
     e = cudaFuncSetAttribute(onebit::ob_pack_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              onebit::kPackSmemBytes);
-    if (e != cudaSuccess) return bail(e);
+    if (e != cudaSuccess) return bail(OB_ERR_CUDA);
     e = cudaStreamCreateWithFlags(&c->copy_stream, cudaStreamNonBlocking);
-    if (e != cudaSuccess) return bail(e);
+    if (e != cudaSuccess) return bail(OB_ERR_CUDA);
     for (int k = 0; k < 2 && e == cudaSuccess; ++k) {
         e = cudaEventCreateWithFlags(&c->ev_copied[k], cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_consumed[k], cudaEventDisableTiming);
     }
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c->ev_start, cudaEventDisableTiming);
-    if (e != cudaSuccess) return bail(e);
+    if (e != cudaSuccess) return bail(OB_ERR_CUDA);
     // zero the state, upload the work list
     const Plan &pl = c->plan;
     e = cudaMemsetAsync(c->ws, 0, c->cv.tiles, c->stream);
@@ -875,13 +881,13 @@ ob_status ob_create(int n_tensors, const int64_t *numel, int W, float beta1, flo
         e = cudaMemcpyAsync(c->chunk_seg_base(), pl.chunk_seg_base.data(),
                             pl.chunk_seg_base.size() * 4, cudaMemcpyHostToDevice, c->stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
-    if (e != cudaSuccess) return bail(e);
+    if (e != cudaSuccess) return bail(OB_ERR_CUDA);
     {
         std::lock_guard<std::mutex> lk(g_live_mu);
         try {
             g_live.insert(c);
         } catch (const std::bad_alloc &) {
-            return bail(cudaSuccess), OB_ERR_OOM;
+            return bail(OB_ERR_OOM);
         }
     }
     *out = c;
