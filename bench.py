@@ -377,12 +377,16 @@ def run_b200(args) -> None:
     achieved = algo["ob_pack_kernel"] / pack_avg_s / 1e9
     step_gbs = algo["step"] / (ms_per_step / 1e3) / 1e9
     model_gbs = algo["model"] / (ms_per_step / 1e3) / 1e9
+    # per kernel, per step (the server stage, its scales and the update run in
+    # chunk groups, the update of one group overlapping the next group's
+    # server stage, so their times can add up to more than the step)
     per_kernel = {}
     for name, (kms, cnt) in prof.items():
         if cnt:
-            entry = {"ms_avg": kms / cnt, "share": kms / max(1e-12, sum(v[0] for v in prof.values()))}
+            entry = {"ms_per_step": kms / args.steps, "launches_per_step": cnt / args.steps,
+                     "share": kms / max(1e-12, sum(v[0] for v in prof.values()))}
             if name in algo:
-                entry["gbs"] = algo[name] / (kms / cnt / 1e3) / 1e9
+                entry["gbs"] = algo[name] / (kms / args.steps / 1e3) / 1e9
             per_kernel[name] = entry
 
     # end to end: host gradients in pinned memory, copied in every step, and
