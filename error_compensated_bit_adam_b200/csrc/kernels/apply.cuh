@@ -24,25 +24,45 @@ struct ApplyParams {
 // words, m_hat = sign' s'_j, and takes a momentum SGD step preconditioned by
 // the frozen denominator: p -= lr (m_hat / d); m = m_hat (m is left as the
 // words and scales themselves unless a dense copy is asked for).
+//
+// The per-element IEEE division keeps the compiler from issuing a slot's
+// loads ahead of the previous slot's arithmetic, and holding all slots in
+// registers costs residency; so each thread first copies all its d and p
+// slots into shared memory (cp.async, 32 KiB per CTA), then computes.
 template <bool FULL>
-__device__ __forceinline__ void apply_tile(const ApplyParams &P, const Tile &tile) {
+__device__ __forceinline__ void apply_tile(const ApplyParams &P, const Tile &tile, float4 (*sd)[kThreads],
+                                           float4 (*spp)[kThreads]) {
     const int tid = threadIdx.x, lane = tid & 31;
     const uint32_t sb = __float_as_uint(P.sp[tile.tensor * P.W + tile.chunk]);
     const int shift = 4 * (lane & 7);
+    const uint64_t pol = evict_first_policy();
+    uint32_t inv[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int off = 4 * (tid + kThreads * u);
+        inv[u] = 0;
+        if (FULL || off < tile.count) {
+            const int64_t i = tile.begin + off;
+            cp_async16(&sd[u][tid], P.d + i, pol);
+            cp_async16(&spp[u][tid], P.p + i, pol);
+            inv[u] = ~(__ldg(P.sbits + (i >> 5)) >> shift);
+        }
+    }
+    cp_async_commit();
+    cp_async_wait<0>();
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
         const int off = 4 * (tid + kThreads * u);
         const int real = FULL ? 4 : slot_real(tile.count, off);
         if (!FULL && real == 0) continue;
         const int64_t i = tile.begin + off;
-        const uint32_t inv = ~(__ldg(P.sbits + (i >> 5)) >> shift);
-        const float4 d = ld_stream(P.d + i);
-        float4 p = ld_stream(P.p + i);
+        const float4 d = sd[u][tid];
+        float4 p = spp[u][tid];
         float4 m = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             if (FULL || k < real) {
-                const float m_hat = __uint_as_float(((inv << (31 - k)) & 0x80000000u) | sb);
+                const float m_hat = __uint_as_float(((inv[u] << (31 - k)) & 0x80000000u) | sb);
                 const float delta = __fmul_rn(P.lr, __fdiv_rn(m_hat, get(d, k)));
                 set(p, k, __fsub_rn(get(p, k), delta));
                 set(m, k, m_hat);
@@ -54,11 +74,13 @@ __device__ __forceinline__ void apply_tile(const ApplyParams &P, const Tile &til
 }
 
 __global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constant__ ApplyParams P) {
+    __shared__ float4 sd[kUnroll][kThreads];   // this thread's d slots
+    __shared__ float4 spp[kUnroll][kThreads];  // and p slots
     const Tile tile = P.tiles[blockIdx.x];
     if (tile.count == kTile)
-        apply_tile<true>(P, tile);
+        apply_tile<true>(P, tile, sd, spp);
     else
-        apply_tile<false>(P, tile);
+        apply_tile<false>(P, tile, sd, spp);
 }
 
 }  // namespace onebit
