@@ -288,6 +288,100 @@ def measure_e2e(opt, wl, n_pad, dev_grads, args, world, dev) -> dict:
         return {"value": None, "unit": UNIT, "error": repr(exc)}
 
 
+def measure_overlap(wl, args, dev, world) -> dict:
+    """Bucketed compressed steps overlapping a synthetic backward pass.
+
+    The tensor list is cut into buckets of about --bucket-elems elements,
+    each stepped by its own context on its own stream (graph mode).  The
+    backward of bucket b is modelled as two bf16 GEMMs of 2 * tokens * n_b
+    FLOPs each (weight and input gradients of n_b parameters over
+    --overlap-tokens tokens), run on the main stream in reverse bucket order;
+    bucket b's step starts when its backward GEMMs are done.  Reports the
+    backward alone, the steps alone, both interleaved, and the share of the
+    shorter of the two that the interleaving hid."""
+    from error_compensated_bit_adam_b200.buckets import BucketedOneBitAdam, split_buckets
+    buckets = split_buckets(wl.numels, args.bucket_elems)
+    bk = BucketedOneBitAdam(wl.numels, wl.W, buckets, graph=True, device=dev,
+                            priority=args.overlap_priority, **WL.HYPER)
+    grads = []
+    for b, ts in enumerate(buckets):
+        sub = WL.Workload(f"{wl.name}-bucket{b}", tuple(wl.shapes[t] for t in ts), wl.W, 0, 0,
+                          wl.seed + 1000 + b, wl.fan_in_scaling, wl.zero_fraction)
+        offs, n_pad = bk.layout(b)
+        g = torch.empty((wl.W, n_pad), dtype=torch.float32, device=dev)
+        WL.fill_grads(sub, 0, WL.grad_scale_vector(sub, offs, n_pad, device=dev), g)
+        grads.append(g)
+    K = 1024
+    gemms = []
+    for ts in buckets:
+        n_b = sum(wl.numels[t] for t in ts)
+        N = max(1, -(-n_b // K))
+        a = torch.randn(args.overlap_tokens, K, device=dev, dtype=torch.bfloat16)
+        w = torch.randn(K, N, device=dev, dtype=torch.bfloat16)
+        gemms.append((a, w, torch.empty(args.overlap_tokens, N, device=dev, dtype=torch.bfloat16),
+                      torch.empty(K, N, device=dev, dtype=torch.bfloat16)))
+
+    def backward(b):
+        a, w, out_x, out_w = gemms[b]
+        torch.matmul(a, w, out=out_x)              # input-gradient-sized GEMM
+        torch.matmul(a.t(), out_x, out=out_w)      # weight-gradient-sized GEMM
+
+    torch.cuda.synchronize(dev)
+    for b in range(len(buckets)):
+        bk.warmup_step(b, grads[b])
+    bk.wait()
+    bk.freeze()
+    for _ in range(2):
+        for b in range(len(buckets)):
+            bk.step(b, grads[b])
+            backward(b)
+    bk.wait()
+    torch.cuda.synchronize(dev)
+
+    def timed(run, reps):
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            run()
+        e1.record()
+        torch.cuda.synchronize(dev)
+        return max_over_ranks(e0.elapsed_time(e1), world) / reps
+
+    order = list(reversed(range(len(buckets))))
+
+    def only_backward():
+        for b in order:
+            backward(b)
+
+    def only_steps():
+        for b in order:
+            bk.step(b, grads[b])
+        bk.wait()
+
+    def both():
+        for b in order:
+            backward(b)
+            ev = torch.cuda.Event()
+            ev.record()
+            bk.step(b, grads[b], ev)
+        bk.wait()
+
+    reps = max(3, min(args.steps, 10))
+    t_b, t_s, t_o = timed(only_backward, reps), timed(only_steps, reps), timed(both, reps)
+    flops = sum(4 * args.overlap_tokens * K * max(1, -(-sum(wl.numels[t] for t in ts) // K))
+                for ts in buckets)
+    bk.close()
+    return {"buckets": len(buckets), "bucket_elems": args.bucket_elems,
+            "stream_priority": args.overlap_priority,
+            "backward_model": f"2 bf16 GEMMs per bucket, {args.overlap_tokens} tokens, "
+                              f"{flops / 1e12:.2f} TFLOP per pass",
+            "backward_ms": t_b, "steps_ms": t_s, "overlapped_ms": t_o,
+            "sequential_ms": t_b + t_s,
+            "hidden_fraction_of_shorter": (t_b + t_s - t_o) / min(t_b, t_s)}
+
+
 def run_b200(args) -> None:
     from error_compensated_bit_adam_b200.optimizer import OneBitAdam
 
@@ -394,6 +488,12 @@ def run_b200(args) -> None:
     e2e = ({"value": None, "unit": UNIT, "skipped": "--no-e2e"} if args.no_e2e
            else measure_e2e(opt, wl, n_pad, grads[0], args, world, dev))
 
+    overlap = None
+    if args.overlap:
+        del grads
+        torch.cuda.empty_cache()
+        overlap = measure_overlap(wl, args, dev, world)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl.W)
@@ -419,6 +519,7 @@ def run_b200(args) -> None:
                          "avg_launch_ms": pack_avg_s * 1e3},
             "kernels": per_kernel,
             "graph_mode": graph,
+            "overlap": overlap,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
@@ -447,6 +548,12 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-gradient end-to-end leg")
     ap.add_argument("--graph", action="store_true",
                     help="also time the steps replayed as one CUDA graph each")
+    ap.add_argument("--overlap", action="store_true",
+                    help="also measure bucketed steps overlapping a synthetic backward pass")
+    ap.add_argument("--bucket-elems", type=int, default=1 << 25)
+    ap.add_argument("--overlap-tokens", type=int, default=4096)
+    ap.add_argument("--overlap-priority", type=int, default=0,
+                    help="CUDA stream priority of the bucket streams (negative = higher)")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "b200" and not args.n:
         ap.error("--warmup must be >= 3")
