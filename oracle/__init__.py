@@ -91,6 +91,11 @@ class Oracle:
         L.orc_server_compress.restype = i32
         L.orc_apply.argtypes = [i64, i32, f32, vp, vp, vp, vp, vp]
         L.orc_apply.restype = None
+        L.orc_server_compress_chunk.argtypes = [i64, i32, i32, vp, vp, vp, vp, ctypes.POINTER(f32),
+                                                vp]
+        L.orc_server_compress_chunk.restype = i32
+        L.orc_apply_chunk.argtypes = [i64, i32, i32, f32, vp, f32, vp, vp, vp]
+        L.orc_apply_chunk.restype = None
         self.L = L
         self.path = path
 
@@ -163,6 +168,25 @@ class Oracle:
         self.L.orc_apply(n, s_srv.size, lr, _ptr(sbits), _ptr(s_srv), _ptr(d), _ptr(p), _ptr(m))
 
 
+    def server_compress_chunk(self, j: int, bits: Sequence[np.ndarray], s, e_s: np.ndarray,
+                              sbits: np.ndarray) -> np.float32:
+        """Server stage of chunk j only: writes chunk j's elements of e_s and
+        its words of sbits; returns s'_j."""
+        n = e_s.size
+        s = np.ascontiguousarray(s, np.float32)
+        out = ctypes.c_float()
+        rc = self.L.orc_server_compress_chunk(n, len(bits), j, _ptr_array(bits), _ptr(s), _ptr(e_s),
+                                              _ptr(_u32(sbits)), ctypes.byref(out), None)
+        if rc != 0:
+            raise MemoryError("oracle server stage out of memory")
+        return np.float32(out.value)
+
+    def apply_chunk(self, j: int, W: int, lr: float, sbits: np.ndarray, s_srv_j, d: np.ndarray,
+                    p: np.ndarray, m: np.ndarray) -> None:
+        self.L.orc_apply_chunk(p.size, W, j, lr, _ptr(_u32(sbits)), float(s_srv_j), _ptr(d),
+                               _ptr(p), _ptr(m))
+
+
 _default: Optional[Oracle] = None
 
 
@@ -183,8 +207,8 @@ class OracleRun:
 
     threads > 1 runs independent oracle calls concurrently (ctypes releases
     the GIL): the worker stage of every (tensor, worker), the server stage
-    and update of every tensor, and slices of the elementwise warmup and
-    freeze.  Each call is still the plain single-threaded C function, so
+    and update of every (tensor, server chunk), and slices of the
+    elementwise warmup and freeze.  Each call is still the plain single-threaded C function, so
     the results do not depend on `threads`.
     """
 
@@ -280,6 +304,18 @@ class OracleRun:
             self.s_srv[t] = ss
             self.o.apply_update(self.hp["lr"], sb, ss, self.d[t], self.p[t], self.m[t])
 
+        def chunk_job(t, j):  # chunks are independent: own elements, scale and words
+            bits = [self.bits_w[w][t] for w in range(W)]
+            self.s_srv[t, j] = self.o.server_compress_chunk(j, bits, self.s_w[:, t], self.e_s[t],
+                                                            self.sbits[t])
+            self.o.apply_chunk(j, W, self.hp["lr"], self.sbits[t], self.s_srv[t, j], self.d[t],
+                               self.p[t], self.m[t])
+
         self._run([lambda t=t, w=w: worker_job(t, w) for t in range(T) for w in range(W)])
-        self._run([lambda t=t: server_job(t) for t in range(T)])
+        if self.threads == 1:
+            self._run([lambda t=t: server_job(t) for t in range(T)])
+        else:
+            for t in range(T):
+                self.sbits[t] = np.zeros(self.o.num_words(self.numel[t]), np.uint32)
+            self._run([lambda t=t, j=j: chunk_job(t, j) for t in range(T) for j in range(W)])
         self.t_compressed += 1

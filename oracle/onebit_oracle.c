@@ -209,65 +209,84 @@ ORC_API int orc_worker_compress(int64_t n, float beta1, const float *m, const fl
     return 0;
 }
 
-/* Server stage [1BA, Proposed method, 3-4]: server j receives chunk j of
- * every worker's packed signs plus every worker's scale.  For element i of
- * chunk j:
+/* Server stage of one chunk [1BA, Proposed method, 3-4]: server j receives
+ * chunk j of every worker's packed signs plus every worker's scale.  For
+ * element i of chunk j:
  *   acc = +0.0; acc = acc + sign_w(i)*s_w  for w = 0..W-1 in order
  *   y   = acc / W + e_s(i)               (average, plus the server error)
  * then the chunk is compressed again:
  *   s'_j = ||y over chunk j||_2 / sqrt(len_j)   (0 for an empty chunk)
  *   sbits: 1 where y >= 0
  *   e_s = y - sign(y)*s'_j.
- * bits[w] holds worker w's ceil(n/32) words, s[w] its scale.  e_s is
- * updated in place; sbits receives ceil(n/32) words; s_srv receives W
- * chunk scales; y_out, if not NULL, receives y.  Returns 0 or -1. */
-ORC_API int orc_server_compress(int64_t n, int W, const uint32_t *const *bits, const float *s,
-                                float *e_s, uint32_t *sbits, float *s_srv, float *y_out) {
+ * bits[w] holds worker w's ceil(n/32) words, s[w] its scale.  Only chunk
+ * j's elements of e_s and y_out (if not NULL) and chunk j's words of sbits
+ * are written (chunks start on 128-element boundaries, so no word is
+ * shared with another chunk).  *s_srv_j receives s'_j.  Returns 0 or -1. */
+ORC_API int orc_server_compress_chunk(int64_t n, int W, int j, const uint32_t *const *bits,
+                                      const float *s, float *e_s, uint32_t *sbits, float *s_srv_j,
+                                      float *y_out) {
     const float wf = (float)W;
+    int64_t b, e;
+    orc_chunk_range(n, W, j, &b, &e);
     float *y = y_out;
     if (!y) {
-        y = (float *)calloc((size_t)(n > 0 ? n : 1), sizeof(float));
+        y = (float *)calloc((size_t)(e > b ? e : 1), sizeof(float));
         if (!y) return -1;
+        y -= b;  /* index y by element, like y_out */
     }
-    for (int j = 0; j < W; ++j) {
-        int64_t b, e;
-        orc_chunk_range(n, W, j, &b, &e);
-        double sum_sq = 0.0;
-        for (int64_t i = b; i < e; ++i) {
-            float acc = 0.0f;
-            for (int w = 0; w < W; ++w) acc = acc + signed_scale(get_bit(bits[w], i), s[w]);
-            const float avg = acc / wf;
-            y[i] = avg + e_s[i];
-            sum_sq += (double)y[i] * (double)y[i];
-        }
-        s_srv[j] = rms_scale(sum_sq, e - b);
+    double sum_sq = 0.0;
+    for (int64_t i = b; i < e; ++i) {
+        float acc = 0.0f;
+        for (int w = 0; w < W; ++w) acc = acc + signed_scale(get_bit(bits[w], i), s[w]);
+        const float avg = acc / wf;
+        y[i] = avg + e_s[i];
+        sum_sq += (double)y[i] * (double)y[i];
     }
-    pack_signs(n, y, sbits);
-    for (int j = 0; j < W; ++j) {
-        int64_t b, e;
-        orc_chunk_range(n, W, j, &b, &e);
-        for (int64_t i = b; i < e; ++i) e_s[i] = y[i] - signed_scale(sign_bit(y[i]), s_srv[j]);
-    }
-    if (y != y_out) free(y);
+    const float sj = rms_scale(sum_sq, e - b);
+    if (e > b)  /* an empty chunk owns no word, not even the tensor's last */
+        for (int64_t k = b / 32; k < (e + 31) / 32; ++k) sbits[k] = 0u;
+    for (int64_t i = b; i < e; ++i)
+        if (sign_bit(y[i])) sbits[i >> 5] |= (uint32_t)1u << (i & 31);
+    for (int64_t i = b; i < e; ++i) e_s[i] = y[i] - signed_scale(sign_bit(y[i]), sj);
+    *s_srv_j = sj;
+    if (y != y_out) free(y + b);
     return 0;
 }
 
-/* Gather and update [1BA, Proposed method, 1-2]: every worker receives all
- * server chunks and decodes the averaged momentum m_hat = sign'(i)*s'_j
- * (exact), which replaces the momentum; the parameters take one momentum
- * SGD step preconditioned by the frozen denominator d:
- *   p = p - lr * (m_hat / d);   m = m_hat. */
+/* Server stage of a whole tensor: every chunk j = 0..W-1 as above.  sbits
+ * receives ceil(n/32) words, s_srv the W chunk scales, y_out (if not
+ * NULL) y.  Returns 0 or -1. */
+ORC_API int orc_server_compress(int64_t n, int W, const uint32_t *const *bits, const float *s,
+                                float *e_s, uint32_t *sbits, float *s_srv, float *y_out) {
+    memset(sbits, 0, (size_t)orc_num_words(n) * sizeof(uint32_t));
+    for (int j = 0; j < W; ++j)
+        if (orc_server_compress_chunk(n, W, j, bits, s, e_s, sbits, &s_srv[j], y_out) != 0)
+            return -1;
+    return 0;
+}
+
+/* Gather and update of one chunk [1BA, Proposed method, 1-2]: every worker
+ * receives all server chunks and decodes the averaged momentum
+ * m_hat = sign'(i)*s'_j (exact), which replaces the momentum; the
+ * parameters take one momentum SGD step preconditioned by the frozen
+ * denominator d:
+ *   p = p - lr * (m_hat / d);   m = m_hat.
+ * Only chunk j's elements are written. */
+ORC_API void orc_apply_chunk(int64_t n, int W, int j, float lr, const uint32_t *sbits,
+                             float s_srv_j, const float *d, float *p, float *m) {
+    int64_t b, e;
+    orc_chunk_range(n, W, j, &b, &e);
+    for (int64_t i = b; i < e; ++i) {
+        const float m_hat = signed_scale(get_bit(sbits, i), s_srv_j);
+        const float ratio = m_hat / d[i];
+        const float delta = lr * ratio;
+        p[i] = p[i] - delta;
+        m[i] = m_hat;
+    }
+}
+
+/* Gather and update of a whole tensor: every chunk as above. */
 ORC_API void orc_apply(int64_t n, int W, float lr, const uint32_t *sbits, const float *s_srv,
                        const float *d, float *p, float *m) {
-    for (int j = 0; j < W; ++j) {
-        int64_t b, e;
-        orc_chunk_range(n, W, j, &b, &e);
-        for (int64_t i = b; i < e; ++i) {
-            const float m_hat = signed_scale(get_bit(sbits, i), s_srv[j]);
-            const float ratio = m_hat / d[i];
-            const float delta = lr * ratio;
-            p[i] = p[i] - delta;
-            m[i] = m_hat;
-        }
-    }
+    for (int j = 0; j < W; ++j) orc_apply_chunk(n, W, j, lr, sbits, s_srv[j], d, p, m);
 }

@@ -45,20 +45,24 @@ MUTANTS = [
      "signed_scale(get_bit(bits[w], i), s[0])"),
     ("server_reads_neighbour_bit", "signed_scale(get_bit(bits[w], i), s[w])",
      "signed_scale(get_bit(bits[w], i ^ 1), s[w])"),
-    ("server_error_uses_chunk0_scale",
-     "e_s[i] = y[i] - signed_scale(sign_bit(y[i]), s_srv[j]);",
-     "e_s[i] = y[i] - signed_scale(sign_bit(y[i]), s_srv[0]);"),
+    ("server_error_uses_worker0_scale",
+     "e_s[i] = y[i] - signed_scale(sign_bit(y[i]), sj);",
+     "e_s[i] = y[i] - signed_scale(sign_bit(y[i]), s[0]);"),
     ("server_error_wrong_sign", "e_s[i] = y[i] - signed_scale(", "e_s[i] = y[i] + signed_scale("),
     ("chunks_not_word_group_aligned", "const int64_t cw = ((per + 3) / 4) * 4;",
      "const int64_t cw = per;"),
-    ("apply_wrong_sign", "p[i] = p[i] - delta;\n            m[i] = m_hat;",
-     "p[i] = p[i] + delta;\n            m[i] = m_hat;"),
-    ("apply_keeps_old_momentum", "            m[i] = m_hat;\n", "            (void)m;\n"),
-    ("apply_uses_chunk0_scale", "signed_scale(get_bit(sbits, i), s_srv[j])",
-     "signed_scale(get_bit(sbits, i), s_srv[0])"),
+    ("apply_wrong_sign", "p[i] = p[i] - delta;\n        m[i] = m_hat;",
+     "p[i] = p[i] + delta;\n        m[i] = m_hat;"),
+    ("apply_keeps_old_momentum", "        m[i] = m_hat;\n", "        (void)m;\n"),
+    ("apply_uses_chunk0_scale", "orc_apply_chunk(n, W, j, lr, sbits, s_srv[j], d, p, m);",
+     "orc_apply_chunk(n, W, j, lr, sbits, s_srv[0], d, p, m);"),
     ("apply_multiplies_by_d", "const float ratio = m_hat / d[i];", "const float ratio = m_hat * d[i];"),
     ("packing_bit_order_reversed", "words[i >> 5] |= (uint32_t)1u << (i & 31);",
      "words[i >> 5] |= (uint32_t)1u << (31 - (i & 31));"),
+    ("server_packing_bit_order_reversed", "sbits[i >> 5] |= (uint32_t)1u << (i & 31);",
+     "sbits[i >> 5] |= (uint32_t)1u << (31 - (i & 31));"),
+    ("server_empty_chunk_clears_a_word", "    if (e > b)  /* an empty chunk owns no word, not even the tensor's last */\n",
+     "    if (1)\n"),
 ]
 
 MUTANT_CFLAGS = [f for f in oracle.CFLAGS if f != "-Werror"]
