@@ -51,10 +51,12 @@ def shortened(wl: WL.Workload, warmup: int, compressed: int) -> WL.Workload:
                        wl.zero_fraction)
 
 
+# the headline workloads: 10 free-running compressed steps, then parameters
+# within 1e-5 relative L2 (plus every step's words and scales)
 FULL = {
-    WL.BERT_LARGE_FLAT_W8.name: shortened(WL.BERT_LARGE_FLAT_W8, 2, 3),
-    WL.ENCODER_24L_W16.name: shortened(WL.ENCODER_24L_W16, 1, 2),
-    WL.RAGGED_2000_W8.name: shortened(WL.RAGGED_2000_W8, 1, 2),
+    WL.BERT_LARGE_FLAT_W8.name: shortened(WL.BERT_LARGE_FLAT_W8, 2, 10),
+    WL.ENCODER_24L_W16.name: shortened(WL.ENCODER_24L_W16, 2, 10),
+    WL.RAGGED_2000_W8.name: shortened(WL.RAGGED_2000_W8, 2, 10),
 }
 # sweep points: the whole oracle up to W*n = 2^30 worker elements; above
 # that (up to 2^34, minutes of single-core oracle time each) sampled
