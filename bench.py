@@ -55,6 +55,8 @@ def algorithmic_bytes(n_real: int, W: int) -> dict:
       pack    1/8 (server words -> m) + W (4 g + 4 x_prev + 4 x) + W/8 (words)
       server  W/8 (words) + 4 (y_prev) + 4 (y) + 1/8 (words)
       apply   1/8 (words) + 4 (d) + 8 (p read and write)
+      warmup  4W (g) + 24 (m, v, p read and write)   [pre-path]
+      freeze  8 (v read, d written)                  [pre-path]
     The scale kernels move ~0.  'model' is the dense-momentum byte model
     12W + W/4 + 28.25 (126.25 B at W=8) the effective-bandwidth target is
     quoted on."""
@@ -62,7 +64,10 @@ def algorithmic_bytes(n_real: int, W: int) -> dict:
     server = n_real * (W / 8 + 8 + 1 / 8)
     apply = n_real * (1 / 8 + 4 + 8)
     return {"ob_pack_kernel": pack, "ob_server_kernel": server, "ob_apply_kernel": apply,
-            "step": pack + server + apply, "model": n_real * (12 * W + W / 4 + 28.25)}
+            "step": pack + server + apply, "model": n_real * (12 * W + W / 4 + 28.25),
+            # the untimed pre-path: Adam reads W gradients and reads and
+            # writes m, v and p; the freeze reads v and writes d in its place
+            "ob_warmup_kernel": n_real * (4 * W + 24), "ob_freeze_kernel": n_real * 8}
 
 
 def kernel_sources_sha256(files) -> str:
@@ -409,11 +414,14 @@ def run_b200(args) -> None:
     grads = [torch.empty((wl.W, n_pad), dtype=torch.float32, device=dev) for _ in range(n_sets)]
 
     step = 0
-    for _ in range(wl.warmup_steps):           # full-precision Adam warmup, untimed
+    opt.profile(True)                          # the pre-path's kernels, by their own events
+    for _ in range(wl.warmup_steps):           # full-precision Adam warmup, outside the step
         WL.fill_grads(wl, step, scale, grads[0])
         step += 1
         opt.warmup_step(grads[0])
     opt.freeze()
+    pre_prof = opt.profile_read(reset=True)
+    opt.profile(False)
     for gs in grads:                           # fresh draws for the timed steps
         WL.fill_grads(wl, step, scale, gs)
         step += 1
@@ -483,6 +491,17 @@ def run_b200(args) -> None:
                 entry["gbs"] = algo[name] / (kms / args.steps / 1e3) / 1e9
             per_kernel[name] = entry
 
+    # the pre-path (full-precision Adam warmup and the freeze), timed by the
+    # library's event pairs around each launch; the gradients each warmup
+    # launch reads (4W bytes per parameter) are far larger than L2
+    pre_path = {}
+    for name in ("ob_warmup_kernel", "ob_freeze_kernel"):
+        kms, cnt = pre_prof[name]
+        if cnt:
+            gbs = algo[name] / (kms / cnt / 1e3) / 1e9
+            pre_path[name] = {"launches": cnt, "avg_launch_ms": kms / cnt, "gbs": gbs,
+                              "frac_of_measured_hbm": gbs / peak["hbm_gbs"]}
+
     # end to end: host gradients in pinned memory, copied in every step, and
     # the step's server scales read back, through ob_compressed_step_host
     e2e = ({"value": None, "unit": UNIT, "skipped": "--no-e2e"} if args.no_e2e
@@ -518,6 +537,7 @@ def run_b200(args) -> None:
                          "algorithmic_bytes_per_launch": algo["ob_pack_kernel"],
                          "avg_launch_ms": pack_avg_s * 1e3},
             "kernels": per_kernel,
+            "pre_path": pre_path,
             "graph_mode": graph,
             "overlap": overlap,
             "cpu_baseline": cpu,
