@@ -293,6 +293,63 @@ def measure_e2e(opt, wl, n_pad, dev_grads, args, world, dev) -> dict:
         return {"value": None, "unit": UNIT, "error": repr(exc)}
 
 
+def measure_split_ranks(wl, args, dev) -> dict:
+    """The split step (distributed.LocalRanks) as G ranks on this one GPU,
+    each with its own context, the exchanges done by device copies: each
+    rank's own kernels (worker stage of W/G workers, server stage of its
+    chunks, the update) timed by its context's event pairs.  That is the
+    compute of one GPU in a G-GPU run; the exchange over NVLink is not
+    measured here (one GPU), only its bytes are reported."""
+    from error_compensated_bit_adam_b200.distributed import LocalRanks
+    G = args.split_ranks
+    offsets, n_pad = B.ob_layout(wl.numels)
+    need = G * (B.ob_workspace_bytes(wl.numels, wl.W) + 4 * n_pad) + 4 * wl.W * n_pad + (1 << 30)
+    free = torch.cuda.mem_get_info(dev)[0]
+    if free < need:
+        return {"G": G, "skipped": f"needs {need / 1e9:.1f} GB of device memory, {free / 1e9:.1f} free"}
+    params = WL.make_params(wl, offsets, n_pad, device=dev)
+    scale = WL.grad_scale_vector(wl, offsets, n_pad, device=dev)
+    ranks = LocalRanks(wl.numels, wl.W, G, device=dev, **WL.HYPER)
+    g = torch.empty((wl.W, n_pad), dtype=torch.float32, device=dev)
+    try:
+        for r in ranks.ranks:
+            r.params.copy_(params)
+        del params
+        WL.fill_grads(wl, 0, scale, g)
+        ranks.warmup_step(g)
+        ranks.freeze()
+        WL.fill_grads(wl, 1, scale, g)
+        del scale
+        for _ in range(max(1, args.warmup)):
+            ranks.step(g)
+        torch.cuda.synchronize(dev)
+        for r in ranks.ranks:
+            r.opt.profile(True)
+            r.opt.profile_read(reset=True)
+        K = max(1, min(args.steps, 20))
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(K):
+            ranks.step(g)
+        t1.record()
+        torch.cuda.synchronize(dev)
+        per_rank = []
+        for r in ranks.ranks:
+            prof = r.opt.profile_read(reset=True)
+            r.opt.profile(False)
+            per_rank.append({name: ms / K for name, (ms, cnt) in prof.items() if cnt})
+        compute = [sum(p.values()) for p in per_rank]
+        return {"G": G, "W": wl.W, "workers_per_rank": wl.W // G, "steps": K,
+                "ms_per_step_all_ranks_on_one_gpu": t0.elapsed_time(t1) / K,
+                "rank_compute_ms_per_step": compute,
+                "rank0_kernels_ms_per_step": per_rank[0],
+                "exchange_bytes_per_rank_per_step": ranks.ranks[0].exchange_bytes(),
+                "note": "each rank's own kernels, timed by its context; the exchange between "
+                        "ranks is device copies on one GPU here, not NVLink, and is not timed"}
+    finally:
+        ranks.close()
+
+
 def measure_overlap(wl, args, dev, world) -> dict:
     """Bucketed compressed steps overlapping a synthetic backward pass.
 
@@ -513,6 +570,14 @@ def run_b200(args) -> None:
         torch.cuda.empty_cache()
         overlap = measure_overlap(wl, args, dev, world)
 
+    split = None
+    if args.split_ranks:
+        opt.close()                            # release this context's device memory first
+        opt.workspace = opt.params = opt._staging = None
+        params = grads = None
+        torch.cuda.empty_cache()
+        split = measure_split_ranks(wl, args, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl.W)
@@ -540,6 +605,7 @@ def run_b200(args) -> None:
             "pre_path": pre_path,
             "graph_mode": graph,
             "overlap": overlap,
+            "split_ranks": split,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
@@ -570,6 +636,8 @@ def main(argv=None):
                     help="also time the steps replayed as one CUDA graph each")
     ap.add_argument("--overlap", action="store_true",
                     help="also measure bucketed steps overlapping a synthetic backward pass")
+    ap.add_argument("--split-ranks", type=int, default=0,
+                    help="also run the split step as G ranks on this GPU and time each rank's share")
     ap.add_argument("--bucket-elems", type=int, default=1 << 25)
     ap.add_argument("--overlap-tokens", type=int, default=4096)
     ap.add_argument("--overlap-priority", type=int, default=0,

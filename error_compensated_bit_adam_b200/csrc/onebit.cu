@@ -300,6 +300,13 @@ struct ob_ctx {
     bool use_graph = false;
     StepGraph graph;
     bool broken = false;
+    // workers computed by the worker stage (all of them unless a split step
+    // narrows the range), and the server chunks this context serves: chunk j
+    // of every tensor when j % shard_G == shard_rank (all when shard_G == 1)
+    int w_begin = 0, w_end = 0;
+    int shard_G = 1, shard_rank = 0;
+    // split step: 0 idle, 1 after ob_worker_stage, 2 after ob_server_stage
+    int split_stage = 0;
     // profiling
     bool profiling = false;
     std::vector<cudaEvent_t> event_pool;
@@ -412,6 +419,8 @@ onebit::PackParams pack_params(const ob_ctx *c, const float *const *g, int64_t g
     P.n_pad = c->plan.n_pad;
     P.W = c->plan.W;
     P.T = c->plan.T;
+    P.w_begin = c->w_begin;
+    P.w_end = c->w_end;
     P.beta1 = c->beta1;
     P.c1 = c->c1;
     return P;
@@ -429,6 +438,7 @@ onebit::ScaleParams worker_scale_params(const ob_ctx *c) {
     P.out_prev = c->s_prev();
     P.out_last = c->s_last();
     P.rows = c->plan.W;
+    P.row_base = c->w_begin;
     P.R = c->plan.T;
     P.out_stride_r = 1;
     P.out_stride_row = c->plan.T;
@@ -450,6 +460,8 @@ onebit::ServerParams server_params(const ob_ctx *c) {
     P.T = c->plan.T;
     P.w_pow2 = (W & (W - 1)) == 0;
     P.inv_w = 1.0f / (float)W;  // exact for a power of two
+    P.owner_mod = c->shard_G;
+    P.owner_rem = c->shard_rank;
     return P;
 }
 
@@ -491,7 +503,7 @@ struct Geometry {
 };
 Geometry pack_geometry(int tiles) { return {grid1(tiles), dim3(kThreads), (size_t)onebit::kPackSmemBytes}; }
 Geometry worker_scale_geometry(const ob_ctx *c) {
-    return {dim3((unsigned)c->plan.T, (unsigned)c->plan.W, (unsigned)c->plan.tensor_max_seg),
+    return {dim3((unsigned)c->plan.T, (unsigned)(c->w_end - c->w_begin), (unsigned)c->plan.tensor_max_seg),
             dim3(kScaleThreads), 0};
 }
 Geometry server_geometry(const ob_ctx *c) {
@@ -512,19 +524,19 @@ ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int ti
     return fail_cuda(c, cudaGetLastError());
 }
 
-// Everything of a compressed step after the worker stage's tile kernels.
-ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
-    const int nt = c->n_tiles();
-    pack_timer.stop();
-    {
-        KernelTimer k(c, OB_K_PACK_SCALE);
-        const Geometry G = worker_scale_geometry(c);
-        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(worker_scale_params(c));
-        k.stop();
-        ob_status st = fail_cuda(c, cudaGetLastError());
-        if (st != OB_OK) return st;
-    }
-    if (nt > 0) {
+// The worker scales of the workers [w_begin, w_end).
+ob_status launch_worker_scales(ob_ctx *c) {
+    if (c->w_end <= c->w_begin) return OB_OK;
+    KernelTimer k(c, OB_K_PACK_SCALE);
+    const Geometry G = worker_scale_geometry(c);
+    onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(worker_scale_params(c));
+    k.stop();
+    return fail_cuda(c, cudaGetLastError());
+}
+
+// The server stage of the chunks this context serves, and their scales.
+ob_status launch_server(ob_ctx *c) {
+    if (c->n_tiles() > 0) {
         KernelTimer k(c, OB_K_SERVER);
         const Geometry G = server_geometry(c);
         onebit::ob_server_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_params(c));
@@ -532,23 +544,30 @@ ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
         ob_status st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
     }
-    {
-        KernelTimer k(c, OB_K_SERVER_SCALE);
-        const Geometry G = server_scale_geometry(c);
-        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_scale_params(c));
-        k.stop();
-        ob_status st = fail_cuda(c, cudaGetLastError());
-        if (st != OB_OK) return st;
-    }
-    if (nt > 0) {
-        KernelTimer k(c, OB_K_APPLY);
-        const Geometry G = apply_geometry(c);
-        onebit::ob_apply_kernel<<<G.grid, G.block, G.smem, c->stream>>>(apply_params(c));
-        k.stop();
-        ob_status st = fail_cuda(c, cudaGetLastError());
-        if (st != OB_OK) return st;
-    }
-    return OB_OK;
+    KernelTimer k(c, OB_K_SERVER_SCALE);
+    const Geometry G = server_scale_geometry(c);
+    onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_scale_params(c));
+    k.stop();
+    return fail_cuda(c, cudaGetLastError());
+}
+
+// Gather and update.
+ob_status launch_apply(ob_ctx *c) {
+    if (c->n_tiles() == 0) return OB_OK;
+    KernelTimer k(c, OB_K_APPLY);
+    const Geometry G = apply_geometry(c);
+    onebit::ob_apply_kernel<<<G.grid, G.block, G.smem, c->stream>>>(apply_params(c));
+    k.stop();
+    return fail_cuda(c, cudaGetLastError());
+}
+
+// Everything of a compressed step after the worker stage's tile kernels.
+ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
+    pack_timer.stop();
+    ob_status st = launch_worker_scales(c);
+    if (st == OB_OK) st = launch_server(c);
+    if (st == OB_OK) st = launch_apply(c);
+    return st;
 }
 
 // ------------------------------------------------------------- graph mode
@@ -642,10 +661,10 @@ ob_status graph_step(ob_ctx *c, const float *const *g) {
     return fail_cuda(c, e);
 }
 
-ob_status check_grads(const ob_ctx *c, const float *const *g) {
+ob_status check_grads(const ob_ctx *c, const float *const *g, int w_begin, int w_end) {
     if (!g) return OB_ERR_INVALID_ARG;
     if (c->plan.n_pad == 0) return OB_OK;  // nothing is read
-    for (int w = 0; w < c->plan.W; ++w) {
+    for (int w = w_begin; w < w_end; ++w) {
         if (!g[w]) return OB_ERR_INVALID_ARG;
         if (!aligned(g[w], 16)) return OB_ERR_ALIGN;
     }
@@ -834,6 +853,8 @@ ob_status ob_create(int n_tensors, const int64_t *numel, int W, float beta1, flo
     c->params = d_params;
     c->ws = static_cast<char *>(d_workspace);
     c->stream = static_cast<cudaStream_t>(cuda_stream);
+    c->w_begin = 0;
+    c->w_end = c->plan.W;
     // Release what was created so far and report `status`.
     auto bail = [&](ob_status status) {
         if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
@@ -919,8 +940,8 @@ void ob_destroy(ob_ctx *c) {
 ob_status ob_warmup_adam_step(ob_ctx *c, const float *const *d_grads) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
-    if (c->frozen) return OB_ERR_PHASE;
-    if ((st = check_grads(c, d_grads)) != OB_OK) return st;
+    if (c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
+    if ((st = check_grads(c, d_grads, 0, c->plan.W)) != OB_OK) return st;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
     if ((st = materialize_momentum(c)) != OB_OK) return st;
@@ -953,7 +974,7 @@ ob_status ob_warmup_adam_step(ob_ctx *c, const float *const *d_grads) {
 ob_status ob_freeze_variance(ob_ctx *c) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
-    if (c->frozen || c->t_warmup < 1) return OB_ERR_PHASE;
+    if (c->frozen || c->t_warmup < 1 || c->split_stage != 0) return OB_ERR_PHASE;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
     const float bc2 = (float)(1.0 - std::pow((double)c->beta2, (double)c->t_warmup));
@@ -977,8 +998,8 @@ ob_status ob_freeze_variance(ob_ctx *c) {
 ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
-    if (!c->frozen) return OB_ERR_PHASE;
-    if ((st = check_grads(c, d_grads)) != OB_OK) return st;
+    if (!c->frozen || c->split_stage != 0 || c->shard_G != 1) return OB_ERR_PHASE;
+    if ((st = check_grads(c, d_grads, 0, c->plan.W)) != OB_OK) return st;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
     if (c->use_graph && !c->profiling) {
@@ -988,6 +1009,103 @@ ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
         if ((st = launch_pack(c, d_grads, 0, 0, c->n_tiles())) != OB_OK) return st;
         if ((st = launch_after_pack(c, pack)) != OB_OK) return st;
     }
+    c->m_dense = false;
+    c->t_compressed += 1;
+    return OB_OK;
+}
+
+// ------------------------------------------------------- the split step
+//
+// One compressed step in three calls, for a data-parallel run in which each
+// process computes some of the workers and serves some of the server
+// chunks; the caller's collectives run between the calls (see onebit.h).
+
+ob_status ob_set_server_shard(ob_ctx *c, int n_shards, int shard) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (n_shards < 1 || n_shards > c->plan.W || shard < 0 || shard >= n_shards) return OB_ERR_INVALID_ARG;
+    if (c->split_stage != 0) return OB_ERR_PHASE;
+    c->shard_G = n_shards;
+    c->shard_rank = shard;
+    return OB_OK;
+}
+
+ob_status ob_worker_stage(ob_ctx *c, const float *const *d_grads, int w_begin, int w_count) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
+    if (w_begin < 0 || w_count < 0 || w_begin > c->plan.W - w_count) return OB_ERR_INVALID_ARG;
+    if ((st = check_grads(c, d_grads, w_begin, w_begin + w_count)) != OB_OK) return st;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    c->w_begin = w_begin;
+    c->w_end = w_begin + w_count;
+    if (w_count > 0) {
+        KernelTimer pack(c, OB_K_PACK);
+        st = launch_pack(c, d_grads, 0, 0, c->n_tiles());
+        pack.stop();
+    }
+    if (st == OB_OK) st = launch_worker_scales(c);
+    c->w_begin = 0;
+    c->w_end = c->plan.W;
+    if (st != OB_OK) return st;
+    c->split_stage = 1;
+    return OB_OK;
+}
+
+ob_status ob_worker_exchange_buffers(ob_ctx *c, uint32_t **d_bits, size_t *bits_row_bytes,
+                                     float **d_scales, size_t *scales_row_bytes) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!d_bits || !bits_row_bytes || !d_scales || !scales_row_bytes) return OB_ERR_INVALID_ARG;
+    *d_bits = c->bits();
+    *bits_row_bytes = (size_t)(c->plan.n_pad / 32) * 4;
+    *d_scales = c->s_prev();
+    *scales_row_bytes = (size_t)c->plan.T * 4;
+    return OB_OK;
+}
+
+ob_status ob_server_stage(ob_ctx *c) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (c->split_stage != 1) return OB_ERR_PHASE;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    // the exchange filled the scale rows of the workers computed elsewhere;
+    // keep the copy that S_WORKER reads in step with them
+    cudaError_t e = cudaMemcpyAsync(c->s_last(), c->s_prev(), (size_t)c->plan.W * c->plan.T * 4,
+                                    cudaMemcpyDeviceToDevice, c->stream);
+    if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    if ((st = launch_server(c)) != OB_OK) return st;
+    c->split_stage = 2;
+    return OB_OK;
+}
+
+ob_status ob_server_exchange_buffers(ob_ctx *c, uint32_t **d_sbits, size_t *sbits_bytes,
+                                     float **d_scales, size_t *scales_bytes) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!d_sbits || !sbits_bytes || !d_scales || !scales_bytes) return OB_ERR_INVALID_ARG;
+    *d_sbits = c->sbits();
+    *sbits_bytes = (size_t)(c->plan.n_pad / 32) * 4;
+    *d_scales = c->sp_last();
+    *scales_bytes = (size_t)c->plan.T * c->plan.W * 4;
+    return OB_OK;
+}
+
+ob_status ob_apply_update(ob_ctx *c) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (c->split_stage != 2) return OB_ERR_PHASE;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    // the exchange completed the scales in sp_last; the next server stage
+    // decodes its y_prev with sp_prev
+    cudaError_t e = cudaMemcpyAsync(c->sp_prev(), c->sp_last(), (size_t)c->plan.T * c->plan.W * 4,
+                                    cudaMemcpyDeviceToDevice, c->stream);
+    if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    if ((st = launch_apply(c)) != OB_OK) return st;
+    c->split_stage = 0;
     c->m_dense = false;
     c->t_compressed += 1;
     return OB_OK;
@@ -1020,7 +1138,7 @@ ob_status ob_compressed_step_host(ob_ctx *c, const float *const *h_grads, void *
                                   size_t staging_bytes, float *h_server_scales) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
-    if (!c->frozen) return OB_ERR_PHASE;
+    if (!c->frozen || c->split_stage != 0 || c->shard_G != 1) return OB_ERR_PHASE;
     if (!h_grads || !d_staging) return OB_ERR_INVALID_ARG;
     for (int w = 0; w < c->plan.W; ++w)
         if (!h_grads[w]) return OB_ERR_INVALID_ARG;
@@ -1115,6 +1233,7 @@ ob_status ob_read_state(ob_ctx *c, int kind, int index, void *host_dst, size_t b
 ob_status ob_write_state(ob_ctx *c, int kind, int index, const void *host_src, size_t bytes) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
+    if (c->split_stage != 0) return OB_ERR_PHASE;
     if (!host_src) return OB_ERR_INVALID_ARG;
     const size_t want = state_bytes(c, kind);
     if (want == 0 || bytes != want) return OB_ERR_INVALID_ARG;

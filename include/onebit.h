@@ -199,6 +199,71 @@ OB_API ob_status ob_host_staging_bytes(const ob_ctx *ctx, size_t *bytes);
 OB_API ob_status ob_compressed_step_host(ob_ctx *ctx, const float *const *h_grads, void *d_staging,
                                   size_t staging_bytes, float *h_server_scales);
 
+/* --------------------------------------------------------------------
+ * The split step: one compressed step in three calls, for a data-parallel
+ * run over G processes (one per GPU) in which process r computes workers
+ * [w_begin, w_begin + w_count) and serves the server chunks j with
+ * j % G == r of every tensor -- the worker stage and the server stage of
+ * the compressed collective [1BA, Proposed method, 4] with the exchange
+ * between them done by the caller's collectives:
+ *
+ *   ob_set_server_shard(ctx, G, r)                    once
+ *   per step:
+ *     ob_worker_stage(ctx, d_grads, w_begin, w_count)
+ *     all-gather of the worker rows of ob_worker_exchange_buffers
+ *     ob_server_stage(ctx)
+ *     sum-all-reduce of ob_server_exchange_buffers (words as 32-bit
+ *       integers, scales as floats)
+ *     ob_apply_update(ctx)
+ *
+ * Every process holds a context over the whole tensor list with all W
+ * workers (the rows of other processes' workers are filled by the
+ * exchange); p, m and d are the same on every process.  The result equals
+ * ob_compressed_step of one context with the same W bit for bit: the sums
+ * of the exchange add exact zeros to each word and scale.  With G = 1 and
+ * no collectives the three calls are ob_compressed_step.  While a split
+ * step is open (between ob_worker_stage and ob_apply_update) only these
+ * calls, ob_read_state and ob_destroy are accepted; ob_compressed_step and
+ * ob_compressed_step_host need G = 1.  Warmup steps need the gradients of
+ * all W workers on every process (the warmup averages them in worker
+ * order). */
+
+/* Serve the chunks j with j % n_shards == shard (1 <= n_shards <= W,
+ * 0 <= shard < n_shards).  Default: n_shards = 1 (every chunk).
+ * OB_ERR_PHASE inside a split step. */
+OB_API ob_status ob_set_server_shard(ob_ctx *ctx, int n_shards, int shard);
+
+/* Worker stage of workers [w_begin, w_begin + w_count) (w_count may be 0):
+ * momentum, error feedback, 1-bit compression and worker scales, as in
+ * ob_compressed_step.  d_grads: host array of W device pointers, only the
+ * entries of the range read (the others may be NULL).  OB_ERR_PHASE before
+ * the freeze or inside a split step. */
+OB_API ob_status ob_worker_stage(ob_ctx *ctx, const float *const *d_grads, int w_begin, int w_count);
+
+/* Device buffers of the worker stage's outputs, one row per worker, rows
+ * adjacent (row w at base + w * row_bytes): *d_bits uint32[W][n_padded/32]
+ * sign words, *d_scales float[W][n_tensors] worker scales.  Owned by the
+ * context (inside its workspace); valid until ob_destroy. */
+OB_API ob_status ob_worker_exchange_buffers(ob_ctx *ctx, uint32_t **d_bits, size_t *bits_row_bytes,
+                                            float **d_scales, size_t *scales_row_bytes);
+
+/* Server stage of the served chunks (all worker rows must hold this step's
+ * words and scales): average, server error, re-compression and server
+ * scales.  The words of chunks served elsewhere are set to 0 and their
+ * scales to 0.  OB_ERR_PHASE unless ob_worker_stage came before. */
+OB_API ob_status ob_server_stage(ob_ctx *ctx);
+
+/* Device buffers of the server stage's outputs: *d_sbits uint32[n_padded/32]
+ * server sign words, *d_scales float[n_tensors][W] server scales.  Owned
+ * by the context; valid until ob_destroy. */
+OB_API ob_status ob_server_exchange_buffers(ob_ctx *ctx, uint32_t **d_sbits, size_t *sbits_bytes,
+                                            float **d_scales, size_t *scales_bytes);
+
+/* Gather and update with every chunk's words and scales present: closes
+ * the split step (the compressed step count advances).  OB_ERR_PHASE unless
+ * ob_server_stage came before. */
+OB_API ob_status ob_apply_update(ob_ctx *ctx);
+
 /* Copy one piece of state to host memory.  kind: ob_state_kind.  index:
  * the worker for OB_STATE_E_WORKER / OB_STATE_BITS_WORKER, else 0.  bytes:
  * must equal the size listed with the kind.  Waits for the stream first.

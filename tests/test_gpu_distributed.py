@@ -1,0 +1,127 @@
+"""The split step (ob_worker_stage / ob_server_stage / ob_apply_update with
+the exchanges between them) against one ob_compressed_step context.
+
+G ranks run in one process on one GPU (distributed.LocalRanks), each with
+its own context, the exchanges done by device copies and sums.  The bar is
+bit for bit: parameters, momentum, the server words and scales, and every
+worker's words and scales on every rank, after warmup, freeze and several
+compressed steps with fresh gradients."""
+import numpy as np
+import pytest
+import torch
+
+from error_compensated_bit_adam_b200 import _binding as B
+from error_compensated_bit_adam_b200 import workloads as WL
+from error_compensated_bit_adam_b200.distributed import DistributedOneBitAdam, LocalRanks
+from error_compensated_bit_adam_b200.optimizer import OneBitAdam
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    # (tensor sizes, W, G)
+    "flat-W8-G8": ((1 << 18,), 8, 8),
+    "flat-W8-G2": ((1 << 18,), 8, 2),
+    "ragged-W8-G4": ((100_003, 31, 0, 4097, 70_000), 8, 4),
+    "ragged-W6-G3": ((50_001, 129, 12_345), 6, 3),
+    "empty-chunks-W16-G4": ((100, 33, 5000), 16, 4),
+    "W4-G1": ((30_000, 7), 4, 1),
+}
+
+
+def _run(sizes, W, G, warmup=2, compressed=4, seed=31):
+    wl = WL.Workload(f"split-{W}-{G}", tuple((n,) for n in sizes), W, warmup, compressed, seed=seed,
+                     zero_fraction=0.2)
+    offsets, n_pad = B.ob_layout(wl.numels)
+    params = WL.make_params(wl, offsets, n_pad, device="cuda")
+    scale = WL.grad_scale_vector(wl, offsets, n_pad, device="cuda")
+    ref = OneBitAdam(wl.numels, W, params=params.clone(), **WL.HYPER)
+    ranks = LocalRanks(wl.numels, W, G, **WL.HYPER)
+    for r in ranks.ranks:
+        r.params.copy_(params)
+    g = torch.empty((W, n_pad), device="cuda")
+    step = 0
+    for _ in range(warmup):
+        WL.fill_grads(wl, step, scale, g)
+        step += 1
+        ref.warmup_step(g)
+        ranks.warmup_step(g)
+    ref.freeze()
+    ranks.freeze()
+    for _ in range(compressed):
+        WL.fill_grads(wl, step, scale, g)
+        step += 1
+        ref.step(g)
+        ranks.step(g)
+    torch.cuda.synchronize()
+    return ref, ranks
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_split_step_equals_one_context(name):
+    sizes, W, G = CASES[name]
+    ref, ranks = _run(sizes, W, G)
+    try:
+        want = {k: ref.read(k) for k in (B.OB_STATE_P, B.OB_STATE_M, B.OB_STATE_BITS_SERVER,
+                                          B.OB_STATE_S_SERVER, B.OB_STATE_S_WORKER, B.OB_STATE_STEP)}
+        want_bits = [ref.read(B.OB_STATE_BITS_WORKER, w) for w in range(W)]
+        for r in ranks.ranks:
+            for k, v in want.items():
+                np.testing.assert_array_equal(r.read(k), v, err_msg=f"{name} rank {r.rank} kind {k}")
+            for w in range(W):
+                np.testing.assert_array_equal(r.read(B.OB_STATE_BITS_WORKER, w), want_bits[w])
+            for w in range(r.w_begin, r.w_begin + r.w_local):  # errors live with their worker
+                np.testing.assert_array_equal(r.read(B.OB_STATE_E_WORKER, w),
+                                              ref.read(B.OB_STATE_E_WORKER, w))
+        # the server error of chunk j lives on rank j % G
+        e_ref = ref.read(B.OB_STATE_E_SERVER)
+        offsets, _ = ref.layout()
+        for rk in ranks.ranks:
+            e = rk.read(B.OB_STATE_E_SERVER)
+            for t, n in enumerate(sizes):
+                for j in range(W):
+                    if j % G != rk.rank:
+                        continue
+                    b, end = B.ob_chunk_range(n, W, j)
+                    np.testing.assert_array_equal(e[offsets[t] + b:offsets[t] + end],
+                                                  e_ref[offsets[t] + b:offsets[t] + end])
+    finally:
+        ref.close()
+        ranks.close()
+
+
+def test_split_step_phase_rules():
+    opt = DistributedOneBitAdam([4096], 4, rank=1, world=2, **WL.HYPER)
+    try:
+        ctx = opt.opt.ctx
+        g = torch.zeros((4, 4096), device="cuda")
+        opt.warmup_step(g)
+        with pytest.raises(B.OnebitError) as e:
+            B.ob_server_stage(ctx)                  # before the freeze / worker stage
+        assert e.value.status == B.OB_ERR_PHASE
+        opt.freeze()
+        with pytest.raises(B.OnebitError) as e:
+            B.ob_compressed_step(ctx, [g[w].data_ptr() for w in range(4)])  # sharded context
+        assert e.value.status == B.OB_ERR_PHASE
+        with pytest.raises(B.OnebitError) as e:
+            B.ob_worker_stage(ctx, [0, 0, g[2].data_ptr(), g[3].data_ptr()], 2, 3)  # past W
+        assert e.value.status == B.OB_ERR_INVALID_ARG
+        with pytest.raises(B.OnebitError) as e:
+            B.ob_worker_stage(ctx, [0, 0, 0, g[3].data_ptr()], 2, 2)  # a NULL gradient in range
+        assert e.value.status == B.OB_ERR_INVALID_ARG
+        opt.worker_stage([g[2], g[3]])
+        for call in (lambda: B.ob_worker_stage(ctx, [0, 0, g[2].data_ptr(), g[3].data_ptr()], 2, 2),
+                     lambda: B.ob_apply_update(ctx),
+                     lambda: B.ob_set_server_shard(ctx, 1, 0),
+                     lambda: opt.opt.write(B.OB_STATE_P, 0, np.zeros(4096, np.float32)),
+                     lambda: opt.warmup_step(g)):
+            with pytest.raises(B.OnebitError) as e:
+                call()
+            assert e.value.status == B.OB_ERR_PHASE
+        opt.server_stage()
+        opt.apply_update()
+        assert opt.read(B.OB_STATE_STEP)[1] == 1
+        with pytest.raises(B.OnebitError) as e:
+            B.ob_set_server_shard(ctx, 5, 0)        # more shards than workers
+        assert e.value.status == B.OB_ERR_INVALID_ARG
+    finally:
+        opt.close()
