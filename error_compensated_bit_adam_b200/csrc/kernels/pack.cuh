@@ -25,7 +25,6 @@ struct PackParams {
     double *partial;                 // [W][n_tiles]: sum of x^2 per tile
     int64_t n_pad;
     int W, T;
-    int w_begin, w_end;              // the workers this launch computes (all W: 0, W)
     float beta1, c1;
 };
 
@@ -76,8 +75,8 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
     extern __shared__ float4 pipe[];  // [kPackStages][2 (g, x_prev)][kUnroll][kThreads]
     const uint64_t pol = evict_first_policy();
     auto issue = [&](int w) {
-        if (w < P.w_end) {
-            const int st = (w - P.w_begin) % kPackStages;
+        if (w < P.W) {
+            const int st = w % kPackStages;
             const float *gw = P.g[w] + (tile.begin - P.g_offset);
             const float *xw = P.x + (int64_t)w * P.n_pad + tile.begin;
 #pragma unroll
@@ -92,11 +91,11 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
         cp_async_commit();  // one group per worker, empty past the last
     };
 #pragma unroll
-    for (int k = 0; k < kPackStages - 1; ++k) issue(P.w_begin + k);
-    for (int w = P.w_begin; w < P.w_end; ++w) {
+    for (int k = 0; k < kPackStages - 1; ++k) issue(k);
+    for (int w = 0; w < P.W; ++w) {
         issue(w + kPackStages - 1);
         cp_async_wait<kPackStages - 1>();  // worker w's group has landed
-        const int st = (w - P.w_begin) % kPackStages;
+        const int st = w % kPackStages;
         const float s_prev = P.s_prev[w * P.T + tile.tensor];
         float *xw = P.x + (int64_t)w * P.n_pad + tile.begin;
         uint32_t *bw = P.bits + (int64_t)w * words_per_worker + (tile.begin >> 5);
@@ -136,7 +135,7 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
         if (lane == 0) red[warp][w] = t;
     }
     __syncthreads();
-    if (tid >= P.w_begin && tid < P.w_end) {
+    if (tid < P.W) {
         double acc = 0.0;
 #pragma unroll
         for (int k = 0; k < kWarps; ++k) acc += red[k][tid];

@@ -81,7 +81,6 @@ struct ScaleParams {
     unsigned *counter;         // [R][rows], zero between launches
     float *out_prev, *out_last;
     int rows;                  // workers (worker scales) or 1 (server scales)
-    int row_base;              // row of blockIdx.y == 0
     int R;
     int out_stride_r, out_stride_row;  // out[r * stride_r + row * stride_row]
 };
@@ -89,7 +88,7 @@ struct ScaleParams {
 // Grid (R, rows, segments): worker scales use ranges = tensors and one row
 // per worker; server scales use ranges = (tensor, chunk) and one row.
 __global__ void __launch_bounds__(kScaleThreads) ob_scale_kernel(const __grid_constant__ ScaleParams P) {
-    const int r = blockIdx.x, row = P.row_base + (int)blockIdx.y, seg = blockIdx.z;
+    const int r = blockIdx.x, row = blockIdx.y, seg = blockIdx.z;
     const int lo = P.range_begin[r], hi = P.range_begin[r + 1];
     const int nseg = num_segments(hi - lo);
     if (seg >= nseg) return;

@@ -23,7 +23,6 @@ struct ServerParams {
     int W, T;
     float inv_w;            // 1/W when W is a power of two (then acc*inv_w == acc/W exactly)
     int w_pow2;
-    int owner_mod, owner_rem;  // served chunks: chunk % owner_mod == owner_rem (all when owner_mod == 1)
 };
 
 // Two independent IEEE round-to-nearest additions in one instruction
@@ -137,14 +136,6 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
     const int tid = threadIdx.x;
     const int64_t words_per_worker = P.n_pad >> 5;
     const int64_t word0 = tile.begin >> 5;
-    if (P.owner_mod > 1 && tile.chunk % P.owner_mod != P.owner_rem) {
-        // another process serves this chunk: its words are zero here (the
-        // exchange sums every process's words, and chunks never share a
-        // word) and it adds nothing to this process's server scales
-        for (int k = tid; k < ((tile.count + 31) >> 5); k += kThreads) P.sbits[word0 + k] = 0u;
-        if (tid == 0) P.partial[tile_id] = 0.0;
-        return;
-    }
     const int groups = (((tile.count + 31) >> 5) + 3) >> 2;  // 16-byte word groups with real elements
 
     for (int idx = tid; idx < P.W * (kTileWords / 4); idx += kThreads) {

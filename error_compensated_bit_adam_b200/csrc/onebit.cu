@@ -300,12 +300,7 @@ struct ob_ctx {
     bool use_graph = false;
     StepGraph graph;
     bool broken = false;
-    // workers computed by the worker stage (all of them unless a split step
-    // narrows the range), and the server chunks this context serves: chunk j
-    // of every tensor when j % shard_G == shard_rank (all when shard_G == 1)
-    int w_begin = 0, w_end = 0;
-    int shard_G = 1, shard_rank = 0;
-    // split step: 0 idle, 1 after ob_worker_stage, 2 after ob_server_stage
+    // split step (ob_worker_stage ... ob_finish_step): 1 while one is open
     int split_stage = 0;
     // profiling
     bool profiling = false;
@@ -419,8 +414,6 @@ onebit::PackParams pack_params(const ob_ctx *c, const float *const *g, int64_t g
     P.n_pad = c->plan.n_pad;
     P.W = c->plan.W;
     P.T = c->plan.T;
-    P.w_begin = c->w_begin;
-    P.w_end = c->w_end;
     P.beta1 = c->beta1;
     P.c1 = c->c1;
     return P;
@@ -438,7 +431,6 @@ onebit::ScaleParams worker_scale_params(const ob_ctx *c) {
     P.out_prev = c->s_prev();
     P.out_last = c->s_last();
     P.rows = c->plan.W;
-    P.row_base = c->w_begin;
     P.R = c->plan.T;
     P.out_stride_r = 1;
     P.out_stride_row = c->plan.T;
@@ -460,8 +452,6 @@ onebit::ServerParams server_params(const ob_ctx *c) {
     P.T = c->plan.T;
     P.w_pow2 = (W & (W - 1)) == 0;
     P.inv_w = 1.0f / (float)W;  // exact for a power of two
-    P.owner_mod = c->shard_G;
-    P.owner_rem = c->shard_rank;
     return P;
 }
 
@@ -503,7 +493,7 @@ struct Geometry {
 };
 Geometry pack_geometry(int tiles) { return {grid1(tiles), dim3(kThreads), (size_t)onebit::kPackSmemBytes}; }
 Geometry worker_scale_geometry(const ob_ctx *c) {
-    return {dim3((unsigned)c->plan.T, (unsigned)(c->w_end - c->w_begin), (unsigned)c->plan.tensor_max_seg),
+    return {dim3((unsigned)c->plan.T, (unsigned)c->plan.W, (unsigned)c->plan.tensor_max_seg),
             dim3(kScaleThreads), 0};
 }
 Geometry server_geometry(const ob_ctx *c) {
@@ -524,19 +514,19 @@ ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int ti
     return fail_cuda(c, cudaGetLastError());
 }
 
-// The worker scales of the workers [w_begin, w_end).
-ob_status launch_worker_scales(ob_ctx *c) {
-    if (c->w_end <= c->w_begin) return OB_OK;
-    KernelTimer k(c, OB_K_PACK_SCALE);
-    const Geometry G = worker_scale_geometry(c);
-    onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(worker_scale_params(c));
-    k.stop();
-    return fail_cuda(c, cudaGetLastError());
-}
-
-// The server stage of the chunks this context serves, and their scales.
-ob_status launch_server(ob_ctx *c) {
-    if (c->n_tiles() > 0) {
+// Everything of a compressed step after the worker stage's tile kernels.
+ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
+    const int nt = c->n_tiles();
+    pack_timer.stop();
+    {
+        KernelTimer k(c, OB_K_PACK_SCALE);
+        const Geometry G = worker_scale_geometry(c);
+        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(worker_scale_params(c));
+        k.stop();
+        ob_status st = fail_cuda(c, cudaGetLastError());
+        if (st != OB_OK) return st;
+    }
+    if (nt > 0) {
         KernelTimer k(c, OB_K_SERVER);
         const Geometry G = server_geometry(c);
         onebit::ob_server_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_params(c));
@@ -544,30 +534,23 @@ ob_status launch_server(ob_ctx *c) {
         ob_status st = fail_cuda(c, cudaGetLastError());
         if (st != OB_OK) return st;
     }
-    KernelTimer k(c, OB_K_SERVER_SCALE);
-    const Geometry G = server_scale_geometry(c);
-    onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_scale_params(c));
-    k.stop();
-    return fail_cuda(c, cudaGetLastError());
-}
-
-// Gather and update.
-ob_status launch_apply(ob_ctx *c) {
-    if (c->n_tiles() == 0) return OB_OK;
-    KernelTimer k(c, OB_K_APPLY);
-    const Geometry G = apply_geometry(c);
-    onebit::ob_apply_kernel<<<G.grid, G.block, G.smem, c->stream>>>(apply_params(c));
-    k.stop();
-    return fail_cuda(c, cudaGetLastError());
-}
-
-// Everything of a compressed step after the worker stage's tile kernels.
-ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
-    pack_timer.stop();
-    ob_status st = launch_worker_scales(c);
-    if (st == OB_OK) st = launch_server(c);
-    if (st == OB_OK) st = launch_apply(c);
-    return st;
+    {
+        KernelTimer k(c, OB_K_SERVER_SCALE);
+        const Geometry G = server_scale_geometry(c);
+        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_scale_params(c));
+        k.stop();
+        ob_status st = fail_cuda(c, cudaGetLastError());
+        if (st != OB_OK) return st;
+    }
+    if (nt > 0) {
+        KernelTimer k(c, OB_K_APPLY);
+        const Geometry G = apply_geometry(c);
+        onebit::ob_apply_kernel<<<G.grid, G.block, G.smem, c->stream>>>(apply_params(c));
+        k.stop();
+        ob_status st = fail_cuda(c, cudaGetLastError());
+        if (st != OB_OK) return st;
+    }
+    return OB_OK;
 }
 
 // ------------------------------------------------------------- graph mode
@@ -661,10 +644,10 @@ ob_status graph_step(ob_ctx *c, const float *const *g) {
     return fail_cuda(c, e);
 }
 
-ob_status check_grads(const ob_ctx *c, const float *const *g, int w_begin, int w_end) {
+ob_status check_grads(const ob_ctx *c, const float *const *g) {
     if (!g) return OB_ERR_INVALID_ARG;
     if (c->plan.n_pad == 0) return OB_OK;  // nothing is read
-    for (int w = w_begin; w < w_end; ++w) {
+    for (int w = 0; w < c->plan.W; ++w) {
         if (!g[w]) return OB_ERR_INVALID_ARG;
         if (!aligned(g[w], 16)) return OB_ERR_ALIGN;
     }
@@ -853,8 +836,6 @@ ob_status ob_create(int n_tensors, const int64_t *numel, int W, float beta1, flo
     c->params = d_params;
     c->ws = static_cast<char *>(d_workspace);
     c->stream = static_cast<cudaStream_t>(cuda_stream);
-    c->w_begin = 0;
-    c->w_end = c->plan.W;
     // Release what was created so far and report `status`.
     auto bail = [&](ob_status status) {
         if (c->copy_stream) cudaStreamDestroy(c->copy_stream);
@@ -941,7 +922,7 @@ ob_status ob_warmup_adam_step(ob_ctx *c, const float *const *d_grads) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
-    if ((st = check_grads(c, d_grads, 0, c->plan.W)) != OB_OK) return st;
+    if ((st = check_grads(c, d_grads)) != OB_OK) return st;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
     if ((st = materialize_momentum(c)) != OB_OK) return st;
@@ -998,8 +979,8 @@ ob_status ob_freeze_variance(ob_ctx *c) {
 ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
-    if (!c->frozen || c->split_stage != 0 || c->shard_G != 1) return OB_ERR_PHASE;
-    if ((st = check_grads(c, d_grads, 0, c->plan.W)) != OB_OK) return st;
+    if (!c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
+    if ((st = check_grads(c, d_grads)) != OB_OK) return st;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
     if (c->use_graph && !c->profiling) {
@@ -1016,39 +997,54 @@ ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
 
 // ------------------------------------------------------- the split step
 //
-// One compressed step in three calls, for a data-parallel run in which each
-// process computes some of the workers and serves some of the server
-// chunks; the caller's collectives run between the calls (see onebit.h).
-
-ob_status ob_set_server_shard(ob_ctx *c, int n_shards, int shard) {
-    ob_status st = check_ctx(c);
-    if (st != OB_OK) return st;
-    if (n_shards < 1 || n_shards > c->plan.W || shard < 0 || shard >= n_shards) return OB_ERR_INVALID_ARG;
-    if (c->split_stage != 0) return OB_ERR_PHASE;
-    c->shard_G = n_shards;
-    c->shard_rank = shard;
-    return OB_OK;
-}
+// One compressed step in two calls for a data-parallel run in which each
+// process computes some of the workers (see onebit.h).  Host code only:
+// the step's own kernels, the worker-stage ones launched on a view of the
+// worker rows [w_begin, w_begin + w_count) as if those were all workers.
 
 ob_status ob_worker_stage(ob_ctx *c, const float *const *d_grads, int w_begin, int w_count) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (!c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
-    if (w_begin < 0 || w_count < 0 || w_begin > c->plan.W - w_count) return OB_ERR_INVALID_ARG;
-    if ((st = check_grads(c, d_grads, w_begin, w_begin + w_count)) != OB_OK) return st;
+    const int W = c->plan.W;
+    if (w_begin < 0 || w_count < 0 || w_begin > W - w_count || !d_grads) return OB_ERR_INVALID_ARG;
+    if (c->plan.n_pad > 0)
+        for (int w = w_begin; w < w_begin + w_count; ++w) {
+            if (!d_grads[w]) return OB_ERR_INVALID_ARG;
+            if (!aligned(d_grads[w], 16)) return OB_ERR_ALIGN;
+        }
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
-    c->w_begin = w_begin;
-    c->w_end = w_begin + w_count;
-    if (w_count > 0) {
-        KernelTimer pack(c, OB_K_PACK);
-        st = launch_pack(c, d_grads, 0, 0, c->n_tiles());
-        pack.stop();
+    // The worker stage reads m densely here: its lazy decode indexes the
+    // server scales by the worker count, which the view changes.
+    if ((st = materialize_momentum(c)) != OB_OK) return st;
+    const size_t n = (size_t)c->plan.n_pad, T = (size_t)c->plan.T, nt = (size_t)c->n_tiles();
+    if (w_count > 0 && nt > 0) {
+        onebit::PackParams P = pack_params(c, d_grads, 0, 0);
+        for (int i = 0; i < OB_MAX_WORKERS; ++i) P.g[i] = i < w_count ? d_grads[w_begin + i] : nullptr;
+        P.x = c->x() + (size_t)w_begin * n;
+        P.bits = c->bits() + (size_t)w_begin * (n / 32);
+        P.s_prev = c->s_prev() + (size_t)w_begin * T;
+        P.partial = c->partial_w() + (size_t)w_begin * nt;
+        P.W = w_count;
+        KernelTimer k(c, OB_K_PACK);
+        const Geometry G = pack_geometry((int)nt);
+        onebit::ob_pack_kernel<<<G.grid, G.block, G.smem, c->stream>>>(P);
+        k.stop();
+        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
     }
-    if (st == OB_OK) st = launch_worker_scales(c);
-    c->w_begin = 0;
-    c->w_end = c->plan.W;
-    if (st != OB_OK) return st;
+    if (w_count > 0) {
+        onebit::ScaleParams S = worker_scale_params(c);
+        S.partial = c->partial_w() + (size_t)w_begin * nt;
+        S.out_prev = c->s_prev() + (size_t)w_begin * T;
+        S.out_last = c->s_last() + (size_t)w_begin * T;
+        S.rows = w_count;
+        KernelTimer k(c, OB_K_PACK_SCALE);
+        const dim3 grid((unsigned)T, (unsigned)w_count, (unsigned)c->plan.tensor_max_seg);
+        onebit::ob_scale_kernel<<<grid, dim3(kScaleThreads), 0, c->stream>>>(S);
+        k.stop();
+        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
+    }
     c->split_stage = 1;
     return OB_OK;
 }
@@ -1065,46 +1061,39 @@ ob_status ob_worker_exchange_buffers(ob_ctx *c, uint32_t **d_bits, size_t *bits_
     return OB_OK;
 }
 
-ob_status ob_server_stage(ob_ctx *c) {
+ob_status ob_finish_step(ob_ctx *c) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (c->split_stage != 1) return OB_ERR_PHASE;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
-    // the exchange filled the scale rows of the workers computed elsewhere;
-    // keep the copy that S_WORKER reads in step with them
+    // the exchange filled the other workers' rows of s_prev; S_WORKER reads
+    // the copy in s_last
     cudaError_t e = cudaMemcpyAsync(c->s_last(), c->s_prev(), (size_t)c->plan.W * c->plan.T * 4,
                                     cudaMemcpyDeviceToDevice, c->stream);
     if ((st = fail_cuda(c, e)) != OB_OK) return st;
-    if ((st = launch_server(c)) != OB_OK) return st;
-    c->split_stage = 2;
-    return OB_OK;
-}
-
-ob_status ob_server_exchange_buffers(ob_ctx *c, uint32_t **d_sbits, size_t *sbits_bytes,
-                                     float **d_scales, size_t *scales_bytes) {
-    ob_status st = check_ctx(c);
-    if (st != OB_OK) return st;
-    if (!d_sbits || !sbits_bytes || !d_scales || !scales_bytes) return OB_ERR_INVALID_ARG;
-    *d_sbits = c->sbits();
-    *sbits_bytes = (size_t)(c->plan.n_pad / 32) * 4;
-    *d_scales = c->sp_last();
-    *scales_bytes = (size_t)c->plan.T * c->plan.W * 4;
-    return OB_OK;
-}
-
-ob_status ob_apply_update(ob_ctx *c) {
-    ob_status st = check_ctx(c);
-    if (st != OB_OK) return st;
-    if (c->split_stage != 2) return OB_ERR_PHASE;
-    DeviceGuard dg(c->device);
-    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
-    // the exchange completed the scales in sp_last; the next server stage
-    // decodes its y_prev with sp_prev
-    cudaError_t e = cudaMemcpyAsync(c->sp_prev(), c->sp_last(), (size_t)c->plan.T * c->plan.W * 4,
-                                    cudaMemcpyDeviceToDevice, c->stream);
-    if ((st = fail_cuda(c, e)) != OB_OK) return st;
-    if ((st = launch_apply(c)) != OB_OK) return st;
+    const int nt = c->n_tiles();
+    if (nt > 0) {
+        KernelTimer k(c, OB_K_SERVER);
+        const Geometry G = server_geometry(c);
+        onebit::ob_server_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_params(c));
+        k.stop();
+        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
+    }
+    {
+        KernelTimer k(c, OB_K_SERVER_SCALE);
+        const Geometry G = server_scale_geometry(c);
+        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_scale_params(c));
+        k.stop();
+        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
+    }
+    if (nt > 0) {
+        KernelTimer k(c, OB_K_APPLY);
+        const Geometry G = apply_geometry(c);
+        onebit::ob_apply_kernel<<<G.grid, G.block, G.smem, c->stream>>>(apply_params(c));
+        k.stop();
+        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
+    }
     c->split_stage = 0;
     c->m_dense = false;
     c->t_compressed += 1;
@@ -1138,7 +1127,7 @@ ob_status ob_compressed_step_host(ob_ctx *c, const float *const *h_grads, void *
                                   size_t staging_bytes, float *h_server_scales) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
-    if (!c->frozen || c->split_stage != 0 || c->shard_G != 1) return OB_ERR_PHASE;
+    if (!c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
     if (!h_grads || !d_staging) return OB_ERR_INVALID_ARG;
     for (int w = 0; w < c->plan.W; ++w)
         if (!h_grads[w]) return OB_ERR_INVALID_ARG;

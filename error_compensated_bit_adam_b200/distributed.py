@@ -3,25 +3,24 @@
 The compressed collective of the review page "1-bit Adam: Communication
 Efficient Large-Scale Training with Adam's Convergence Speed" ("Proposed
 method", 4) has a worker stage (every worker compresses its momentum and
-sends server j the part of its words that chunk j covers) and a server
-stage (server j averages its chunk, compresses it again and sends the
-result to every worker).  Here process r of G computes workers
-[r W/G, (r+1) W/G) and serves the chunks j with j % G == r; between the
-library's three calls (ob_worker_stage, ob_server_stage, ob_apply_update)
-the process exchanges
+sends its words and scale onward) and a server stage (the compressed
+momenta are averaged, compressed again and returned to every worker).
+Here process r of G computes the worker stage of workers
+[r W/G, (r+1) W/G) with ob_worker_stage, the worker rows (sign words and
+scales) are all-gathered, and every process then runs the server stage of
+every chunk and the update with ob_finish_step.  Given the same rows, every
+process computes the same server words, so nothing is sent back, and every
+process ends the step with the same parameters, bit for bit equal to one
+ob_compressed_step over all W workers.
 
-  * the worker rows (sign words and scales) by an all-gather, and
-  * the server words and scales by a sum-all-reduce: every process holds
-    zeros in the chunks it does not serve, so the sums are exact.
-
-The all-gather sends every worker's full row to every process, where the
-pages send each server only its chunk: W/G times more bytes for the same
-result, in exchange for one collective over the library's own layout.
-Every process ends the step with the same parameters, bit for bit equal to
-one ob_compressed_step over all W workers.
+Against the pages' exchange (each server receives only its chunk of every
+worker's words and returns its chunk to every worker) this sends each
+process every worker's whole row and repeats the server stage on every
+process: one collective over the library's own layout, and no kernel
+beyond the single-GPU step's.
 
 LocalRanks runs the same split step for G ranks inside one process on one
-GPU, each rank a context of its own, with the exchange done by device
+GPU, each rank a context of its own, with the all-gather done by device
 copies: the single-GPU form of the path, used to check it against one
 context and to time each rank's share of the work.
 """
@@ -43,9 +42,9 @@ def _view(workspace: torch.Tensor, ptr: int, nbytes: int, dtype: torch.dtype) ->
 
 
 class TorchExchange:
-    """The split step's two exchanges over a torch.distributed group (NCCL
-    for CUDA tensors, gloo for CPU tensors).  Collectives run on the current
-    stream; every rank calls them in the same order."""
+    """The split step's exchange over a torch.distributed group (NCCL for
+    CUDA tensors, gloo for CPU tensors).  The collective runs on the current
+    stream; every rank calls it in the same order."""
 
     def __init__(self, group=None):
         import torch.distributed as dist
@@ -62,9 +61,6 @@ class TorchExchange:
         mine = rows[begin:begin + count].view(-1)
         self.dist.all_gather_into_tensor(flat, mine, group=self.group)
 
-    def sum_(self, buf: torch.Tensor) -> None:
-        self.dist.all_reduce(buf, op=self.dist.ReduceOp.SUM, group=self.group)
-
 
 class DistributedOneBitAdam:
     """One process's part of a data-parallel 1-bit Adam run.
@@ -73,7 +69,7 @@ class DistributedOneBitAdam:
     process keeps a context over the whole tensor list with all W workers
     (parameters, momentum and variance are the same everywhere).  The phase
     methods below are the split step; ``step`` runs them with ``exchange``
-    (a TorchExchange by default)."""
+    (a TorchExchange by default) between the two library calls."""
 
     def __init__(self, numel: Sequence[int], W: int, *, rank: int, world: int, exchange=None,
                  device=None, stream: Optional[torch.cuda.Stream] = None, **hyper):
@@ -83,16 +79,12 @@ class DistributedOneBitAdam:
         self.W = int(W)
         self.w_local = self.W // self.world
         self.w_begin = self.rank * self.w_local
-        self.exchange = exchange
+        self.exchange_impl = exchange
         self.opt = OneBitAdam(numel, W, device=device, stream=stream, **hyper)
         ctx, ws = self.opt.ctx, self.opt.workspace
-        B.ob_set_server_shard(ctx, self.world, self.rank)
         bits, bits_row, scales, scales_row = B.ob_worker_exchange_buffers(ctx)
         self.worker_bits = _view(ws, bits, self.W * bits_row, torch.int32).view(self.W, -1)
         self.worker_scales = _view(ws, scales, self.W * scales_row, torch.float32).view(self.W, -1)
-        sbits, sbits_bytes, sp, sp_bytes = B.ob_server_exchange_buffers(ctx)
-        self.server_bits = _view(ws, sbits, sbits_bytes, torch.int32)
-        self.server_scales = _view(ws, sp, sp_bytes, torch.float32)
 
     @property
     def params(self) -> torch.Tensor:
@@ -126,31 +118,23 @@ class DistributedOneBitAdam:
             ptrs[self.w_begin + i] = g.data_ptr()
         B.ob_worker_stage(self.opt.ctx, ptrs, self.w_begin, self.w_local)
 
-    def server_stage(self) -> None:
-        B.ob_server_stage(self.opt.ctx)
+    def finish_step(self) -> None:
+        B.ob_finish_step(self.opt.ctx)
 
-    def apply_update(self) -> None:
-        B.ob_apply_update(self.opt.ctx)
+    def exchange(self, ex) -> None:
+        ex.gather_rows(self.worker_bits, self.w_begin, self.w_local)
+        ex.gather_rows(self.worker_scales, self.w_begin, self.w_local)
 
     def step(self, local_grads: Sequence[torch.Tensor]) -> None:
-        ex = self.exchange if self.exchange is not None else TorchExchange()
+        ex = self.exchange_impl if self.exchange_impl is not None else TorchExchange()
         with torch.cuda.stream(self.opt.stream):
             self.worker_stage(local_grads)
-            ex.gather_rows(self.worker_bits, self.w_begin, self.w_local)
-            ex.gather_rows(self.worker_scales, self.w_begin, self.w_local)
-            self.server_stage()
-            ex.sum_(self.server_bits)
-            ex.sum_(self.server_scales)
-            self.apply_update()
+            self.exchange(ex)
+            self.finish_step()
 
-    def exchange_bytes(self) -> dict:
-        """Bytes each exchange moves into this process per step."""
-        row_bits = self.worker_bits.shape[1] * 4
-        row_scales = self.worker_scales.shape[1] * 4
-        others = self.W - self.w_local
-        return {"worker_rows_gathered": others * (row_bits + row_scales),
-                "server_words_and_scales_summed": self.server_bits.numel() * 4
-                + self.server_scales.numel() * 4}
+    def exchange_bytes(self) -> int:
+        """Bytes the all-gather brings into this process per step."""
+        return (self.W - self.w_local) * (self.worker_bits.shape[1] + self.worker_scales.shape[1]) * 4
 
     def read(self, kind: int, index: int = 0):
         return self.opt.read(kind, index)
@@ -161,9 +145,9 @@ class DistributedOneBitAdam:
 
 class LocalRanks:
     """G ranks of the split step in one process on one GPU, stepped in
-    lockstep; the exchanges are device copies and sums.  No kernel of one
-    rank waits for another's: each call finishes its rank's launches before
-    the next rank's are queued on the same stream."""
+    lockstep; the all-gather is device copies.  No kernel of one rank waits
+    for another's: the ranks' launches are queued one after another on the
+    same stream."""
 
     def __init__(self, numel: Sequence[int], W: int, G: int, device=None, **hyper):
         self.G, self.W = int(G), int(W)
@@ -182,18 +166,11 @@ class LocalRanks:
             r.freeze()
 
     def _gather_rows(self, attr: str) -> None:
-        blocks = [getattr(r, attr)[r.w_begin:r.w_begin + r.w_local] for r in self.ranks]
         for dst in self.ranks:
-            for src, blk in zip(self.ranks, blocks):
+            for src in self.ranks:
                 if src is not dst:
-                    getattr(dst, attr)[src.w_begin:src.w_begin + src.w_local].copy_(blk)
-
-    def _sum(self, attr: str) -> None:
-        total = getattr(self.ranks[0], attr).clone()
-        for r in self.ranks[1:]:
-            total += getattr(r, attr)
-        for r in self.ranks:
-            getattr(r, attr).copy_(total)
+                    rows = slice(src.w_begin, src.w_begin + src.w_local)
+                    getattr(dst, attr)[rows].copy_(getattr(src, attr)[rows])
 
     def step(self, all_grads: torch.Tensor) -> None:
         """all_grads: [W, n_padded]; rank r gets its workers' rows."""
@@ -202,11 +179,7 @@ class LocalRanks:
         self._gather_rows("worker_bits")
         self._gather_rows("worker_scales")
         for r in self.ranks:
-            r.server_stage()
-        self._sum("server_bits")
-        self._sum("server_scales")
-        for r in self.ranks:
-            r.apply_update()
+            r.finish_step()
 
     def close(self) -> None:
         for r in self.ranks:

@@ -200,44 +200,36 @@ OB_API ob_status ob_compressed_step_host(ob_ctx *ctx, const float *const *h_grad
                                   size_t staging_bytes, float *h_server_scales);
 
 /* --------------------------------------------------------------------
- * The split step: one compressed step in three calls, for a data-parallel
- * run over G processes (one per GPU) in which process r computes workers
- * [w_begin, w_begin + w_count) and serves the server chunks j with
- * j % G == r of every tensor -- the worker stage and the server stage of
- * the compressed collective [1BA, Proposed method, 4] with the exchange
- * between them done by the caller's collectives:
+ * The split step: one compressed step in two calls, for a data-parallel
+ * run over G processes (one per GPU) in which process r computes the
+ * workers [w_begin, w_begin + w_count) -- the worker stage of the
+ * compressed collective [1BA, Proposed method, 4] -- and the caller moves
+ * their outputs to the other processes in between:
  *
- *   ob_set_server_shard(ctx, G, r)                    once
  *   per step:
  *     ob_worker_stage(ctx, d_grads, w_begin, w_count)
  *     all-gather of the worker rows of ob_worker_exchange_buffers
- *     ob_server_stage(ctx)
- *     sum-all-reduce of ob_server_exchange_buffers (words as 32-bit
- *       integers, scales as floats)
- *     ob_apply_update(ctx)
+ *     ob_finish_step(ctx)       server stage, gather and update
  *
  * Every process holds a context over the whole tensor list with all W
- * workers (the rows of other processes' workers are filled by the
- * exchange); p, m and d are the same on every process.  The result equals
- * ob_compressed_step of one context with the same W bit for bit: the sums
- * of the exchange add exact zeros to each word and scale.  With G = 1 and
- * no collectives the three calls are ob_compressed_step.  While a split
- * step is open (between ob_worker_stage and ob_apply_update) only these
- * calls, ob_read_state and ob_destroy are accepted; ob_compressed_step and
- * ob_compressed_step_host need G = 1.  Warmup steps need the gradients of
- * all W workers on every process (the warmup averages them in worker
- * order). */
-
-/* Serve the chunks j with j % n_shards == shard (1 <= n_shards <= W,
- * 0 <= shard < n_shards).  Default: n_shards = 1 (every chunk).
- * OB_ERR_PHASE inside a split step. */
-OB_API ob_status ob_set_server_shard(ob_ctx *ctx, int n_shards, int shard);
+ * workers' rows and runs the server stage of every chunk itself: with the
+ * same inputs every process computes the same server words, so nothing has
+ * to be sent back.  p, m and d stay the same on every process, and the
+ * result equals ob_compressed_step over all W workers bit for bit.  While
+ * a split step is open (between the two calls) only ob_finish_step,
+ * ob_worker_exchange_buffers, ob_read_state and ob_destroy are accepted;
+ * the other step calls and ob_write_state return OB_ERR_PHASE.  Warmup
+ * steps need the gradients of all W workers on every process (the warmup
+ * averages them in worker order). */
 
 /* Worker stage of workers [w_begin, w_begin + w_count) (w_count may be 0):
  * momentum, error feedback, 1-bit compression and worker scales, as in
  * ob_compressed_step.  d_grads: host array of W device pointers, only the
- * entries of the range read (the others may be NULL).  OB_ERR_PHASE before
- * the freeze or inside a split step. */
+ * entries of the range read (the others may be NULL).  The momentum is
+ * first decoded into its dense buffer (one extra pass of 4 bytes per
+ * parameter).  OB_ERR_PHASE before the freeze or while a split step is
+ * open; OB_ERR_INVALID_ARG for a range outside [0, W) or a NULL gradient
+ * in it. */
 OB_API ob_status ob_worker_stage(ob_ctx *ctx, const float *const *d_grads, int w_begin, int w_count);
 
 /* Device buffers of the worker stage's outputs, one row per worker, rows
@@ -247,22 +239,11 @@ OB_API ob_status ob_worker_stage(ob_ctx *ctx, const float *const *d_grads, int w
 OB_API ob_status ob_worker_exchange_buffers(ob_ctx *ctx, uint32_t **d_bits, size_t *bits_row_bytes,
                                             float **d_scales, size_t *scales_row_bytes);
 
-/* Server stage of the served chunks (all worker rows must hold this step's
- * words and scales): average, server error, re-compression and server
- * scales.  The words of chunks served elsewhere are set to 0 and their
- * scales to 0.  OB_ERR_PHASE unless ob_worker_stage came before. */
-OB_API ob_status ob_server_stage(ob_ctx *ctx);
-
-/* Device buffers of the server stage's outputs: *d_sbits uint32[n_padded/32]
- * server sign words, *d_scales float[n_tensors][W] server scales.  Owned
- * by the context; valid until ob_destroy. */
-OB_API ob_status ob_server_exchange_buffers(ob_ctx *ctx, uint32_t **d_sbits, size_t *sbits_bytes,
-                                            float **d_scales, size_t *scales_bytes);
-
-/* Gather and update with every chunk's words and scales present: closes
- * the split step (the compressed step count advances).  OB_ERR_PHASE unless
- * ob_server_stage came before. */
-OB_API ob_status ob_apply_update(ob_ctx *ctx);
+/* Close the split step once every worker row holds this step's words and
+ * scales: server stage, server scales, gather and update, as in
+ * ob_compressed_step (the compressed step count advances).  OB_ERR_PHASE
+ * unless ob_worker_stage came before. */
+OB_API ob_status ob_finish_step(ob_ctx *ctx);
 
 /* Copy one piece of state to host memory.  kind: ob_state_kind.  index:
  * the worker for OB_STATE_E_WORKER / OB_STATE_BITS_WORKER, else 0.  bytes:

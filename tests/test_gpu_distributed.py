@@ -1,9 +1,9 @@
-"""The split step (ob_worker_stage / ob_server_stage / ob_apply_update with
-the exchanges between them) against one ob_compressed_step context.
+"""The split step (ob_worker_stage, the all-gather of the worker rows,
+ob_finish_step) against one ob_compressed_step context.
 
 G ranks run in one process on one GPU (distributed.LocalRanks), each with
-its own context, the exchanges done by device copies and sums.  The bar is
-bit for bit: parameters, momentum, the server words and scales, and every
+its own context, the all-gather done by device copies.  The bar is bit for
+bit: parameters, momentum, the server words, scales and error, and every
 worker's words and scales on every rank, after warmup, freeze and several
 compressed steps with fresh gradients."""
 import numpy as np
@@ -62,7 +62,8 @@ def test_split_step_equals_one_context(name):
     ref, ranks = _run(sizes, W, G)
     try:
         want = {k: ref.read(k) for k in (B.OB_STATE_P, B.OB_STATE_M, B.OB_STATE_BITS_SERVER,
-                                          B.OB_STATE_S_SERVER, B.OB_STATE_S_WORKER, B.OB_STATE_STEP)}
+                                          B.OB_STATE_S_SERVER, B.OB_STATE_E_SERVER,
+                                          B.OB_STATE_S_WORKER, B.OB_STATE_STEP)}
         want_bits = [ref.read(B.OB_STATE_BITS_WORKER, w) for w in range(W)]
         for r in ranks.ranks:
             for k, v in want.items():
@@ -72,18 +73,6 @@ def test_split_step_equals_one_context(name):
             for w in range(r.w_begin, r.w_begin + r.w_local):  # errors live with their worker
                 np.testing.assert_array_equal(r.read(B.OB_STATE_E_WORKER, w),
                                               ref.read(B.OB_STATE_E_WORKER, w))
-        # the server error of chunk j lives on rank j % G
-        e_ref = ref.read(B.OB_STATE_E_SERVER)
-        offsets, _ = ref.layout()
-        for rk in ranks.ranks:
-            e = rk.read(B.OB_STATE_E_SERVER)
-            for t, n in enumerate(sizes):
-                for j in range(W):
-                    if j % G != rk.rank:
-                        continue
-                    b, end = B.ob_chunk_range(n, W, j)
-                    np.testing.assert_array_equal(e[offsets[t] + b:offsets[t] + end],
-                                                  e_ref[offsets[t] + b:offsets[t] + end])
     finally:
         ref.close()
         ranks.close()
@@ -94,34 +83,37 @@ def test_split_step_phase_rules():
     try:
         ctx = opt.opt.ctx
         g = torch.zeros((4, 4096), device="cuda")
+        ptrs = [0, 0, g[2].data_ptr(), g[3].data_ptr()]
         opt.warmup_step(g)
-        with pytest.raises(B.OnebitError) as e:
-            B.ob_server_stage(ctx)                  # before the freeze / worker stage
-        assert e.value.status == B.OB_ERR_PHASE
+        for call in (lambda: B.ob_worker_stage(ctx, ptrs, 2, 2),  # before the freeze
+                     lambda: B.ob_finish_step(ctx)):
+            with pytest.raises(B.OnebitError) as e:
+                call()
+            assert e.value.status == B.OB_ERR_PHASE
         opt.freeze()
-        with pytest.raises(B.OnebitError) as e:
-            B.ob_compressed_step(ctx, [g[w].data_ptr() for w in range(4)])  # sharded context
-        assert e.value.status == B.OB_ERR_PHASE
-        with pytest.raises(B.OnebitError) as e:
-            B.ob_worker_stage(ctx, [0, 0, g[2].data_ptr(), g[3].data_ptr()], 2, 3)  # past W
-        assert e.value.status == B.OB_ERR_INVALID_ARG
+        for bad in ((2, 3), (-1, 1)):                          # outside [0, W)
+            with pytest.raises(B.OnebitError) as e:
+                B.ob_worker_stage(ctx, ptrs, *bad)
+            assert e.value.status == B.OB_ERR_INVALID_ARG
         with pytest.raises(B.OnebitError) as e:
             B.ob_worker_stage(ctx, [0, 0, 0, g[3].data_ptr()], 2, 2)  # a NULL gradient in range
         assert e.value.status == B.OB_ERR_INVALID_ARG
         opt.worker_stage([g[2], g[3]])
-        for call in (lambda: B.ob_worker_stage(ctx, [0, 0, g[2].data_ptr(), g[3].data_ptr()], 2, 2),
-                     lambda: B.ob_apply_update(ctx),
-                     lambda: B.ob_set_server_shard(ctx, 1, 0),
+        for call in (lambda: B.ob_worker_stage(ctx, ptrs, 2, 2),
+                     lambda: B.ob_compressed_step(ctx, [g[w].data_ptr() for w in range(4)]),
                      lambda: opt.opt.write(B.OB_STATE_P, 0, np.zeros(4096, np.float32)),
                      lambda: opt.warmup_step(g)):
             with pytest.raises(B.OnebitError) as e:
                 call()
             assert e.value.status == B.OB_ERR_PHASE
-        opt.server_stage()
-        opt.apply_update()
+        opt.read(B.OB_STATE_BITS_WORKER, 2)                     # reading is allowed
+        opt.finish_step()
         assert opt.read(B.OB_STATE_STEP)[1] == 1
         with pytest.raises(B.OnebitError) as e:
-            B.ob_set_server_shard(ctx, 5, 0)        # more shards than workers
-        assert e.value.status == B.OB_ERR_INVALID_ARG
+            B.ob_finish_step(ctx)                              # no split step open
+        assert e.value.status == B.OB_ERR_PHASE
+        B.ob_worker_stage(ctx, [0, 0, 0, 0], 0, 0)             # an empty range is a no-op stage
+        B.ob_finish_step(ctx)
+        assert opt.read(B.OB_STATE_STEP)[1] == 2
     finally:
         opt.close()
