@@ -16,7 +16,10 @@
  *     stage and a server stage) averages the compressed momentum.
  * The calls below follow that two-phase statement:
  *   ob_create -> ob_warmup_adam_step* -> ob_freeze_variance ->
- *   ob_compressed_step* (state machine enforced; OB_ERR_PHASE otherwise).
+ *   ob_compressed_step* (state machine enforced; OB_ERR_PHASE otherwise),
+ * where a compressed step may also be taken as the split step
+ * (ob_worker_stage, an exchange by the caller, ob_finish_step) when the
+ * workers are spread over several processes.
  *
  * Conventions shared by every call
  *   - Every call returns an ob_status and never aborts, throws or exits.

@@ -129,6 +129,11 @@ def test_unknown_or_destroyed_context_is_rejected():
     assert L.ob_freeze_variance(bogus) == B.OB_ERR_INVALID_ARG
     assert L.ob_compressed_step(bogus, None) == B.OB_ERR_INVALID_ARG
     assert L.ob_freeze_variance(None) == B.OB_ERR_INVALID_ARG
+    assert L.ob_worker_stage(bogus, None, 0, 1) == B.OB_ERR_INVALID_ARG
+    assert L.ob_finish_step(bogus) == B.OB_ERR_INVALID_ARG
+    out_p, out_n = ctypes.c_void_p(), ctypes.c_size_t()
+    assert L.ob_worker_exchange_buffers(bogus, ctypes.byref(out_p), ctypes.byref(out_n),
+                                        ctypes.byref(out_p), ctypes.byref(out_n)) == B.OB_ERR_INVALID_ARG
     L.ob_destroy(bogus)  # ignored
     L.ob_destroy(None)
 
