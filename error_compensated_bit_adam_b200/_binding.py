@@ -55,7 +55,8 @@ EXPORTS = (
     "ob_host_staging_bytes", "ob_compressed_step_host", "ob_read_state", "ob_write_state",
     "ob_profile_enable", "ob_profile_read", "ob_kernel_name", "ob_test_fail_host_alloc",
     "ob_onebit_compress_static", "ob_set_lr", "ob_graph_enable",
-    "ob_worker_stage", "ob_worker_exchange_buffers", "ob_finish_step",
+    "ob_server_shard_range", "ob_set_server_shard", "ob_worker_stage", "ob_worker_exchange_buffers",
+    "ob_server_stage", "ob_server_exchange_buffers", "ob_apply_update",
 )
 
 
@@ -116,10 +117,16 @@ def lib() -> ctypes.CDLL:
         "ob_onebit_compress_static": (i32, [vp, i64, vp, vp, vp, vp]),
         "ob_set_lr": (i32, [vp, f32]),
         "ob_graph_enable": (i32, [vp, i32]),
+        "ob_server_shard_range": (i32, [i32, P64, i32, i32, i32, ctypes.POINTER(i32),
+                                        ctypes.POINTER(i32), P64, P64]),
+        "ob_set_server_shard": (i32, [vp, i32, i32]),
         "ob_worker_stage": (i32, [vp, vp, i32, i32]),
         "ob_worker_exchange_buffers": (i32, [vp, ctypes.POINTER(vp), ctypes.POINTER(sz),
                                              ctypes.POINTER(vp), ctypes.POINTER(sz)]),
-        "ob_finish_step": (i32, [vp]),
+        "ob_server_stage": (i32, [vp]),
+        "ob_server_exchange_buffers": (i32, [vp, ctypes.POINTER(vp), ctypes.POINTER(sz),
+                                             ctypes.POINTER(vp), ctypes.POINTER(sz)]),
+        "ob_apply_update": (i32, [vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -269,21 +276,48 @@ def ob_profile_read(ctx: int, reset: bool = False) -> Tuple[List[float], List[in
 
 # ------------------------------------------------------------ split step
 
+def ob_server_shard_range(numel: Sequence[int], W: int, n_shards: int,
+                          shard: int) -> Tuple[int, int, int, int]:
+    """(chunk_begin, chunk_end, word_begin, word_end) of one shard."""
+    cb, ce = ctypes.c_int(), ctypes.c_int()
+    wb, we = ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().ob_server_shard_range(len(numel), _i64_array(numel), int(W), int(n_shards), int(shard),
+                                       ctypes.byref(cb), ctypes.byref(ce), ctypes.byref(wb),
+                                       ctypes.byref(we)), "ob_server_shard_range")
+    return cb.value, ce.value, wb.value, we.value
+
+
+def ob_set_server_shard(ctx: int, n_shards: int, shard: int) -> None:
+    _check(lib().ob_set_server_shard(ctx, int(n_shards), int(shard)), "ob_set_server_shard")
+
+
 def ob_worker_stage(ctx: int, d_grads: Sequence[int], w_begin: int, w_count: int) -> None:
     _check(lib().ob_worker_stage(ctx, _ptrs(d_grads), int(w_begin), int(w_count)), "ob_worker_stage")
 
 
-def ob_worker_exchange_buffers(ctx: int) -> Tuple[int, int, int, int]:
-    """(d_bits, bits_row_bytes, d_scales, scales_row_bytes)."""
+def _buffers(fn, ctx: int, call: str) -> Tuple[int, int, int, int]:
     a, b = ctypes.c_void_p(), ctypes.c_void_p()
     na, nb = ctypes.c_size_t(), ctypes.c_size_t()
-    _check(lib().ob_worker_exchange_buffers(ctx, ctypes.byref(a), ctypes.byref(na), ctypes.byref(b),
-                                            ctypes.byref(nb)), "ob_worker_exchange_buffers")
+    _check(fn(ctx, ctypes.byref(a), ctypes.byref(na), ctypes.byref(b), ctypes.byref(nb)), call)
     return int(a.value or 0), int(na.value), int(b.value or 0), int(nb.value)
 
 
-def ob_finish_step(ctx: int) -> None:
-    _check(lib().ob_finish_step(ctx), "ob_finish_step")
+def ob_worker_exchange_buffers(ctx: int) -> Tuple[int, int, int, int]:
+    """(d_bits, bits_row_bytes, d_scales, scales_row_bytes)."""
+    return _buffers(lib().ob_worker_exchange_buffers, ctx, "ob_worker_exchange_buffers")
+
+
+def ob_server_stage(ctx: int) -> None:
+    _check(lib().ob_server_stage(ctx), "ob_server_stage")
+
+
+def ob_server_exchange_buffers(ctx: int) -> Tuple[int, int, int, int]:
+    """(d_sbits, sbits_bytes, d_scales, scales_bytes)."""
+    return _buffers(lib().ob_server_exchange_buffers, ctx, "ob_server_exchange_buffers")
+
+
+def ob_apply_update(ctx: int) -> None:
+    _check(lib().ob_apply_update(ctx), "ob_apply_update")
 
 
 # ------------------------------------------------------ allocation-free call

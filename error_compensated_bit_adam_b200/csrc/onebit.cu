@@ -300,8 +300,12 @@ struct ob_ctx {
     bool use_graph = false;
     StepGraph graph;
     bool broken = false;
-    // split step (ob_worker_stage ... ob_finish_step): 1 while one is open
+    // split step: 0 idle, 1 after ob_worker_stage, 2 after ob_server_stage
     int split_stage = 0;
+    // the server chunks this context serves in a split step: flat chunk
+    // indices t * W + j in [chunk_lo, chunk_hi), contiguous in layout order
+    // (ob_set_server_shard; all of them by default)
+    int chunk_lo = 0, chunk_hi = -1;
     // profiling
     bool profiling = false;
     std::vector<cudaEvent_t> event_pool;
@@ -716,6 +720,33 @@ void launch_decode_momentum(ob_ctx *c, int tile_lo, int tile_hi, float *out, int
         c->tiles(), tile_lo, c->sbits(), c->sp_last(), c->plan.W, out, base);
 }
 
+// Chunks [*lo, *hi) of shard r of G: contiguous in (tensor, chunk) order,
+// cut where the running tile count reaches r/G of all tiles, so every
+// shard gets about the same server-stage work.
+void shard_chunks(const Plan &pl, int G, int r, int *lo, int *hi) {
+    const int C = pl.T * pl.W;
+    const int64_t nt = (int64_t)pl.tiles.size();
+    auto cut = [&](int q) {
+        if (q <= 0) return 0;
+        if (q >= G) return C;
+        const int64_t target = nt * q / G;
+        return (int)(std::lower_bound(pl.chunk_tile_begin.begin(), pl.chunk_tile_begin.begin() + C + 1,
+                                      target) - pl.chunk_tile_begin.begin());
+    };
+    *lo = cut(r);
+    *hi = cut(r + 1);
+}
+
+// First server word of flat chunk c (n_pad/32 for c == T*W): chunk j of a
+// tensor starts at word min(nw, j*cw) of the tensor.
+int64_t chunk_first_word(const Plan &pl, int c) {
+    if (c >= pl.T * pl.W) return pl.n_pad / 32;
+    const int t = c / pl.W, j = c % pl.W;
+    const int64_t nw = (pl.numel[t] + 31) / 32;
+    const int64_t cw = round_up((nw + pl.W - 1) / pl.W, 4);
+    return pl.offset[t] / 32 + std::min<int64_t>(nw, (int64_t)j * cw);
+}
+
 // Rebuild the dense momentum in its own region (before a consumer that
 // needs it dense: the warmup step).
 ob_status materialize_momentum(ob_ctx *c) {
@@ -1061,33 +1092,117 @@ ob_status ob_worker_exchange_buffers(ob_ctx *c, uint32_t **d_bits, size_t *bits_
     return OB_OK;
 }
 
-ob_status ob_finish_step(ob_ctx *c) {
+ob_status ob_set_server_shard(ob_ctx *c, int n_shards, int shard) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (n_shards < 1 || shard < 0 || shard >= n_shards) return OB_ERR_INVALID_ARG;
+    if (c->split_stage != 0) return OB_ERR_PHASE;
+    shard_chunks(c->plan, n_shards, shard, &c->chunk_lo, &c->chunk_hi);
+    return OB_OK;
+}
+
+ob_status ob_server_shard_range(int n_tensors, const int64_t *numel, int W, int n_shards, int shard,
+                                int *chunk_begin, int *chunk_end, int64_t *word_begin,
+                                int64_t *word_end) {
+    if (!chunk_begin || !chunk_end || !word_begin || !word_end) return OB_ERR_INVALID_ARG;
+    if (n_shards < 1 || shard < 0 || shard >= n_shards) return OB_ERR_INVALID_ARG;
+    try {
+        Plan pl;
+        ob_status st = make_plan(n_tensors, numel, W, true, &pl);
+        if (st != OB_OK) return st;
+        shard_chunks(pl, n_shards, shard, chunk_begin, chunk_end);
+        *word_begin = chunk_first_word(pl, *chunk_begin);
+        *word_end = chunk_first_word(pl, *chunk_end);
+    } catch (const std::bad_alloc &) {
+        return OB_ERR_OOM;
+    }
+    return OB_OK;
+}
+
+ob_status ob_server_stage(ob_ctx *c) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (c->split_stage != 1) return OB_ERR_PHASE;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    const Plan &pl = c->plan;
+    const int C = pl.T * pl.W;
+    const int lo = c->chunk_lo, hi = c->chunk_hi < 0 ? C : c->chunk_hi;
     // the exchange filled the other workers' rows of s_prev; S_WORKER reads
     // the copy in s_last
-    cudaError_t e = cudaMemcpyAsync(c->s_last(), c->s_prev(), (size_t)c->plan.W * c->plan.T * 4,
+    cudaError_t e = cudaMemcpyAsync(c->s_last(), c->s_prev(), (size_t)pl.W * pl.T * 4,
                                     cudaMemcpyDeviceToDevice, c->stream);
     if ((st = fail_cuda(c, e)) != OB_OK) return st;
-    const int nt = c->n_tiles();
-    if (nt > 0) {
+    // The server stage and its scales on the served chunks only: the
+    // kernels index their tiles and chunks from the pointers they are
+    // given, so a contiguous range is launched through offset pointers.
+    const int t_lo = pl.chunk_tile_begin[lo], t_hi = pl.chunk_tile_begin[hi];
+    if (t_hi > t_lo) {
+        onebit::ServerParams P = server_params(c);
+        P.tiles = c->tiles() + t_lo;
+        P.partial = c->partial_s() + t_lo;
+        Geometry G = server_geometry(c);
+        G.grid = grid1(t_hi - t_lo);
         KernelTimer k(c, OB_K_SERVER);
-        const Geometry G = server_geometry(c);
-        onebit::ob_server_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_params(c));
+        onebit::ob_server_kernel<<<G.grid, G.block, G.smem, c->stream>>>(P);
         k.stop();
         if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
     }
-    {
+    if (hi > lo) {
+        onebit::ScaleParams S = server_scale_params(c);
+        S.range_begin = c->chunk_tile_begin() + lo;
+        S.seg_base = c->chunk_seg_base() + lo;
+        S.count = c->chunk_len() + lo;
+        S.counter = c->counters_s() + lo;  // one row
+        S.out_prev = c->sp_prev() + lo;
+        S.out_last = c->sp_last() + lo;
+        S.R = hi - lo;
+        Geometry G = server_scale_geometry(c);
+        G.grid.x = (unsigned)(hi - lo);
         KernelTimer k(c, OB_K_SERVER_SCALE);
-        const Geometry G = server_scale_geometry(c);
-        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_scale_params(c));
+        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(S);
         k.stop();
         if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
     }
-    if (nt > 0) {
+    // The words and scales of the chunks served elsewhere are zero here, so
+    // that summing every process's buffers gives every chunk its server's.
+    const int64_t w_lo = chunk_first_word(pl, lo), w_hi = chunk_first_word(pl, hi);
+    const int64_t words = pl.n_pad / 32;
+    if (e == cudaSuccess && w_lo > 0) e = cudaMemsetAsync(c->sbits(), 0, (size_t)w_lo * 4, c->stream);
+    if (e == cudaSuccess && w_hi < words)
+        e = cudaMemsetAsync(c->sbits() + w_hi, 0, (size_t)(words - w_hi) * 4, c->stream);
+    if (e == cudaSuccess && lo > 0) e = cudaMemsetAsync(c->sp_last(), 0, (size_t)lo * 4, c->stream);
+    if (e == cudaSuccess && hi < C)
+        e = cudaMemsetAsync(c->sp_last() + hi, 0, (size_t)(C - hi) * 4, c->stream);
+    if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    c->split_stage = 2;
+    return OB_OK;
+}
+
+ob_status ob_server_exchange_buffers(ob_ctx *c, uint32_t **d_sbits, size_t *sbits_bytes,
+                                     float **d_scales, size_t *scales_bytes) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (!d_sbits || !sbits_bytes || !d_scales || !scales_bytes) return OB_ERR_INVALID_ARG;
+    *d_sbits = c->sbits();
+    *sbits_bytes = (size_t)(c->plan.n_pad / 32) * 4;
+    *d_scales = c->sp_last();
+    *scales_bytes = (size_t)c->plan.T * c->plan.W * 4;
+    return OB_OK;
+}
+
+ob_status ob_apply_update(ob_ctx *c) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (c->split_stage != 2) return OB_ERR_PHASE;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    // the exchange completed the server scales in sp_last; the next server
+    // stage decodes its y_prev with sp_prev
+    cudaError_t e = cudaMemcpyAsync(c->sp_prev(), c->sp_last(), (size_t)c->plan.T * c->plan.W * 4,
+                                    cudaMemcpyDeviceToDevice, c->stream);
+    if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    if (c->n_tiles() > 0) {
         KernelTimer k(c, OB_K_APPLY);
         const Geometry G = apply_geometry(c);
         onebit::ob_apply_kernel<<<G.grid, G.block, G.smem, c->stream>>>(apply_params(c));

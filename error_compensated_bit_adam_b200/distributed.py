@@ -3,26 +3,27 @@
 The compressed collective of the review page "1-bit Adam: Communication
 Efficient Large-Scale Training with Adam's Convergence Speed" ("Proposed
 method", 4) has a worker stage (every worker compresses its momentum and
-sends its words and scale onward) and a server stage (the compressed
-momenta are averaged, compressed again and returned to every worker).
-Here process r of G computes the worker stage of workers
-[r W/G, (r+1) W/G) with ob_worker_stage, the worker rows (sign words and
-scales) are all-gathered, and every process then runs the server stage of
-every chunk and the update with ob_finish_step.  Given the same rows, every
-process computes the same server words, so nothing is sent back, and every
-process ends the step with the same parameters, bit for bit equal to one
-ob_compressed_step over all W workers.
+sends server j the part of its words that chunk j covers) and a server
+stage (server j averages its chunk, compresses it again and sends the
+result to every worker).  Here process r of G computes workers
+[r W/G, (r+1) W/G) and serves one contiguous range of the server chunks
+(ob_server_shard_range); between the library's three calls
+(ob_worker_stage, ob_server_stage, ob_apply_update) the process exchanges
 
-Against the pages' exchange (each server receives only its chunk of every
-worker's words and returns its chunk to every worker) this sends each
-process every worker's whole row and repeats the server stage on every
-process: one collective over the library's own layout, and no kernel
-beyond the single-GPU step's.
+  * the worker rows (sign words and scales) by an all-gather, and
+  * the server words and scales by a sum-all-reduce: every process holds
+    zeros in the chunks it does not serve, so the sums are exact.
+
+The all-gather sends every worker's whole row to every process, where the
+pages send each server only its chunk: W/G times more bytes, for one
+collective over the library's own layout.  Every process ends the step
+with the same parameters, bit for bit equal to one ob_compressed_step over
+all W workers.
 
 LocalRanks runs the same split step for G ranks inside one process on one
-GPU, each rank a context of its own, with the all-gather done by device
-copies: the single-GPU form of the path, used to check it against one
-context and to time each rank's share of the work.
+GPU, each rank a context of its own, with the exchanges done by device
+copies and sums: the single-GPU form of the path, used to check it against
+one context and to time each rank's share of the work.
 """
 from __future__ import annotations
 
@@ -42,9 +43,9 @@ def _view(workspace: torch.Tensor, ptr: int, nbytes: int, dtype: torch.dtype) ->
 
 
 class TorchExchange:
-    """The split step's exchange over a torch.distributed group (NCCL for
-    CUDA tensors, gloo for CPU tensors).  The collective runs on the current
-    stream; every rank calls it in the same order."""
+    """The split step's two exchanges over a torch.distributed group (NCCL
+    for CUDA tensors, gloo for CPU tensors).  Collectives run on the current
+    stream; every rank calls them in the same order."""
 
     def __init__(self, group=None):
         import torch.distributed as dist
@@ -61,6 +62,9 @@ class TorchExchange:
         mine = rows[begin:begin + count].view(-1)
         self.dist.all_gather_into_tensor(flat, mine, group=self.group)
 
+    def sum_(self, buf: torch.Tensor) -> None:
+        self.dist.all_reduce(buf, op=self.dist.ReduceOp.SUM, group=self.group)
+
 
 class DistributedOneBitAdam:
     """One process's part of a data-parallel 1-bit Adam run.
@@ -69,7 +73,7 @@ class DistributedOneBitAdam:
     process keeps a context over the whole tensor list with all W workers
     (parameters, momentum and variance are the same everywhere).  The phase
     methods below are the split step; ``step`` runs them with ``exchange``
-    (a TorchExchange by default) between the two library calls."""
+    (a TorchExchange by default) between the library calls."""
 
     def __init__(self, numel: Sequence[int], W: int, *, rank: int, world: int, exchange=None,
                  device=None, stream: Optional[torch.cuda.Stream] = None, **hyper):
@@ -82,9 +86,14 @@ class DistributedOneBitAdam:
         self.exchange_impl = exchange
         self.opt = OneBitAdam(numel, W, device=device, stream=stream, **hyper)
         ctx, ws = self.opt.ctx, self.opt.workspace
+        B.ob_set_server_shard(ctx, self.world, self.rank)
+        self.chunk_begin, self.chunk_end, _, _ = B.ob_server_shard_range(numel, W, self.world, self.rank)
         bits, bits_row, scales, scales_row = B.ob_worker_exchange_buffers(ctx)
         self.worker_bits = _view(ws, bits, self.W * bits_row, torch.int32).view(self.W, -1)
         self.worker_scales = _view(ws, scales, self.W * scales_row, torch.float32).view(self.W, -1)
+        sbits, sbits_bytes, sp, sp_bytes = B.ob_server_exchange_buffers(ctx)
+        self.server_bits = _view(ws, sbits, sbits_bytes, torch.int32)
+        self.server_scales = _view(ws, sp, sp_bytes, torch.float32)
 
     @property
     def params(self) -> torch.Tensor:
@@ -118,23 +127,37 @@ class DistributedOneBitAdam:
             ptrs[self.w_begin + i] = g.data_ptr()
         B.ob_worker_stage(self.opt.ctx, ptrs, self.w_begin, self.w_local)
 
-    def finish_step(self) -> None:
-        B.ob_finish_step(self.opt.ctx)
+    def server_stage(self) -> None:
+        B.ob_server_stage(self.opt.ctx)
 
-    def exchange(self, ex) -> None:
-        ex.gather_rows(self.worker_bits, self.w_begin, self.w_local)
-        ex.gather_rows(self.worker_scales, self.w_begin, self.w_local)
+    def apply_update(self) -> None:
+        B.ob_apply_update(self.opt.ctx)
+
+    def serves(self, t: int, j: int) -> bool:
+        """Whether this process serves chunk j of tensor t."""
+        return self.chunk_begin <= t * self.W + j < self.chunk_end
 
     def step(self, local_grads: Sequence[torch.Tensor]) -> None:
         ex = self.exchange_impl if self.exchange_impl is not None else TorchExchange()
         with torch.cuda.stream(self.opt.stream):
             self.worker_stage(local_grads)
-            self.exchange(ex)
-            self.finish_step()
+            ex.gather_rows(self.worker_bits, self.w_begin, self.w_local)
+            ex.gather_rows(self.worker_scales, self.w_begin, self.w_local)
+            self.server_stage()
+            if self.world > 1:
+                ex.sum_(self.server_bits)
+                ex.sum_(self.server_scales)
+            self.apply_update()
 
-    def exchange_bytes(self) -> int:
-        """Bytes the all-gather brings into this process per step."""
-        return (self.W - self.w_local) * (self.worker_bits.shape[1] + self.worker_scales.shape[1]) * 4
+    def exchange_bytes(self) -> dict:
+        """Bytes each exchange moves into this process per step (the sum's
+        figure is its buffer size; the bytes on the wire depend on NCCL's
+        algorithm)."""
+        others = self.W - self.w_local
+        return {"worker_rows_all_gather": others * (self.worker_bits.shape[1]
+                                                    + self.worker_scales.shape[1]) * 4,
+                "server_words_and_scales_sum": (self.server_bits.numel() + self.server_scales.numel()) * 4
+                if self.world > 1 else 0}
 
     def read(self, kind: int, index: int = 0):
         return self.opt.read(kind, index)
@@ -145,9 +168,9 @@ class DistributedOneBitAdam:
 
 class LocalRanks:
     """G ranks of the split step in one process on one GPU, stepped in
-    lockstep; the all-gather is device copies.  No kernel of one rank waits
-    for another's: the ranks' launches are queued one after another on the
-    same stream."""
+    lockstep; the exchanges are device copies and sums.  No kernel of one
+    rank waits for another's: the ranks' launches are queued one after
+    another on the same stream."""
 
     def __init__(self, numel: Sequence[int], W: int, G: int, device=None, **hyper):
         self.G, self.W = int(G), int(W)
@@ -172,6 +195,13 @@ class LocalRanks:
                     rows = slice(src.w_begin, src.w_begin + src.w_local)
                     getattr(dst, attr)[rows].copy_(getattr(src, attr)[rows])
 
+    def _sum(self, attr: str) -> None:
+        total = getattr(self.ranks[0], attr).clone()
+        for r in self.ranks[1:]:
+            total += getattr(r, attr)
+        for r in self.ranks:
+            getattr(r, attr).copy_(total)
+
     def step(self, all_grads: torch.Tensor) -> None:
         """all_grads: [W, n_padded]; rank r gets its workers' rows."""
         for r in self.ranks:
@@ -179,7 +209,12 @@ class LocalRanks:
         self._gather_rows("worker_bits")
         self._gather_rows("worker_scales")
         for r in self.ranks:
-            r.finish_step()
+            r.server_stage()
+        if self.G > 1:
+            self._sum("server_bits")
+            self._sum("server_scales")
+        for r in self.ranks:
+            r.apply_update()
 
     def close(self) -> None:
         for r in self.ranks:

@@ -18,8 +18,8 @@
  *   ob_create -> ob_warmup_adam_step* -> ob_freeze_variance ->
  *   ob_compressed_step* (state machine enforced; OB_ERR_PHASE otherwise),
  * where a compressed step may also be taken as the split step
- * (ob_worker_stage, an exchange by the caller, ob_finish_step) when the
- * workers are spread over several processes.
+ * (ob_worker_stage, ob_server_stage, ob_apply_update, with the caller's
+ * exchanges between them) when the workers are spread over processes.
  *
  * Conventions shared by every call
  *   - Every call returns an ob_status and never aborts, throws or exits.
@@ -203,27 +203,49 @@ OB_API ob_status ob_compressed_step_host(ob_ctx *ctx, const float *const *h_grad
                                   size_t staging_bytes, float *h_server_scales);
 
 /* --------------------------------------------------------------------
- * The split step: one compressed step in two calls, for a data-parallel
+ * The split step: one compressed step in three calls, for a data-parallel
  * run over G processes (one per GPU) in which process r computes the
- * workers [w_begin, w_begin + w_count) -- the worker stage of the
- * compressed collective [1BA, Proposed method, 4] -- and the caller moves
- * their outputs to the other processes in between:
+ * workers [w_begin, w_begin + w_count) and serves one contiguous range of
+ * the server chunks -- the worker stage and the server stage of the
+ * compressed collective [1BA, Proposed method, 4], with the caller moving
+ * each stage's outputs between the processes:
  *
+ *   ob_set_server_shard(ctx, G, r)                        once
  *   per step:
  *     ob_worker_stage(ctx, d_grads, w_begin, w_count)
- *     all-gather of the worker rows of ob_worker_exchange_buffers
- *     ob_finish_step(ctx)       server stage, gather and update
+ *     all-gather of the worker rows (ob_worker_exchange_buffers)
+ *     ob_server_stage(ctx)
+ *     sum-all-reduce of ob_server_exchange_buffers (words as 32-bit
+ *       integers, scales as floats)
+ *     ob_apply_update(ctx)
  *
  * Every process holds a context over the whole tensor list with all W
- * workers' rows and runs the server stage of every chunk itself: with the
- * same inputs every process computes the same server words, so nothing has
- * to be sent back.  p, m and d stay the same on every process, and the
- * result equals ob_compressed_step over all W workers bit for bit.  While
- * a split step is open (between the two calls) only ob_finish_step,
- * ob_worker_exchange_buffers, ob_read_state and ob_destroy are accepted;
- * the other step calls and ob_write_state return OB_ERR_PHASE.  Warmup
- * steps need the gradients of all W workers on every process (the warmup
- * averages them in worker order). */
+ * workers' rows; p, m and d stay the same on every process.  Each server
+ * word and scale is written by one process and is zero on the others, so
+ * the sums are exact and the result equals ob_compressed_step over all W
+ * workers bit for bit.  With G = 1 the server exchange is not needed.
+ * While a split step is open (from ob_worker_stage to ob_apply_update)
+ * only its next call, the exchange-buffer calls, ob_read_state and
+ * ob_destroy are accepted; the other step calls, ob_set_server_shard and
+ * ob_write_state return OB_ERR_PHASE.  Warmup steps need the gradients of
+ * all W workers on every process (the warmup averages them in worker
+ * order).  The server error (E_SERVER) of a process is this step's only on
+ * the chunks it serves. */
+
+/* Chunks [*chunk_begin, *chunk_end) of shard `shard` of n_shards, in flat
+ * index t * W + j (tensor t, server j), and the server words
+ * [*word_begin, *word_end) they cover.  The shards are contiguous in
+ * (tensor, chunk) order, cut so that each holds about the same number of
+ * 4096-element tiles; together they cover every chunk and word once.
+ * Host only. */
+OB_API ob_status ob_server_shard_range(int n_tensors, const int64_t *numel, int W, int n_shards,
+                                       int shard, int *chunk_begin, int *chunk_end,
+                                       int64_t *word_begin, int64_t *word_end);
+
+/* Serve the chunks of shard `shard` of n_shards (ob_server_shard_range) in
+ * the split step.  Default: every chunk.  OB_ERR_PHASE while a split step
+ * is open. */
+OB_API ob_status ob_set_server_shard(ob_ctx *ctx, int n_shards, int shard);
 
 /* Worker stage of workers [w_begin, w_begin + w_count) (w_count may be 0):
  * momentum, error feedback, 1-bit compression and worker scales, as in
@@ -242,11 +264,23 @@ OB_API ob_status ob_worker_stage(ob_ctx *ctx, const float *const *d_grads, int w
 OB_API ob_status ob_worker_exchange_buffers(ob_ctx *ctx, uint32_t **d_bits, size_t *bits_row_bytes,
                                             float **d_scales, size_t *scales_row_bytes);
 
-/* Close the split step once every worker row holds this step's words and
- * scales: server stage, server scales, gather and update, as in
- * ob_compressed_step (the compressed step count advances).  OB_ERR_PHASE
- * unless ob_worker_stage came before. */
-OB_API ob_status ob_finish_step(ob_ctx *ctx);
+/* Server stage of the served chunks, once every worker row holds this
+ * step's words and scales: average, server error, re-compression and
+ * server scales, as in ob_compressed_step; the words and scales of the
+ * other chunks are set to 0.  OB_ERR_PHASE unless ob_worker_stage came
+ * before. */
+OB_API ob_status ob_server_stage(ob_ctx *ctx);
+
+/* Device buffers of the server stage's outputs: *d_sbits uint32[n_padded/32]
+ * server sign words, *d_scales float[n_tensors][W] server scales.  Owned
+ * by the context; valid until ob_destroy. */
+OB_API ob_status ob_server_exchange_buffers(ob_ctx *ctx, uint32_t **d_sbits, size_t *sbits_bytes,
+                                            float **d_scales, size_t *scales_bytes);
+
+/* Gather and update with every chunk's words and scales present; closes
+ * the split step (the compressed step count advances).  OB_ERR_PHASE
+ * unless ob_server_stage came before. */
+OB_API ob_status ob_apply_update(ob_ctx *ctx);
 
 /* Copy one piece of state to host memory.  kind: ob_state_kind.  index:
  * the worker for OB_STATE_E_WORKER / OB_STATE_BITS_WORKER, else 0.  bytes:

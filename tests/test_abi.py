@@ -130,7 +130,9 @@ def test_unknown_or_destroyed_context_is_rejected():
     assert L.ob_compressed_step(bogus, None) == B.OB_ERR_INVALID_ARG
     assert L.ob_freeze_variance(None) == B.OB_ERR_INVALID_ARG
     assert L.ob_worker_stage(bogus, None, 0, 1) == B.OB_ERR_INVALID_ARG
-    assert L.ob_finish_step(bogus) == B.OB_ERR_INVALID_ARG
+    assert L.ob_server_stage(bogus) == B.OB_ERR_INVALID_ARG
+    assert L.ob_apply_update(bogus) == B.OB_ERR_INVALID_ARG
+    assert L.ob_set_server_shard(bogus, 1, 0) == B.OB_ERR_INVALID_ARG
     out_p, out_n = ctypes.c_void_p(), ctypes.c_size_t()
     assert L.ob_worker_exchange_buffers(bogus, ctypes.byref(out_p), ctypes.byref(out_n),
                                         ctypes.byref(out_p), ctypes.byref(out_n)) == B.OB_ERR_INVALID_ARG

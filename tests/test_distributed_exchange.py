@@ -1,7 +1,12 @@
-"""The split step's exchange on the CPU: TorchExchange over world_size-2
-gloo ranks (the in-place all-gather of each rank's block of worker rows,
-32-bit words with bit 31 set included), and the argument checks of
-DistributedOneBitAdam that need no GPU."""
+"""The split step's host logic on the CPU.
+
+* ob_server_shard_range: the shards are contiguous, cover every server
+  chunk and word exactly once, agree with ob_chunk_range's element ranges,
+  and hold about the same number of tiles.
+* TorchExchange over world_size-2 gloo ranks: the in-place all-gather of
+  each rank's block of worker rows and the sum-all-reduce of zero-padded
+  32-bit words (bit 31 set included) and float scales.
+* The argument checks of DistributedOneBitAdam that need no GPU."""
 import os
 import socket
 
@@ -10,6 +15,42 @@ import pytest
 import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
+
+from error_compensated_bit_adam_b200 import _binding as B
+
+TILE = 4096
+
+
+def _tiles_of_chunk(n, W, j):
+    b, e = B.ob_chunk_range(n, W, j)
+    return -(-(e - b) // TILE)
+
+
+@pytest.mark.parametrize("numel,W,G", [([335544320], 8, 8), ([100_003, 31, 0, 4097, 70_000], 8, 4),
+                                       ([50_001, 129, 12_345], 6, 3), ([100, 33, 5000], 16, 4),
+                                       ([0, 0], 4, 3), ([1 << 20] * 5 + [7], 4, 8), ([33], 4, 1)])
+def test_server_shards_partition_chunks_and_words(numel, W, G):
+    offsets, n_pad = B.ob_layout(numel)
+    C = len(numel) * W
+    shards = [B.ob_server_shard_range(numel, W, G, r) for r in range(G)]
+    assert shards[0][0] == 0 and shards[-1][1] == C
+    assert shards[0][2] == 0 and shards[-1][3] == n_pad // 32
+    for a, b in zip(shards, shards[1:]):
+        assert a[1] == b[0] and a[3] == b[2]          # contiguous, no gap or overlap
+    for cb, ce, wb, we in shards:
+        assert cb <= ce and wb <= we
+        # every real word of a served chunk lies in the shard's word range
+        for c in range(cb, ce):
+            t, j = divmod(c, W)
+            b, e = B.ob_chunk_range(numel[t], W, j)
+            if e > b:
+                assert wb <= (offsets[t] + b) // 32 and (offsets[t] + e + 31) // 32 <= we
+    tiles = [sum(_tiles_of_chunk(numel[c // W], W, c % W) for c in range(cb, ce))
+             for cb, ce, _, _ in shards]
+    biggest_chunk = max([_tiles_of_chunk(numel[c // W], W, c % W) for c in range(C)] + [0])
+    assert max(tiles) - min(tiles) <= 2 * biggest_chunk + 1
+    with pytest.raises(B.OnebitError):
+        B.ob_server_shard_range(numel, W, G, G)
 
 
 def _free_port():
@@ -34,7 +75,13 @@ def _rank_main(rank, world, port, out):
         scales = torch.full((W, 3), -1.0, dtype=torch.float32)
         scales[2 * rank:2 * rank + 2] = 0.5 + rank
         ex.gather_rows(scales, 2 * rank, 2)
-        out[rank] = (rows.tolist(), scales.tolist())
+        words = torch.zeros(8, dtype=torch.int32)      # each word written by one rank
+        words[rank::world] = torch.tensor([-7 - rank, 2**30 + rank, -(2**31), 5], dtype=torch.int32)
+        ex.sum_(words)
+        sp = torch.zeros(4, dtype=torch.float32)
+        sp[rank::world] = torch.tensor([0.1 + rank, 3e-7])
+        ex.sum_(sp)
+        out[rank] = (rows.tolist(), scales.tolist(), words.tolist(), sp.tolist())
     finally:
         dist.destroy_process_group()
 
@@ -46,7 +93,10 @@ def test_torch_exchange_on_two_gloo_ranks():
         mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
     assert res[0] == res[1]
-    rows, scales = res[0]
+    rows, scales, words, sp = res[0]
+    assert words == [-7, -8, 2**30, 2**30 + 1, -(2**31), -(2**31), 5, 5]
+    assert sp == [np.float32(0.1).item(), np.float32(1.1).item(),
+                  np.float32(3e-7).item(), np.float32(3e-7).item()]
     for q in range(world):
         blk = (np.arange(10).reshape(2, 5) + 100 * q).tolist()
         blk[0][0] = -(2**31) + q

@@ -1,11 +1,13 @@
-"""The split step (ob_worker_stage, the all-gather of the worker rows,
-ob_finish_step) against one ob_compressed_step context.
+"""The split step (ob_worker_stage / ob_server_stage / ob_apply_update with
+the exchanges between them) against one ob_compressed_step context.
 
 G ranks run in one process on one GPU (distributed.LocalRanks), each with
-its own context, the all-gather done by device copies.  The bar is bit for
-bit: parameters, momentum, the server words, scales and error, and every
-worker's words and scales on every rank, after warmup, freeze and several
-compressed steps with fresh gradients."""
+its own context and its own range of server chunks, the exchanges done by
+device copies and sums.  The bar is bit for bit: parameters, momentum, the
+server words and scales, and every worker's words and scales on every
+rank, the worker errors on their rank and the server error on the rank
+serving each chunk, after warmup, freeze and several compressed steps with
+fresh gradients."""
 import numpy as np
 import pytest
 import torch
@@ -62,8 +64,7 @@ def test_split_step_equals_one_context(name):
     ref, ranks = _run(sizes, W, G)
     try:
         want = {k: ref.read(k) for k in (B.OB_STATE_P, B.OB_STATE_M, B.OB_STATE_BITS_SERVER,
-                                          B.OB_STATE_S_SERVER, B.OB_STATE_E_SERVER,
-                                          B.OB_STATE_S_WORKER, B.OB_STATE_STEP)}
+                                          B.OB_STATE_S_SERVER, B.OB_STATE_S_WORKER, B.OB_STATE_STEP)}
         want_bits = [ref.read(B.OB_STATE_BITS_WORKER, w) for w in range(W)]
         for r in ranks.ranks:
             for k, v in want.items():
@@ -73,6 +74,20 @@ def test_split_step_equals_one_context(name):
             for w in range(r.w_begin, r.w_begin + r.w_local):  # errors live with their worker
                 np.testing.assert_array_equal(r.read(B.OB_STATE_E_WORKER, w),
                                               ref.read(B.OB_STATE_E_WORKER, w))
+        # the server error of a chunk lives on the rank serving it
+        e_ref = ref.read(B.OB_STATE_E_SERVER)
+        offsets, _ = ref.layout()
+        served = 0
+        for rk in ranks.ranks:
+            e = rk.read(B.OB_STATE_E_SERVER)
+            for t, n in enumerate(sizes):
+                for j in range(W):
+                    if rk.serves(t, j):
+                        served += 1
+                        b, end = B.ob_chunk_range(n, W, j)
+                        np.testing.assert_array_equal(e[offsets[t] + b:offsets[t] + end],
+                                                      e_ref[offsets[t] + b:offsets[t] + end])
+        assert served == len(sizes) * W
     finally:
         ref.close()
         ranks.close()
@@ -86,7 +101,8 @@ def test_split_step_phase_rules():
         ptrs = [0, 0, g[2].data_ptr(), g[3].data_ptr()]
         opt.warmup_step(g)
         for call in (lambda: B.ob_worker_stage(ctx, ptrs, 2, 2),  # before the freeze
-                     lambda: B.ob_finish_step(ctx)):
+                     lambda: B.ob_server_stage(ctx),
+                     lambda: B.ob_apply_update(ctx)):
             with pytest.raises(B.OnebitError) as e:
                 call()
             assert e.value.status == B.OB_ERR_PHASE
@@ -100,6 +116,8 @@ def test_split_step_phase_rules():
         assert e.value.status == B.OB_ERR_INVALID_ARG
         opt.worker_stage([g[2], g[3]])
         for call in (lambda: B.ob_worker_stage(ctx, ptrs, 2, 2),
+                     lambda: B.ob_apply_update(ctx),
+                     lambda: B.ob_set_server_shard(ctx, 1, 0),
                      lambda: B.ob_compressed_step(ctx, [g[w].data_ptr() for w in range(4)]),
                      lambda: opt.opt.write(B.OB_STATE_P, 0, np.zeros(4096, np.float32)),
                      lambda: opt.warmup_step(g)):
@@ -107,13 +125,19 @@ def test_split_step_phase_rules():
                 call()
             assert e.value.status == B.OB_ERR_PHASE
         opt.read(B.OB_STATE_BITS_WORKER, 2)                     # reading is allowed
-        opt.finish_step()
+        opt.server_stage()
+        with pytest.raises(B.OnebitError) as e:
+            B.ob_server_stage(ctx)                             # twice
+        assert e.value.status == B.OB_ERR_PHASE
+        opt.apply_update()
         assert opt.read(B.OB_STATE_STEP)[1] == 1
         with pytest.raises(B.OnebitError) as e:
-            B.ob_finish_step(ctx)                              # no split step open
-        assert e.value.status == B.OB_ERR_PHASE
+            B.ob_set_server_shard(ctx, 2, 2)                   # no such shard
+        assert e.value.status == B.OB_ERR_INVALID_ARG
+        B.ob_set_server_shard(ctx, 1, 0)                       # serve everything again
         B.ob_worker_stage(ctx, [0, 0, 0, 0], 0, 0)             # an empty range is a no-op stage
-        B.ob_finish_step(ctx)
+        B.ob_server_stage(ctx)
+        B.ob_apply_update(ctx)
         assert opt.read(B.OB_STATE_STEP)[1] == 2
     finally:
         opt.close()
