@@ -1046,9 +1046,11 @@ ob_status ob_worker_stage(ob_ctx *c, const float *const *d_grads, int w_begin, i
         }
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
-    // The worker stage reads m densely here: its lazy decode indexes the
-    // server scales by the worker count, which the view changes.
-    if ((st = materialize_momentum(c)) != OB_OK) return st;
+    // The worker stage's lazy momentum decode reads the server scale of
+    // (tensor t, chunk j) at t * W + j with W the launch's worker count,
+    // which the view changes; with one tensor that index is j whatever W
+    // is, otherwise the momentum is decoded densely first.
+    if (c->plan.T > 1 && (st = materialize_momentum(c)) != OB_OK) return st;
     const size_t n = (size_t)c->plan.n_pad, T = (size_t)c->plan.T, nt = (size_t)c->n_tiles();
     if (w_count > 0 && nt > 0) {
         onebit::PackParams P = pack_params(c, d_grads, 0, 0);

@@ -250,11 +250,11 @@ OB_API ob_status ob_set_server_shard(ob_ctx *ctx, int n_shards, int shard);
 /* Worker stage of workers [w_begin, w_begin + w_count) (w_count may be 0):
  * momentum, error feedback, 1-bit compression and worker scales, as in
  * ob_compressed_step.  d_grads: host array of W device pointers, only the
- * entries of the range read (the others may be NULL).  The momentum is
- * first decoded into its dense buffer (one extra pass of 4 bytes per
- * parameter).  OB_ERR_PHASE before the freeze or while a split step is
- * open; OB_ERR_INVALID_ARG for a range outside [0, W) or a NULL gradient
- * in it. */
+ * entries of the range read (the others may be NULL).  For a list of more
+ * than one tensor the momentum is first decoded into its dense buffer (one
+ * extra pass of 4 bytes per parameter).  OB_ERR_PHASE before the freeze or
+ * while a split step is open; OB_ERR_INVALID_ARG for a range outside
+ * [0, W) or a NULL gradient in it. */
 OB_API ob_status ob_worker_stage(ob_ctx *ctx, const float *const *d_grads, int w_begin, int w_count);
 
 /* Device buffers of the worker stage's outputs, one row per worker, rows
