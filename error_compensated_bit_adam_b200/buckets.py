@@ -17,7 +17,6 @@ from typing import List, Optional, Sequence
 
 import torch
 
-from . import _binding as B
 from .optimizer import Grads, OneBitAdam
 
 

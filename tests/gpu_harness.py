@@ -5,8 +5,7 @@ path, except in re-synced runs, where the state *entering* a step is copied
 from the oracle INTO the GPU (never the other way)."""
 from __future__ import annotations
 
-import math
-from typing import List, Optional
+from typing import Optional
 
 import numpy as np
 import torch
