@@ -556,7 +556,9 @@ def run_b200(args) -> None:
         if cnt:
             gbs = algo[name] / (kms / cnt / 1e3) / 1e9
             pre_path[name] = {"launches": cnt, "avg_launch_ms": kms / cnt, "gbs": gbs,
-                              "frac_of_measured_hbm": gbs / peak["hbm_gbs"]}
+                              "frac_of_measured_hbm": gbs / peak["hbm_gbs"],
+                              "algorithmic_bytes_per_launch": algo[name],
+                              "traffic": measured_traffic(name, wl.n, wl.W)}
 
     # end to end: host gradients in pinned memory, copied in every step, and
     # the step's server scales read back, through ob_compressed_step_host
