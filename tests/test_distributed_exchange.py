@@ -110,3 +110,34 @@ def test_worker_split_must_divide_W():
         DistributedOneBitAdam([10], 6, rank=0, world=4)
     with pytest.raises(ValueError):
         DistributedOneBitAdam([10], 4, rank=2, world=2)
+
+
+def _rank_leaves(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    from error_compensated_bit_adam_b200.distributed import TorchExchange
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    ex = TorchExchange()
+    rows = torch.zeros((2 * world, 4), dtype=torch.int32)
+    ex.gather_rows(rows, 2 * rank, 2)                  # one step's exchange together
+    dist.barrier()
+    if rank == 1:
+        out[rank] = "left"                              # leaves between steps, nothing in flight
+        os._exit(0)
+    try:
+        ex.gather_rows(rows, 2 * rank, 2)              # the next step's exchange
+        out[rank] = "no error"
+    except Exception as e:  # the group's timeout or the closed connection
+        out[rank] = f"error: {type(e).__name__}"
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_is_detected_at_the_next_exchange():
+    world = 2
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_rank_leaves, args=(world, _free_port(), out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[1] == "left"
+    assert res[0].startswith("error"), res[0]
