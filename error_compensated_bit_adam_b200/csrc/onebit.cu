@@ -18,6 +18,7 @@
 #include <vector>
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>  // header-only; a no-op unless a profiler is attached
 
 #include "../../include/onebit.h"
 #include "onebit_kernels.cuh"
@@ -367,11 +368,24 @@ cudaEvent_t take_event(ob_ctx *c) {
     return e;
 }
 
+// An NVTX range over one library call (shown by Nsight tools beside the
+// CUDA launches it makes).
+struct NvtxCall {
+    explicit NvtxCall(const char *name) { nvtxRangePushA(name); }
+    ~NvtxCall() { nvtxRangePop(); }
+    NvtxCall(const NvtxCall &) = delete;
+    NvtxCall &operator=(const NvtxCall &) = delete;
+};
+
+// Around each kernel launch: an NVTX range named after the kernel and,
+// while profiling is on, a pair of CUDA events on the context's stream.
 struct KernelTimer {
     ob_ctx *c;
     int id;
     cudaEvent_t a = nullptr, b = nullptr;
+    nvtxRangeId_t range = 0;
     KernelTimer(ob_ctx *ctx, int k) : c(ctx), id(k) {
+        range = nvtxRangeStartA(kKernelNames[k]);
         if (!c->profiling) return;
         a = take_event(c);
         b = take_event(c);
@@ -384,6 +398,8 @@ struct KernelTimer {
         }
     }
     void stop() {
+        if (range) nvtxRangeEnd(range);
+        range = 0;
         if (!c->profiling || !a || !b) return;
         cudaEventRecord(b, c->stream);
         c->pending.push_back({id, {a, b}});
@@ -950,6 +966,7 @@ void ob_destroy(ob_ctx *c) {
 }
 
 ob_status ob_warmup_adam_step(ob_ctx *c, const float *const *d_grads) {
+    NvtxCall nvtx("ob_warmup_adam_step");
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
@@ -984,6 +1001,7 @@ ob_status ob_warmup_adam_step(ob_ctx *c, const float *const *d_grads) {
 }
 
 ob_status ob_freeze_variance(ob_ctx *c) {
+    NvtxCall nvtx("ob_freeze_variance");
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (c->frozen || c->t_warmup < 1 || c->split_stage != 0) return OB_ERR_PHASE;
@@ -1008,6 +1026,7 @@ ob_status ob_freeze_variance(ob_ctx *c) {
 }
 
 ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
+    NvtxCall nvtx("ob_compressed_step");
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (!c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
@@ -1034,6 +1053,7 @@ ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
 // worker rows [w_begin, w_begin + w_count) as if those were all workers.
 
 ob_status ob_worker_stage(ob_ctx *c, const float *const *d_grads, int w_begin, int w_count) {
+    NvtxCall nvtx("ob_worker_stage");
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (!c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
@@ -1122,6 +1142,7 @@ ob_status ob_server_shard_range(int n_tensors, const int64_t *numel, int W, int 
 }
 
 ob_status ob_server_stage(ob_ctx *c) {
+    NvtxCall nvtx("ob_server_stage");
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (c->split_stage != 1) return OB_ERR_PHASE;
@@ -1194,6 +1215,7 @@ ob_status ob_server_exchange_buffers(ob_ctx *c, uint32_t **d_sbits, size_t *sbit
 }
 
 ob_status ob_apply_update(ob_ctx *c) {
+    NvtxCall nvtx("ob_apply_update");
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (c->split_stage != 2) return OB_ERR_PHASE;
@@ -1242,6 +1264,7 @@ ob_status ob_host_staging_bytes(const ob_ctx *c, size_t *bytes) {
 
 ob_status ob_compressed_step_host(ob_ctx *c, const float *const *h_grads, void *d_staging,
                                   size_t staging_bytes, float *h_server_scales) {
+    NvtxCall nvtx("ob_compressed_step_host");
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
     if (!c->frozen || c->split_stage != 0) return OB_ERR_PHASE;
