@@ -3,6 +3,9 @@
 * ob_server_shard_range: the shards are contiguous, cover every server
   chunk and word exactly once, agree with ob_chunk_range's element ranges,
   and hold about the same number of tiles.
+* The sums are exact: each shard's server words and scales (the oracle's
+  per-chunk server stage on the shard's chunks, zeros elsewhere) summed
+  over the shards equal the one-server result, bit for bit.
 * TorchExchange over world_size-2 gloo ranks: the in-place all-gather of
   each rank's block of worker rows and the sum-all-reduce of zero-padded
   32-bit words (bit 31 set included) and float scales.
@@ -51,6 +54,50 @@ def test_server_shards_partition_chunks_and_words(numel, W, G):
     assert max(tiles) - min(tiles) <= 2 * biggest_chunk + 1
     with pytest.raises(B.OnebitError):
         B.ob_server_shard_range(numel, W, G, G)
+
+
+def _shard_sums(numel, W, G, seed):
+    """One tensor list's server stage computed whole and per shard (the
+    oracle's per-chunk server stage on the shard's chunks, zeros in the
+    words and scales of the others), summed over the shards."""
+    import oracle
+    o = oracle.default()
+    rng = np.random.default_rng(seed)
+    shards = [B.ob_server_shard_range(numel, W, G, r) for r in range(G)]
+    for t, n in enumerate(numel):
+        bits = [rng.integers(0, 2**32, o.num_words(n), dtype=np.uint64).astype(np.uint32)
+                for _ in range(W)]
+        if n % 32:
+            for b in bits:  # padding bits are 0
+                b[-1] &= np.uint32((1 << (n % 32)) - 1)
+        s = rng.uniform(0.5, 2.0, W).astype(np.float32)
+        e0 = rng.normal(0, 0.1, n).astype(np.float32)
+        e_one = e0.copy()
+        words_one, s_one = o.server_compress(bits, s, e_one)
+        words_sum = np.zeros(o.num_words(n), np.int64)
+        s_sum = np.zeros(W, np.float32)
+        for cb, ce, _, _ in shards:
+            e_r = e0.copy()
+            words_r = np.zeros(o.num_words(n), np.uint32)
+            s_r = np.zeros(W, np.float32)
+            for j in range(W):
+                if cb <= t * W + j < ce:
+                    s_r[j] = o.server_compress_chunk(j, bits, s, e_r, words_r)
+                    b, e = o.chunk_range(n, W, j)
+                    np.testing.assert_array_equal(e_r[b:e], e_one[b:e])  # server error on its shard
+            words_sum += words_r.view(np.int32).astype(np.int64)
+            s_sum = s_sum + s_r
+        yield words_one, s_one, words_sum, s_sum
+
+
+@pytest.mark.parametrize("numel,W,G", [([1 << 16], 8, 8), ([100_003, 31, 0, 4097, 70_000], 8, 4),
+                                       ([50_001, 129, 12_345], 6, 3), ([100, 33, 5000], 16, 4),
+                                       ([33], 4, 2)])
+def test_shard_sums_equal_one_server(numel, W, G):
+    for words_one, s_one, words_sum, s_sum in _shard_sums(numel, W, G, seed=W * G + len(numel)):
+        # 32-bit integer sums with one non-zero term per word: no carries
+        assert np.array_equal(words_sum.astype(np.int32).view(np.uint32), words_one)
+        assert np.array_equal(s_sum, s_one)
 
 
 def _free_port():
