@@ -84,6 +84,7 @@ class DistributedOneBitAdam:
         self.w_local = self.W // self.world
         self.w_begin = self.rank * self.w_local
         self.exchange_impl = exchange
+        self._zeros: Optional[torch.Tensor] = None
         self.opt = OneBitAdam(numel, W, device=device, stream=stream, **hyper)
         ctx, ws = self.opt.ctx, self.opt.workspace
         B.ob_set_server_shard(ctx, self.world, self.rank)
@@ -108,6 +109,29 @@ class DistributedOneBitAdam:
         [W, n_padded] (the warmup adds them in worker order, so every
         process needs all of them)."""
         self.opt.warmup_step(all_grads)
+
+    def warmup_step_allreduce(self, local_grads: Sequence[torch.Tensor]) -> None:
+        """Full-precision Adam on the average of all W workers' gradients
+        with the sum taken by an all-reduce, as in ordinary data-parallel
+        training: local_grads[i] (worker w_begin + i) is overwritten by the
+        sum over processes of every process's i-th gradient, and the warmup
+        kernel averages those W/G sums and W - W/G zero vectors (adding
+        zeros is exact).  Equal to warmup_step up to the order of the
+        additions inside the all-reduce."""
+        if len(local_grads) != self.w_local:
+            raise ValueError(f"expected {self.w_local} local gradients")
+        ex = self.exchange_impl if self.exchange_impl is not None else TorchExchange()
+        with torch.cuda.stream(self.opt.stream):
+            for g in local_grads:
+                ex.sum_(g)
+            self.warmup_from_sums(local_grads)
+
+    def warmup_from_sums(self, sums: Sequence[torch.Tensor]) -> None:
+        """The warmup step given the all-reduced sums of warmup_step_allreduce."""
+        if self._zeros is None:
+            self._zeros = torch.zeros(self.opt.n_padded, dtype=torch.float32, device=self.opt.device)
+        rows = list(sums) + [self._zeros] * (self.W - len(sums))
+        self.opt.warmup_step(rows)
 
     def freeze(self) -> None:
         self.opt.freeze()
@@ -183,6 +207,18 @@ class LocalRanks:
     def warmup_step(self, all_grads: torch.Tensor) -> None:
         for r in self.ranks:
             r.warmup_step(all_grads)
+
+    def warmup_step_allreduce(self, all_grads: torch.Tensor) -> None:
+        """warmup_step_allreduce of every rank, the all-reduce emulated by
+        sums in rank order (all_grads is left unchanged)."""
+        sums = []
+        for i in range(self.w_local):
+            t = all_grads[i].clone()
+            for r in self.ranks[1:]:
+                t += all_grads[r.w_begin + i]
+            sums.append(t)
+        for r in self.ranks:
+            r.warmup_from_sums(sums)
 
     def freeze(self) -> None:
         for r in self.ranks:

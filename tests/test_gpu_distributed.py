@@ -93,6 +93,49 @@ def test_split_step_equals_one_context(name):
         ranks.close()
 
 
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_allreduce_warmup_matches_the_ordered_warmup(G):
+    """The warmup on all-reduced sums: bit for bit with one rank (the sums
+    are the gradients themselves), within rounding of the sum's order
+    otherwise; the compressed steps after it still track one context."""
+    sizes, W = (100_003, 4097, 33), 4
+    wl = WL.Workload("allreduce-warmup", tuple((n,) for n in sizes), W, 3, 4, seed=41)
+    offsets, n_pad = B.ob_layout(wl.numels)
+    params = WL.make_params(wl, offsets, n_pad, device="cuda")
+    scale = WL.grad_scale_vector(wl, offsets, n_pad, device="cuda")
+    ref = OneBitAdam(wl.numels, W, params=params.clone(), **WL.HYPER)
+    ranks = LocalRanks(wl.numels, W, G, **WL.HYPER)
+    try:
+        for r in ranks.ranks:
+            r.params.copy_(params)
+        g = torch.empty((W, n_pad), device="cuda")
+        for step in range(3):
+            WL.fill_grads(wl, step, scale, g)
+            ref.warmup_step(g)
+            ranks.warmup_step_allreduce(g)
+        ref.freeze()
+        ranks.freeze()
+        p_ref = ref.read(B.OB_STATE_P).astype(np.float64)
+        for r in ranks.ranks:
+            p = r.read(B.OB_STATE_P).astype(np.float64)
+            if G == 1:
+                np.testing.assert_array_equal(p, p_ref)
+                np.testing.assert_array_equal(r.read(B.OB_STATE_D), ref.read(B.OB_STATE_D))
+            else:
+                assert np.linalg.norm(p - p_ref) <= 1e-6 * np.linalg.norm(p_ref)
+        for step in range(3, 7):
+            WL.fill_grads(wl, step, scale, g)
+            ref.step(g)
+            ranks.step(g)
+        p_ref = ref.read(B.OB_STATE_P).astype(np.float64)
+        for r in ranks.ranks:
+            p = r.read(B.OB_STATE_P).astype(np.float64)
+            assert np.linalg.norm(p - p_ref) <= 1e-5 * np.linalg.norm(p_ref)
+    finally:
+        ref.close()
+        ranks.close()
+
+
 def test_split_step_phase_rules():
     opt = DistributedOneBitAdam([4096], 4, rank=1, world=2, **WL.HYPER)
     try:
