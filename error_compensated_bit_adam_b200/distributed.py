@@ -120,7 +120,7 @@ class DistributedOneBitAdam:
         additions inside the all-reduce."""
         if len(local_grads) != self.w_local:
             raise ValueError(f"expected {self.w_local} local gradients")
-        ex = self.exchange_impl if self.exchange_impl is not None else TorchExchange()
+        ex = self._exchange()
         with torch.cuda.stream(self.opt.stream):
             for g in local_grads:
                 ex.sum_(g)
@@ -161,8 +161,13 @@ class DistributedOneBitAdam:
         """Whether this process serves chunk j of tensor t."""
         return self.chunk_begin <= t * self.W + j < self.chunk_end
 
+    def _exchange(self):
+        if self.exchange_impl is None:  # the default process group, made on first use
+            self.exchange_impl = TorchExchange()
+        return self.exchange_impl
+
     def step(self, local_grads: Sequence[torch.Tensor]) -> None:
-        ex = self.exchange_impl if self.exchange_impl is not None else TorchExchange()
+        ex = self._exchange()
         with torch.cuda.stream(self.opt.stream):
             self.worker_stage(local_grads)
             ex.gather_rows(self.worker_bits, self.w_begin, self.w_local)
