@@ -63,6 +63,16 @@ MUTANTS = [
      "sbits[i >> 5] |= (uint32_t)1u << (31 - (i & 31));"),
     ("server_empty_chunk_clears_a_word", "    if (e > b)  /* an empty chunk owns no word, not even the tensor's last */\n",
      "    if (1)\n"),
+    ("freeze_eps_inside_sqrt",
+     "const float root = sqrtf(vhat);\n        d[i] = root + eps;",
+     "const float root = sqrtf(vhat + eps);\n        d[i] = root;"),
+    ("scale_uses_n_minus_1", "return (float)sqrt(sum_sq / (double)count);",
+     "return (float)sqrt(sum_sq / (double)(count > 1 ? count - 1 : 1));"),
+    ("worker_momentum_constants_swapped",
+     "const float m_old = beta1 * m[i];\n        const float m_new = c1 * g[i];",
+     "const float m_old = c1 * m[i];\n        const float m_new = beta1 * g[i];"),
+    ("warmup_variance_uses_beta1", "const float v_old = beta2 * v[i];", "const float v_old = beta1 * v[i];"),
+    ("chunk_words_rounded_down", "const int64_t per = (nw + W - 1) / W;", "const int64_t per = nw / W;"),
 ]
 
 MUTANT_CFLAGS = [f for f in oracle.CFLAGS if f != "-Werror"]
