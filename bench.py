@@ -267,29 +267,40 @@ def measure_e2e(opt, wl, n_pad, dev_grads, args, world, dev) -> dict:
     """The step through the public host-buffer call: every step copies W
     gradient vectors from pinned host memory to the GPU (overlapped with the
     worker stage) and reads the step's server scales back."""
+    # Every rank takes the same collective steps whatever happens locally
+    # (a failure is carried as a flag), so no rank waits on another.
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    err, pinned, host, out, elapsed = None, False, None, None, 0.0
     try:
-        e2e_steps = max(1, min(args.steps, args.e2e_steps))
         try:
             host = torch.empty((wl.W, n_pad), dtype=torch.float32, pin_memory=True)
             pinned = True
         except RuntimeError:
             host = torch.empty((wl.W, n_pad), dtype=torch.float32)
-            pinned = False
         host.copy_(dev_grads)
         out = np.zeros(wl.n_tensors * wl.W, np.float32)
         opt.step_host(host, out)                    # untimed: staging allocation
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        w0 = time.perf_counter()
-        for _ in range(e2e_steps):
-            opt.step_host(host, out)
-        e2e_s = max_over_ranks(time.perf_counter() - w0, world) / e2e_steps
-        return {"value": world * wl.n / e2e_s, "unit": UNIT,
-                "h2d_bytes_per_step": int(host.numel() * 4), "d2h_bytes_per_step": int(out.nbytes),
-                "ms_per_step": e2e_s * 1e3, "pinned": pinned, "steps": e2e_steps,
-                "call": "ob_compressed_step_host"}
+        if torch.cuda.is_available():
+            torch.cuda.synchronize(dev)
     except Exception as exc:  # reported, never hidden
-        return {"value": None, "unit": UNIT, "error": repr(exc)}
+        err = repr(exc)
+    barrier(world)
+    if err is None:
+        try:
+            w0 = time.perf_counter()
+            for _ in range(e2e_steps):
+                opt.step_host(host, out)
+            elapsed = time.perf_counter() - w0
+        except Exception as exc:
+            err = repr(exc)
+    e2e_s = max_over_ranks(elapsed, world) / e2e_steps
+    failed = max_over_ranks(0.0 if err is None else 1.0, world)
+    if failed:
+        return {"value": None, "unit": UNIT, "error": err or "failed on another rank"}
+    return {"value": world * wl.n / e2e_s, "unit": UNIT,
+            "h2d_bytes_per_step": int(host.numel() * 4), "d2h_bytes_per_step": int(out.nbytes),
+            "ms_per_step": e2e_s * 1e3, "pinned": pinned, "steps": e2e_steps,
+            "call": "ob_compressed_step_host"}
 
 
 def measure_split_ranks(wl, args, dev) -> dict:
