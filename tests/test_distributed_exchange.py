@@ -9,7 +9,11 @@
 * TorchExchange over world_size-2 gloo ranks: the in-place all-gather of
   each rank's block of worker rows and the sum-all-reduce of zero-padded
   32-bit words (bit 31 set included) and float scales.
-* The argument checks of DistributedOneBitAdam that need no GPU."""
+* The argument checks of DistributedOneBitAdam that need no GPU.
+* The split step's whole protocol on two gloo ranks, the oracle doing each
+  rank's arithmetic and TorchExchange and the shard ranges the exchange:
+  bit for bit the single-process oracle run.
+* A rank that leaves between steps is noticed at the next exchange."""
 import os
 import socket
 
@@ -188,3 +192,97 @@ def test_a_rank_that_leaves_is_detected_at_the_next_exchange():
         res = dict(out)
     assert res[1] == "left"
     assert res[0].startswith("error"), res[0]
+
+
+def _grads(numel, W, step):
+    rng = np.random.default_rng(1000 + step)
+    return [[rng.normal(0, 1e-3, n).astype(np.float32) for n in numel] for _ in range(W)]
+
+
+def _protocol_rank(rank, world, port, out, numel, W, steps):
+    """One process of the split step with the oracle doing its arithmetic:
+    worker stage of its workers, all-gather of the worker rows, server stage
+    of its shard, sum of the server words and scales, update of everything."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import oracle
+    from error_compensated_bit_adam_b200.distributed import TorchExchange
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        ex = TorchExchange()
+        hp = dict(beta1=0.9, beta2=0.999, eps=1e-8, lr=1e-4)
+        params = [np.random.default_rng(7 + t).normal(0, 0.02, n).astype(np.float32)
+                  for t, n in enumerate(numel)]
+        run = oracle.OracleRun(params, W, hp)          # this process's state
+        o, T, wl = run.o, len(numel), W // world
+        mine = range(rank * wl, (rank + 1) * wl)
+        cb, ce, _, _ = B.ob_server_shard_range(numel, W, world, rank)
+        for step in range(2):
+            run.warmup_step(_grads(numel, W, step))    # every process, every worker
+        run.freeze()
+        for step in range(2, 2 + steps):
+            g = _grads(numel, W, step)
+            words = [torch.zeros((W, o.num_words(n)), dtype=torch.int32) for n in numel]
+            scales = torch.zeros((W, T), dtype=torch.float32)
+            for w in mine:
+                for t in range(T):
+                    b, s = run.worker_stage(w, t, g[w][t])
+                    words[t][w] = torch.from_numpy(b.view(np.int32))
+                    scales[w, t] = float(s)
+            for t in range(T):
+                ex.gather_rows(words[t], rank * wl, wl)
+            ex.gather_rows(scales, rank * wl, wl)
+            sbits = [np.zeros(o.num_words(n), np.uint32) for n in numel]
+            s_srv = np.zeros((T, W), np.float32)
+            for t in range(T):
+                rows = [words[t][w].numpy().view(np.uint32).copy() for w in range(W)]
+                for j in range(W):
+                    if cb <= t * W + j < ce:
+                        s_srv[t, j] = o.server_compress_chunk(j, rows, scales[:, t].numpy(),
+                                                              run.e_s[t], sbits[t])
+            sw = [torch.from_numpy(sb.view(np.int32)) for sb in sbits]
+            for t in range(T):
+                ex.sum_(sw[t])
+            st_ = torch.from_numpy(s_srv)
+            ex.sum_(st_)
+            for t in range(T):
+                full = sw[t].numpy().view(np.uint32)
+                for j in range(W):
+                    o.apply_chunk(j, W, hp["lr"], full, st_[t, j].item(), run.d[t], run.p[t], run.m[t])
+        served = {(t, j) for t in range(T) for j in range(W) if cb <= t * W + j < ce}
+        out[rank] = ([p.tobytes() for p in run.p], [m.tobytes() for m in run.m],
+                     {w: [e.tobytes() for e in run.e_w[w]] for w in mine},
+                     {(t, j): run.e_s[t][slice(*o.chunk_range(numel[t], W, j))].tobytes()
+                      for (t, j) in served})
+    finally:
+        dist.destroy_process_group()
+
+
+def test_split_protocol_on_gloo_ranks_equals_one_process():
+    import oracle
+    numel, W, world, steps = [5_001, 64, 0, 777], 4, 2, 3
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_protocol_rank, args=(world, _free_port(), out, numel, W, steps), nprocs=world,
+                 join=True)
+        res = dict(out)
+    hp = dict(beta1=0.9, beta2=0.999, eps=1e-8, lr=1e-4)
+    params = [np.random.default_rng(7 + t).normal(0, 0.02, n).astype(np.float32)
+              for t, n in enumerate(numel)]
+    ref = oracle.OracleRun(params, W, hp)
+    for step in range(2):
+        ref.warmup_step(_grads(numel, W, step))
+    ref.freeze()
+    for step in range(2, 2 + steps):
+        ref.compressed_step(_grads(numel, W, step))
+    o = ref.o
+    for r in range(world):
+        p, m, e_w, e_s = res[r]
+        assert p == [a.tobytes() for a in ref.p] and m == [a.tobytes() for a in ref.m]
+        for w, rows in e_w.items():
+            assert rows == [e.tobytes() for e in ref.e_w[w]]
+        for (t, j), blob in e_s.items():
+            assert blob == ref.e_s[t][slice(*o.chunk_range(numel[t], W, j))].tobytes()
+    served = set().union(*(set(res[r][3]) for r in range(world)))
+    assert served == {(t, j) for t in range(len(numel)) for j in range(W)}
