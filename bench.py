@@ -556,6 +556,8 @@ def run_b200(args) -> None:
                      "share": kms / max(1e-12, sum(v[0] for v in prof.values()))}
             if name in algo:
                 entry["gbs"] = algo[name] / (kms / args.steps / 1e3) / 1e9
+                entry["algorithmic_bytes_per_launch"] = algo[name]
+                entry["traffic"] = measured_traffic(name, wl.n, wl.W)
             per_kernel[name] = entry
 
     # the pre-path (full-precision Adam warmup and the freeze), timed by the
