@@ -228,28 +228,26 @@ ORC_API int orc_server_compress_chunk(int64_t n, int W, int j, const uint32_t *c
     const float wf = (float)W;
     int64_t b, e;
     orc_chunk_range(n, W, j, &b, &e);
-    float *y = y_out;
-    if (!y) {
-        y = (float *)calloc((size_t)(e > b ? e : 1), sizeof(float));
-        if (!y) return -1;
-        y -= b;  /* index y by element, like y_out */
-    }
+    /* y of element i is y[i - b]: the chunk's own values, either in y_out
+     * (whose element i is y_out[i]) or in a buffer of the chunk's length */
+    float *y = y_out ? y_out + b : (float *)calloc((size_t)(e > b ? e - b : 1), sizeof(float));
+    if (!y) return -1;
     double sum_sq = 0.0;
     for (int64_t i = b; i < e; ++i) {
         float acc = 0.0f;
         for (int w = 0; w < W; ++w) acc = acc + signed_scale(get_bit(bits[w], i), s[w]);
         const float avg = acc / wf;
-        y[i] = avg + e_s[i];
-        sum_sq += (double)y[i] * (double)y[i];
+        y[i - b] = avg + e_s[i];
+        sum_sq += (double)y[i - b] * (double)y[i - b];
     }
     const float sj = rms_scale(sum_sq, e - b);
     if (e > b)  /* an empty chunk owns no word, not even the tensor's last */
         for (int64_t k = b / 32; k < (e + 31) / 32; ++k) sbits[k] = 0u;
     for (int64_t i = b; i < e; ++i)
-        if (sign_bit(y[i])) sbits[i >> 5] |= (uint32_t)1u << (i & 31);
-    for (int64_t i = b; i < e; ++i) e_s[i] = y[i] - signed_scale(sign_bit(y[i]), sj);
+        if (sign_bit(y[i - b])) sbits[i >> 5] |= (uint32_t)1u << (i & 31);
+    for (int64_t i = b; i < e; ++i) e_s[i] = y[i - b] - signed_scale(sign_bit(y[i - b]), sj);
     *s_srv_j = sj;
-    if (y != y_out) free(y + b);
+    if (!y_out) free(y);
     return 0;
 }
 

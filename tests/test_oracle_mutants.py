@@ -40,15 +40,15 @@ MUTANTS = [
      "const float m_old = beta1 * m[i];\n        const float m_new = c1 * 0.0f * g[i];"),
     ("worker_forgets_error", "x[i] = m_w + e[i];", "x[i] = m_w;"),
     ("server_does_not_average", "const float avg = acc / wf;", "const float avg = acc;"),
-    ("server_forgets_error", "y[i] = avg + e_s[i];", "y[i] = avg;"),
+    ("server_forgets_error", "y[i - b] = avg + e_s[i];", "y[i - b] = avg;"),
     ("server_uses_worker0_scale", "signed_scale(get_bit(bits[w], i), s[w])",
      "signed_scale(get_bit(bits[w], i), s[0])"),
     ("server_reads_neighbour_bit", "signed_scale(get_bit(bits[w], i), s[w])",
      "signed_scale(get_bit(bits[w], i ^ 1), s[w])"),
     ("server_error_uses_worker0_scale",
-     "e_s[i] = y[i] - signed_scale(sign_bit(y[i]), sj);",
-     "e_s[i] = y[i] - signed_scale(sign_bit(y[i]), s[0]);"),
-    ("server_error_wrong_sign", "e_s[i] = y[i] - signed_scale(", "e_s[i] = y[i] + signed_scale("),
+     "e_s[i] = y[i - b] - signed_scale(sign_bit(y[i - b]), sj);",
+     "e_s[i] = y[i - b] - signed_scale(sign_bit(y[i - b]), s[0]);"),
+    ("server_error_wrong_sign", "e_s[i] = y[i - b] - signed_scale(", "e_s[i] = y[i - b] + signed_scale("),
     ("chunks_not_word_group_aligned", "const int64_t cw = ((per + 3) / 4) * 4;",
      "const int64_t cw = per;"),
     ("apply_wrong_sign", "p[i] = p[i] - delta;\n        m[i] = m_hat;",
