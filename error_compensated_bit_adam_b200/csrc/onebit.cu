@@ -1451,16 +1451,15 @@ ob_status ob_profile_read(ob_ctx *c, double *ms, int64_t *launches, int reset) {
 // 128 KiB).  It lives in the library's module, so every GPU that loads the
 // library holds it until the process exits.  Host code may not pass the
 // array's name to a kernel (on the host it is only a stand-in); its device
-// address is looked up once per device with cudaGetSymbolAddress.
+// address is looked up with cudaGetSymbolAddress, with the device current,
+// on every call: the lookup allocates nothing, and an address kept from an
+// earlier call would be stale after the caller reset the device (the
+// module is then loaded again, possibly elsewhere).
 
 namespace {
 
 constexpr int kStaticTiles = (int)(OB_STATIC_MAX_ELEMENTS / kTile);
 static_assert((int64_t)kStaticTiles * kTile == OB_STATIC_MAX_ELEMENTS, "static scratch size");
-constexpr int kStaticDevices = 64;
-
-std::mutex g_static_mu;
-double *g_static_addr[kStaticDevices] = {};
 
 }  // namespace
 
@@ -1473,25 +1472,32 @@ extern "C" ob_status ob_onebit_compress_static(const float *d_x, int64_t n, uint
     if (n > 0 && (!d_x || !d_bits || !d_error)) return OB_ERR_INVALID_ARG;
     if (!aligned(d_x, 16) || !aligned(d_error, 16) || !aligned(d_bits, 4) || !aligned(d_scale, 4))
         return OB_ERR_ALIGN;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kStaticDevices) return OB_ERR_CUDA;
-    double *scratch = nullptr;
-    {
-        std::lock_guard<std::mutex> lk(g_static_mu);
-        if (!g_static_addr[dev]) {
-            void *addr = nullptr;
-            if (cudaGetSymbolAddress(&addr, g_static_partial) != cudaSuccess || !addr)
-                return OB_ERR_CUDA;
-            g_static_addr[dev] = static_cast<double *>(addr);
-        }
-        scratch = g_static_addr[dev];
-    }
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_static_partial) != cudaSuccess || !addr) return OB_ERR_CUDA;
+    double *scratch = static_cast<double *>(addr);
     cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
     const int tiles = (int)((n + kTile - 1) / kTile);
-    if (tiles > 0)
-        onebit::ob_compress_partial_kernel<<<tiles, kThreads, 0, stream>>>(d_x, n, d_bits, scratch);
-    onebit::ob_compress_scale_kernel<<<1, kScaleThreads, 0, stream>>>(scratch, tiles, n, d_scale);
-    if (tiles > 0)
-        onebit::ob_compress_error_kernel<<<tiles, kThreads, 0, stream>>>(d_x, n, d_scale, d_error);
-    return cudaGetLastError() == cudaSuccess ? OB_OK : OB_ERR_CUDA;
+    // Each launch's own status (cudaLaunchKernel returns it), so an error
+    // left by unrelated earlier work is neither reported nor cleared here.
+    if (tiles > 0) {
+        void *args[] = {(void *)&d_x, (void *)&n, (void *)&d_bits, (void *)&scratch};
+        if (cudaLaunchKernel((const void *)onebit::ob_compress_partial_kernel, dim3(tiles),
+                             dim3(kThreads), args, 0, stream) != cudaSuccess)
+            return OB_ERR_CUDA;
+    }
+    {
+        int tiles_arg = tiles;
+        void *args[] = {(void *)&scratch, (void *)&tiles_arg, (void *)&n, (void *)&d_scale};
+        if (cudaLaunchKernel((const void *)onebit::ob_compress_scale_kernel, dim3(1),
+                             dim3(kScaleThreads), args, 0, stream) != cudaSuccess)
+            return OB_ERR_CUDA;
+    }
+    if (tiles > 0) {
+        const float *scale_in = d_scale;
+        void *args[] = {(void *)&d_x, (void *)&n, (void *)&scale_in, (void *)&d_error};
+        if (cudaLaunchKernel((const void *)onebit::ob_compress_error_kernel, dim3(tiles),
+                             dim3(kThreads), args, 0, stream) != cudaSuccess)
+            return OB_ERR_CUDA;
+    }
+    return OB_OK;
 }

@@ -344,17 +344,26 @@ OB_API void ob_test_fail_host_alloc(int countdown);
  * counterpart to this call; it is the worker stage's compressor of
  * ob_compressed_step applied to a given x:
  *   s = ||x||_2 / sqrt(n);  bits: 1 where x >= 0;  e = x - sign(x) s.
+ * The sign words are those of x bit for bit.  The fp64 sum of squares is
+ * taken in an order of its own (per thread, then per tile, then over the
+ * tiles in order), so s can differ from the workspace path's scale in the
+ * last place (within 1e-6 relative); e is that path's bit for bit whenever
+ * the two scales are equal.
  * d_x: device float[n] (16-byte aligned, no padding needed).  d_bits:
  * device uint32[ceil(n/32)] (bits past n are 0).  d_error: device float[n]
- * (16-byte aligned; may not alias d_x).  d_scale: device float[1].  All
- * work is queued on cuda_stream; the call does no cudaMalloc, cudaFree or
- * other allocating call.  The first call on a device looks up the scratch
- * array's device address (with that device current); make that first call
- * before any stream capture.  Every call shares the one scratch array and
- * overwrites the part it reads, so calls that overlap on the GPU (on
- * different streams) race; serialize them.  n above OB_STATIC_MAX_ELEMENTS
- * returns OB_ERR_WORKSPACE; bad pointers OB_ERR_INVALID_ARG / OB_ERR_ALIGN;
- * a failed lookup or launch OB_ERR_CUDA. */
+ * (16-byte aligned; may not alias d_x).  d_scale: device float[1].  With
+ * n = 0 only *d_scale is written (0) and the other pointers may be NULL.
+ * All work is queued on cuda_stream; the call does no cudaMalloc, cudaFree
+ * or other allocating call.  Every call looks up the scratch array's
+ * device address with the current device (a lookup, not an allocation);
+ * the first call on a device also loads the library's device code there,
+ * so make that first call before any stream capture.  Every call shares
+ * the one scratch array and overwrites the part it reads, so calls that
+ * overlap on the GPU (on different streams) race; serialize them.  n above
+ * OB_STATIC_MAX_ELEMENTS returns OB_ERR_WORKSPACE; bad pointers
+ * OB_ERR_INVALID_ARG / OB_ERR_ALIGN; a failed lookup or a failed launch of
+ * this call's own kernels OB_ERR_CUDA (the call checks each launch's own
+ * status; it does not read or clear an error left by earlier work). */
 #define OB_STATIC_MAX_ELEMENTS ((int64_t)1 << 26)
 OB_API ob_status ob_onebit_compress_static(const float *d_x, int64_t n, uint32_t *d_bits,
                                            float *d_error, float *d_scale, void *cuda_stream);

@@ -7,6 +7,7 @@ from error_compensated_bit_adam_b200 import _binding as B
 from error_compensated_bit_adam_b200 import workloads as WL
 from error_compensated_bit_adam_b200.buckets import BucketedOneBitAdam, split_buckets
 from error_compensated_bit_adam_b200.optimizer import OneBitAdam
+import oracle
 
 
 def test_split_buckets_keeps_order_and_sizes():
@@ -22,7 +23,9 @@ def test_split_buckets_keeps_order_and_sizes():
 def test_bucketed_steps_equal_one_context():
     """Tensors are independent problems, so stepping buckets on their own
     streams, each after an event of the producer stream, gives bit for bit
-    what one context over the whole list gives."""
+    what one context over the whole list gives; and both follow the CPU
+    oracle over the same list (sign words and warmup state bit for bit,
+    scales within 1e-6, parameters within 1e-5 relative L2)."""
     wl = WL.Workload("buckets", WL.encoder_shapes(2, 64, 256, 1000, 64), 4, 2, 3, seed=41,
                      fan_in_scaling=True)
     dev = torch.device("cuda")
@@ -39,6 +42,7 @@ def test_bucketed_steps_equal_one_context():
         for t, o in zip(ts, b_offs[b]):
             bk.params(b)[o:o + wl.numels[t]].copy_(params[offs[t]:offs[t] + wl.numels[t]])
     bgrads = [torch.empty((wl.W, bk.layout(b)[1]), device=dev) for b in range(len(buckets))]
+    orc = oracle.OracleRun(WL.split(params.cpu().numpy(), offs, wl.numels), wl.W, WL.HYPER)
 
     def bucket_grads(step):
         WL.fill_grads(wl, step, scale, grads)
@@ -48,18 +52,21 @@ def test_bucketed_steps_equal_one_context():
                 bgrads[b][:, o:o + wl.numels[t]].copy_(grads[:, offs[t]:offs[t] + wl.numels[t]])
         ev = torch.cuda.Event()
         ev.record()
-        return ev
+        host = grads.cpu().numpy()
+        return ev, [WL.split(host[w], offs, wl.numels) for w in range(wl.W)]
 
     for step in range(5):
-        ev = bucket_grads(step)
+        ev, host_g = bucket_grads(step)
         for b in reversed(range(len(buckets))):  # backward order
             (bk.warmup_step if step < 2 else bk.step)(b, bgrads[b], ev)
         if step == 1:
             bk.wait()
             bk.freeze()
         (whole.warmup_step if step < 2 else whole.step)(grads)
+        (orc.warmup_step if step < 2 else orc.compressed_step)(host_g)
         if step == 1:
             whole.freeze()
+            orc.freeze()
         bk.wait()
     torch.cuda.synchronize()
     p_whole = whole.read(B.OB_STATE_P)
@@ -72,5 +79,19 @@ def test_bucketed_steps_equal_one_context():
             c = p_b[o:o + wl.numels[t]]
             assert np.array_equal(a.view(np.uint32), c.view(np.uint32)), (b, t)
             assert np.array_equal(sw_whole[t], sw_b[i])
+            np.testing.assert_allclose(sw_b[i], orc.s_srv[t], rtol=1e-6, err_msg=f"tensor {t}")
+        words_b = bk.opts[b].read(B.OB_STATE_BITS_SERVER)
+        for t, o in zip(ts, b_offs[b]):
+            nw = (wl.numels[t] + 31) // 32
+            got_w = words_b[o // 32:o // 32 + nw]
+            # bit for bit unless a scale rounded differently (the fp64 sums
+            # of squares are added in different orders): then at most 1e-3
+            # of the signs may differ
+            diff = int(np.unpackbits((got_w ^ orc.sbits[t]).view(np.uint8)).sum())
+            assert diff == 0 or (not np.array_equal(sw_whole, orc.s_srv)
+                                 and diff <= max(1, 1e-3 * 32 * nw)), (b, t, diff)
+    got = np.concatenate(WL.split(p_whole, offs, wl.numels)).astype(np.float64)
+    want = np.concatenate(orc.p).astype(np.float64)
+    assert np.linalg.norm(got - want) <= 1e-5 * np.linalg.norm(want)
     whole.close()
     bk.close()
