@@ -12,9 +12,18 @@ over a list of tensors: every tensor is an independent problem (per-tensor
 scales, packing and server chunks), so a multi-tensor step is the
 per-tensor step applied to each tensor in turn.
 
+The same file holds the 1-bit LAMB variant (layerwise trust ratios on top
+of the same compressed exchange; see the reading in onebit_oracle.c):
+``lamb_warmup_step``, ``lamb_compressed_ratio``, ``lamb_apply_chunk``, and
+``OracleRun(..., lamb=True)``.
+
 Parity status: every C function is pinned by ``tests/test_oracle_pins.py``
 (and the pins are shown to catch planted mistakes by
-``tests/test_oracle_mutants.py``); no function is "parity unpinned".
+``tests/test_oracle_mutants.py``).  The LAMB functions are pinned by what
+mathematics fixes (the trust ratio equals numpy's norm ratio, the step's
+norm is lr * ||p||, a zero norm reduces the step to Adam's / 1-bit Adam's,
+a float64 message-passing brute force); beyond that their reading of the
+1-bit LAMB page, which prints no update rule, is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -96,6 +105,15 @@ class Oracle:
         L.orc_server_compress_chunk.restype = i32
         L.orc_apply_chunk.argtypes = [i64, i32, i32, f32, vp, f32, vp, vp, vp]
         L.orc_apply_chunk.restype = None
+        L.orc_sum_squares.argtypes = [i64, vp]
+        L.orc_sum_squares.restype = ctypes.c_double
+        L.orc_lamb_warmup_step.argtypes = [i64, i32, i32, f32, f32, f32, f32, vp, vp, vp, vp,
+                                           ctypes.POINTER(f32)]
+        L.orc_lamb_warmup_step.restype = i32
+        L.orc_lamb_compressed_ratio.argtypes = [i64, i32, vp, vp, vp, vp]
+        L.orc_lamb_compressed_ratio.restype = f32
+        L.orc_lamb_apply_chunk.argtypes = [i64, i32, i32, f32, f32, vp, f32, vp, vp, vp]
+        L.orc_lamb_apply_chunk.restype = None
         self.L = L
         self.path = path
 
@@ -187,6 +205,37 @@ class Oracle:
                                _ptr(p), _ptr(m))
 
 
+    # ----------------------------------------------------- 1-bit LAMB
+    def sum_squares(self, x: np.ndarray) -> float:
+        return float(self.L.orc_sum_squares(_f32(x).size, _ptr(x)))
+
+    def lamb_warmup_step(self, t: int, hp: dict, g: Sequence[np.ndarray], m: np.ndarray,
+                         v: np.ndarray, p: np.ndarray) -> np.float32:
+        """One 1-bit LAMB warmup step of one tensor; returns its trust ratio."""
+        n = m.size
+        for a in (*g, m, v, p):
+            _f32(a)
+            assert a.size == n
+        ratio = ctypes.c_float()
+        rc = self.L.orc_lamb_warmup_step(n, len(g), t, hp["beta1"], hp["beta2"], hp["eps"],
+                                         hp["lr"], _ptr_array(g), _ptr(m), _ptr(v), _ptr(p),
+                                         ctypes.byref(ratio))
+        if rc != 0:
+            raise MemoryError("oracle LAMB warmup out of memory")
+        return np.float32(ratio.value)
+
+    def lamb_compressed_ratio(self, W: int, sbits: np.ndarray, s_srv, d: np.ndarray,
+                              p: np.ndarray) -> np.float32:
+        s_srv = np.ascontiguousarray(s_srv, np.float32)
+        return np.float32(self.L.orc_lamb_compressed_ratio(p.size, W, _ptr(_u32(sbits)), _ptr(s_srv),
+                                                           _ptr(_f32(d)), _ptr(_f32(p))))
+
+    def lamb_apply_chunk(self, j: int, W: int, lr: float, ratio, sbits: np.ndarray, s_srv_j,
+                         d: np.ndarray, p: np.ndarray, m: np.ndarray) -> None:
+        self.L.orc_lamb_apply_chunk(p.size, W, j, lr, float(ratio), _ptr(_u32(sbits)),
+                                    float(s_srv_j), _ptr(d), _ptr(p), _ptr(m))
+
+
 _default: Optional[Oracle] = None
 
 
@@ -210,12 +259,19 @@ class OracleRun:
     and update of every (tensor, server chunk), and slices of the
     elementwise warmup and freeze.  Each call is still the plain single-threaded C function, so
     the results do not depend on `threads`.
+
+    lamb=True runs 1-bit LAMB: the warmup and the update scale each
+    tensor's step by its trust ratio (kept in ``ratio`` after each step);
+    the warmup then runs one call per tensor, the compressed step the
+    server stage of every chunk before any update.
     """
 
     SLICE = 1 << 22  # elements per warmup/freeze call when threaded
 
     def __init__(self, params: Sequence[np.ndarray], W: int, hp: dict,
-                 oracle: Optional[Oracle] = None, threads: int = 1):
+                 oracle: Optional[Oracle] = None, threads: int = 1, lamb: bool = False):
+        self.lamb = bool(lamb)
+        self.ratio: Optional[np.ndarray] = None  # [T] trust ratios of the last step (LAMB)
         self.threads = max(1, int(threads))
         self.o = oracle or default()
         self.W = int(W)
@@ -258,6 +314,15 @@ class OracleRun:
         assert self.d is None, "already frozen"
         self.t_warmup += 1
         t_step = self.t_warmup
+        if self.lamb:  # the trust ratio needs the whole tensor: one call per tensor
+            self.ratio = np.zeros(self.T, np.float32)
+
+            def lamb_job(t):
+                self.ratio[t] = self.o.lamb_warmup_step(t_step, self.hp,
+                                                        [grads[w][t] for w in range(self.W)],
+                                                        self.m[t], self.v[t], self.p[t])
+            self._run([lambda t=t: lamb_job(t) for t in range(self.T)])
+            return
         jobs = []
         for t in range(self.T):
             for a, b in self._slices(self.numel[t]):
@@ -312,6 +377,26 @@ class OracleRun:
                                self.p[t], self.m[t])
 
         self._run([lambda t=t, w=w: worker_job(t, w) for t in range(T) for w in range(W)])
+        if self.lamb:  # server stage of every chunk, then each tensor's ratio, then the update
+            def srv_job(t, j):
+                bits = [self.bits_w[w][t] for w in range(W)]
+                self.s_srv[t, j] = self.o.server_compress_chunk(j, bits, self.s_w[:, t],
+                                                                self.e_s[t], self.sbits[t])
+
+            for t in range(T):
+                self.sbits[t] = np.zeros(self.o.num_words(self.numel[t]), np.uint32)
+            self._run([lambda t=t, j=j: srv_job(t, j) for t in range(T) for j in range(W)])
+            self.ratio = np.zeros(T, np.float32)
+
+            def ratio_job(t):
+                self.ratio[t] = self.o.lamb_compressed_ratio(W, self.sbits[t], self.s_srv[t],
+                                                             self.d[t], self.p[t])
+            self._run([lambda t=t: ratio_job(t) for t in range(T)])
+            self._run([lambda t=t, j=j: self.o.lamb_apply_chunk(
+                j, W, self.hp["lr"], self.ratio[t], self.sbits[t], self.s_srv[t, j], self.d[t],
+                self.p[t], self.m[t]) for t in range(T) for j in range(W)])
+            self.t_compressed += 1
+            return
         if self.threads == 1:
             self._run([lambda t=t: server_job(t) for t in range(T)])
         else:

@@ -122,39 +122,49 @@ ORC_API void orc_chunk_range(int64_t n, int W, int j, int64_t *begin, int64_t *e
 /* ------------------------------------------------------------------ */
 
 /* [1BA, Proposed method, 1]: the warmup is plain Adam on the averaged
- * gradient.  One step t (t = 1, 2, ...) over W workers' gradients g[w]:
+ * gradient.  For element i of one step t (t = 1, 2, ...) over W workers'
+ * gradients g[w]:
  *   gbar = (g_0 + g_1 + ... + g_{W-1}) / W   (sum from +0.0, in w order)
  *   m = beta1*m + (1-beta1)*gbar
  *   v = beta2*v + (1-beta2)*gbar^2
- *   p = p - lr * (m/bc1) / (sqrt(v/bc2) + eps),
+ * updated in place, and the returned direction of the step
+ *   r = (m/bc1) / (sqrt(v/bc2) + eps),
  * with bc1 = 1 - beta1^t and bc2 = 1 - beta2^t taken in double and rounded
- * once to float. */
-ORC_API void orc_adam_warmup_step(int64_t n, int W, int t, float beta1, float beta2, float eps,
-                                  float lr, const float *const *g, float *m, float *v, float *p) {
+ * once to float by the caller. */
+static float adam_moments_and_direction(int64_t i, int W, const float *const *g, float beta1,
+                                        float beta2, float bc1, float bc2, float eps, float *m,
+                                        float *v) {
     const float c1 = 1.0f - beta1;
     const float c2 = 1.0f - beta2;
+    const float wf = (float)W;
+    float acc = 0.0f;
+    for (int w = 0; w < W; ++w) acc = acc + g[w][i];
+    const float gbar = acc / wf;
+
+    const float m_old = beta1 * m[i];
+    const float m_new = c1 * gbar;
+    m[i] = m_old + m_new;
+
+    const float gsq = gbar * gbar;
+    const float v_old = beta2 * v[i];
+    const float v_new = c2 * gsq;
+    v[i] = v_old + v_new;
+
+    const float mhat = m[i] / bc1;
+    const float vhat = v[i] / bc2;
+    const float root = sqrtf(vhat);
+    const float denom = root + eps;
+    return mhat / denom;
+}
+
+/* One Adam warmup step: the moments and direction above, then
+ *   p = p - lr * r. */
+ORC_API void orc_adam_warmup_step(int64_t n, int W, int t, float beta1, float beta2, float eps,
+                                  float lr, const float *const *g, float *m, float *v, float *p) {
     const float bc1 = (float)(1.0 - pow((double)beta1, (double)t));
     const float bc2 = (float)(1.0 - pow((double)beta2, (double)t));
-    const float wf = (float)W;
     for (int64_t i = 0; i < n; ++i) {
-        float acc = 0.0f;
-        for (int w = 0; w < W; ++w) acc = acc + g[w][i];
-        const float gbar = acc / wf;
-
-        const float m_old = beta1 * m[i];
-        const float m_new = c1 * gbar;
-        m[i] = m_old + m_new;
-
-        const float gsq = gbar * gbar;
-        const float v_old = beta2 * v[i];
-        const float v_new = c2 * gsq;
-        v[i] = v_old + v_new;
-
-        const float mhat = m[i] / bc1;
-        const float vhat = v[i] / bc2;
-        const float root = sqrtf(vhat);
-        const float denom = root + eps;
-        const float ratio = mhat / denom;
+        const float ratio = adam_moments_and_direction(i, W, g, beta1, beta2, bc1, bc2, eps, m, v);
         const float delta = lr * ratio;
         p[i] = p[i] - delta;
     }
@@ -287,4 +297,97 @@ ORC_API void orc_apply_chunk(int64_t n, int W, int j, float lr, const uint32_t *
 ORC_API void orc_apply(int64_t n, int W, float lr, const uint32_t *sbits, const float *s_srv,
                        const float *d, float *p, float *m) {
     for (int j = 0; j < W; ++j) orc_apply_chunk(n, W, j, lr, sbits, s_srv[j], d, p, m);
+}
+
+/* ------------------------------------------------------------------ */
+/* 1-bit LAMB: layerwise adaptive learning rates                       */
+/* ------------------------------------------------------------------ */
+
+/* The review page "1-bit LAMB: Communication Efficient Large-Scale
+ * Large-Batch Training with LAMB's Convergence Speed" gives only its
+ * abstract: LAMB's adaptive layerwise learning rates are kept while the
+ * communication is compressed, on top of the 1-bit Adam scheme above.  It
+ * prints no update rule.  The reading taken here is the plainest the
+ * abstract supports:
+ *   - the layerwise rate is LAMB's trust ratio of each tensor,
+ *       ratio = ||p|| / ||u||   (1 when either norm is 0),
+ *     u being the tensor's update direction, and the step is
+ *       p = p - (lr * ratio) * u;
+ *   - during the warmup u is full-precision Adam's m_hat / (sqrt(v_hat) +
+ *     eps) (warmup = LAMB);
+ *   - during the compression phase u = m_hat / d, m_hat being the momentum
+ *     decoded from the compressed collective and d the frozen denominator:
+ *     every worker holds the same p and m_hat after the gather, so every
+ *     worker computes the same ratio although the momentum was compressed;
+ *   - the ratio is recomputed at every step (nothing else is frozen).
+ * Norms are sums of squares in double (sequential), the ratio
+ * (float)sqrt(P / U), rounded once; lr * ratio is one float
+ * multiplication.  With ratio = 1 the steps are exactly the Adam warmup and
+ * the 1-bit Adam update above. */
+
+/* Sum of squares in double, sequential. */
+ORC_API double orc_sum_squares(int64_t n, const float *x) {
+    double s = 0.0;
+    for (int64_t i = 0; i < n; ++i) s += (double)x[i] * (double)x[i];
+    return s;
+}
+
+/* LAMB's trust ratio from the squared norms of p and of the update u. */
+static float trust_ratio(double p_sq, double u_sq) {
+    if (p_sq > 0.0 && u_sq > 0.0) return (float)sqrt(p_sq / u_sq);
+    return 1.0f;
+}
+
+/* One warmup step of 1-bit LAMB: the Adam moments of the averaged
+ * gradient as in orc_adam_warmup_step, then the tensor's trust ratio of
+ * p (before the step) and the Adam direction r, then the step.  *ratio_out
+ * receives the ratio.  Returns 0, or -1 when out of memory. */
+ORC_API int orc_lamb_warmup_step(int64_t n, int W, int t, float beta1, float beta2, float eps,
+                                 float lr, const float *const *g, float *m, float *v, float *p,
+                                 float *ratio_out) {
+    const float bc1 = (float)(1.0 - pow((double)beta1, (double)t));
+    const float bc2 = (float)(1.0 - pow((double)beta2, (double)t));
+    float *r = (float *)calloc((size_t)(n > 0 ? n : 1), sizeof(float));
+    if (!r) return -1;
+    for (int64_t i = 0; i < n; ++i)
+        r[i] = adam_moments_and_direction(i, W, g, beta1, beta2, bc1, bc2, eps, m, v);
+    const float ratio = trust_ratio(orc_sum_squares(n, p), orc_sum_squares(n, r));
+    const float lr_t = lr * ratio;
+    for (int64_t i = 0; i < n; ++i) {
+        const float delta = lr_t * r[i];
+        p[i] = p[i] - delta;
+    }
+    free(r);
+    *ratio_out = ratio;
+    return 0;
+}
+
+/* The compression phase's trust ratio of one tensor, once every server
+ * chunk's words and scale are known: p before the step, and the direction
+ * u = m_hat / d with m_hat = sign'(i) * s'_j decoded from the server words.
+ * ||u||^2 is taken as the sum of (m_hat / d)^2 over the elements, each
+ * quotient formed in double from the float values. */
+ORC_API float orc_lamb_compressed_ratio(int64_t n, int W, const uint32_t *sbits, const float *s_srv,
+                                        const float *d, const float *p) {
+    double u_sq = 0.0;
+    for (int j = 0; j < W; ++j) {
+        int64_t b, e;
+        orc_chunk_range(n, W, j, &b, &e);
+        for (int64_t i = b; i < e; ++i) {
+            const double q = (double)signed_scale(get_bit(sbits, i), s_srv[j]) / (double)d[i];
+            u_sq += q * q;
+        }
+    }
+    return trust_ratio(orc_sum_squares(n, p), u_sq);
+}
+
+/* Gather and update of one chunk of the compression phase of 1-bit LAMB:
+ * the 1-bit Adam update of orc_apply_chunk with the tensor's layerwise
+ * rate lr * ratio in place of lr:
+ *   p = p - (lr * ratio) * (m_hat / d);   m = m_hat. */
+ORC_API void orc_lamb_apply_chunk(int64_t n, int W, int j, float lr, float ratio,
+                                  const uint32_t *sbits, float s_srv_j, const float *d, float *p,
+                                  float *m) {
+    const float lr_t = lr * ratio;
+    orc_apply_chunk(n, W, j, lr_t, sbits, s_srv_j, d, p, m);
 }

@@ -363,12 +363,14 @@ def _unpack_bytes(buf: bytes, count: int) -> np.ndarray:
     return np.array(codes, F64)
 
 
-def brute_force_step(W, m, d, p, grads, e_w, e_s):
+def brute_force_step(W, m, d, p, grads, e_w, e_s, lamb=False, lr=None):
     """One compressed step as W workers and W servers exchanging byte
-    messages, in float64.  Returns a dict of results and the bytes sent."""
+    messages, in float64.  Returns a dict of results and the bytes sent.
+    lamb: the update is 1-bit LAMB's, scaled by the trust ratio
+    ||p|| / ||m_hat / d|| (1 when a norm is 0)."""
     n = m.size
     b1 = F64(F32(HP["beta1"]))
-    lr = F64(F32(HP["lr"]))
+    lr = F64(F32(HP["lr"] if lr is None else lr))
     # chunk plan: roundup(ceil(n/W), 128) elements per server, in order
     L = -(-(-(-n // W)) // 128) * 128 if n else 0
     chunks = [(min(n, j * L), min(n, (j + 1) * L)) for j in range(W)]
@@ -403,7 +405,12 @@ def brute_force_step(W, m, d, p, grads, e_w, e_s):
     for j, (b, e) in enumerate(chunks):
         buf, s2 = bcast[j]
         m_hat[b:e] = s2 * _unpack_bytes(buf, e - b)
-    res["p"] = p - lr * m_hat / d
+    u = m_hat / d
+    ratio = 1.0
+    if lamb and np.linalg.norm(p) > 0 and np.linalg.norm(u) > 0:
+        ratio = np.linalg.norm(p) / np.linalg.norm(u)
+    res["ratio"] = ratio
+    res["p"] = p - lr * ratio * u
     res["m"] = m_hat
     res["wire_bytes"] = wire
     return res
@@ -442,6 +449,150 @@ def pin_brute_force_message_passing(o, seed=10):
                 np.testing.assert_allclose(m, ref["m"], rtol=1e-5, atol=1e-12)
                 np.testing.assert_allclose(p, ref["p"], rtol=1e-6, atol=1e-9)
                 np.testing.assert_allclose(e_s, ref["e_s"], rtol=1e-4, atol=1e-9)
+
+
+# ---------------------------------------------------------------------------
+# 1-bit LAMB: layerwise trust ratios  (the 1-bit LAMB review page, Abstract)
+# ---------------------------------------------------------------------------
+
+LAMB_LR = 0.05  # large enough that p_new - p_old is far above p's rounding
+
+
+def pin_lamb_warmup_from_zero_params_is_adam(o, W=3, n=777, seed=21):
+    """With p = 0 the trust ratio is 1 by LAMB's convention, so the first
+    LAMB warmup step is textbook Adam's first step (torch.optim.Adam)."""
+    rng = np.random.default_rng(seed)
+    p = np.zeros(n, F32)
+    tp = torch.nn.Parameter(torch.zeros(n))
+    opt = torch.optim.Adam([tp], lr=hp32("lr"), betas=(hp32("beta1"), hp32("beta2")),
+                           eps=hp32("eps"), foreach=False)
+    g = [rng.normal(0, 1e-3, n).astype(F32) for _ in range(W)]
+    m = np.zeros(n, F32)
+    v = np.zeros(n, F32)
+    ratio = o.lamb_warmup_step(1, HP, g, m, v, p)
+    assert ratio == 1.0, ratio
+    tp.grad = torch.from_numpy((np.sum(np.stack(g).astype(F64), 0) / W).astype(F32))
+    opt.step()
+    np.testing.assert_allclose(m, opt.state[tp]["exp_avg"].numpy(), rtol=3e-6, atol=1e-11)
+    np.testing.assert_allclose(v, opt.state[tp]["exp_avg_sq"].numpy(), rtol=3e-6, atol=1e-17)
+    np.testing.assert_allclose(p, tp.detach().numpy(), rtol=3e-6, atol=2e-9)
+
+
+def _adam_direction(m, v, t):
+    """Adam's update direction from its moments, in float64."""
+    b1, b2, eps = F64(F32(HP["beta1"])), F64(F32(HP["beta2"])), F64(F32(HP["eps"]))
+    mh = m.astype(F64) / (1 - b1 ** t)
+    vh = v.astype(F64) / (1 - b2 ** t)
+    return mh / (np.sqrt(vh) + eps)
+
+
+def pin_lamb_warmup_layerwise_step(o, W=2, n=3000, steps=4, seed=22):
+    """LAMB's layerwise step, from its definition: the trust ratio equals
+    numpy's ||p|| / ||r|| with r Adam's direction, the step is -lr ratio r,
+    so its norm is lr ||p|| whatever the gradients; two tensors that differ
+    only by a factor 10 in p take steps that differ by the same factor."""
+    rng = np.random.default_rng(seed)
+    hp = dict(HP, lr=LAMB_LR)
+    lr = F64(F32(LAMB_LR))
+    base = rng.normal(0, 0.02, n).astype(F32)
+    ps = [base.copy(), (base * F32(10)).astype(F32)]
+    ms = [np.zeros(n, F32) for _ in ps]
+    vs = [np.zeros(n, F32) for _ in ps]
+    for t in range(1, steps + 1):
+        g = [rng.normal(0, 1e-3, n).astype(F32) for _ in range(W)]
+        steps_norm = []
+        for k in range(2):
+            before = ps[k].astype(F64)
+            ratio = o.lamb_warmup_step(t, hp, g, ms[k], vs[k], ps[k])
+            r = _adam_direction(ms[k], vs[k], t)
+            want = np.linalg.norm(before) / np.linalg.norm(r)
+            assert abs(F64(ratio) - want) <= 1e-6 * want, (t, k, ratio, want)
+            delta = ps[k].astype(F64) - before
+            np.testing.assert_allclose(delta, -lr * F64(ratio) * r, rtol=1e-4,
+                                       atol=4 * float(np.max(ulp(ps[k]))))
+            norm = np.linalg.norm(delta)
+            assert abs(norm - lr * np.linalg.norm(before)) <= 1e-5 * lr * np.linalg.norm(before)
+            steps_norm.append(norm)
+        assert abs(steps_norm[1] / steps_norm[0] - 10.0) <= 1e-4
+
+
+def _server_inputs(rng, n, W):
+    o_bits = rng.integers(0, 2 ** 32, (n + 31) // 32, dtype=np.uint64).astype(np.uint32)
+    if n % 32:
+        o_bits[-1] &= np.uint32((1 << (n % 32)) - 1)
+    s_srv = rng.uniform(1e-4, 1e-3, W).astype(F32)
+    d = (np.sqrt(rng.uniform(1e-7, 1e-5, n)) + 1e-8).astype(F32)
+    return o_bits, s_srv, d
+
+
+def pin_lamb_compressed_update(o, seed=23):
+    """The compression phase's LAMB update of one tensor from given server
+    words and chunk scales: m_hat decoded independently (numpy bits), the
+    ratio equal to numpy's ||p|| / ||m_hat / d||, the step -lr ratio
+    m_hat/d with norm lr ||p||, m = m_hat exactly; with p = 0 the ratio is
+    1 and the update is 1-bit Adam's bit for bit."""
+    rng = np.random.default_rng(seed)
+    lr = F64(F32(LAMB_LR))
+    for W, n in ((1, 100), (3, 1000), (8, 5000), (16, 130)):
+        sbits, s_srv, d = _server_inputs(rng, n, W)
+        code = np.where(unpack_words(sbits, n), 1.0, -1.0)
+        m_hat = np.zeros(n)
+        for j in range(W):
+            b, e = o.chunk_range(n, W, j)
+            m_hat[b:e] = code[b:e] * F64(s_srv[j])
+        u = m_hat / d.astype(F64)
+        p = rng.normal(0, 0.02, n).astype(F32)
+        before = p.astype(F64)
+        m = np.zeros(n, F32)
+        ratio = o.lamb_compressed_ratio(W, sbits, s_srv, d, p)
+        want = np.linalg.norm(before) / np.linalg.norm(u)
+        assert abs(F64(ratio) - want) <= 1e-6 * want, (W, n, ratio, want)
+        for j in range(W):
+            o.lamb_apply_chunk(j, W, LAMB_LR, ratio, sbits, s_srv[j], d, p, m)
+        assert np.array_equal(m.astype(F64), m_hat)
+        delta = p.astype(F64) - before
+        np.testing.assert_allclose(delta, -lr * F64(ratio) * u, rtol=1e-4,
+                                   atol=4 * float(np.max(ulp(p))))
+        assert abs(np.linalg.norm(delta) - lr * np.linalg.norm(before)) <= 1e-5 * lr * np.linalg.norm(before)
+        # p = 0: ratio 1, the 1-bit Adam update
+        z, za = np.zeros(n, F32), np.zeros(n, F32)
+        assert o.lamb_compressed_ratio(W, sbits, s_srv, d, z) == 1.0
+        for j in range(W):
+            o.lamb_apply_chunk(j, W, LAMB_LR, F32(1.0), sbits, s_srv[j], d, z, m)
+        o.apply_update(LAMB_LR, sbits, s_srv, d, za, m)
+        assert np.array_equal(z.view(np.uint32), za.view(np.uint32))
+
+
+def pin_lamb_brute_force_message_passing(o, seed=24):
+    """Whole compressed 1-bit LAMB steps against the float64 message-passing
+    brute force with the LAMB update."""
+    rng = np.random.default_rng(seed)
+    hp = dict(HP, lr=LAMB_LR)
+    for W in (1, 2, 3, 8):
+        for n in (5, 33, 200, 300):
+            p = rng.normal(0, 0.02, n).astype(F32)
+            m = rng.normal(0, 1e-3, n).astype(F32)
+            d = (np.sqrt(rng.uniform(1e-7, 1e-5, n)) + 1e-8).astype(F32)
+            e_w = [rng.normal(0, 2e-4, n).astype(F32) for _ in range(W)]
+            e_s = rng.normal(0, 2e-4, n).astype(F32)
+            for _ in range(2):
+                grads = [rng.normal(0, 1e-3, n).astype(F32) for _ in range(W)]
+                ref = brute_force_step(W, m.astype(F64), d.astype(F64), p.astype(F64),
+                                       [g.astype(F64) for g in grads],
+                                       [e.astype(F64) for e in e_w], e_s.astype(F64), lamb=True,
+                                       lr=LAMB_LR)
+                bits, scales = [], []
+                for w in range(W):
+                    b, s = o.worker_compress(hp["beta1"], m, grads[w], e_w[w])
+                    bits.append(b)
+                    scales.append(s)
+                sb, ss = o.server_compress(bits, np.array(scales, F32), e_s)
+                ratio = o.lamb_compressed_ratio(W, sb, ss, d, p)
+                assert abs(F64(ratio) - ref["ratio"]) <= 1e-5 * ref["ratio"], (W, n)
+                for j in range(W):
+                    o.lamb_apply_chunk(j, W, hp["lr"], ratio, sb, ss[j], d, p, m)
+                np.testing.assert_allclose(m, ref["m"], rtol=1e-5, atol=1e-12)
+                np.testing.assert_allclose(p, ref["p"], rtol=1e-5, atol=1e-8)
 
 
 # ---------------------------------------------------------------------------
@@ -497,4 +648,8 @@ ALL_PINS = [
     pin_chunk_layout,
     pin_brute_force_message_passing,
     pin_communication_volume,
+    pin_lamb_warmup_from_zero_params_is_adam,
+    pin_lamb_warmup_layerwise_step,
+    pin_lamb_compressed_update,
+    pin_lamb_brute_force_message_passing,
 ]

@@ -18,8 +18,8 @@ import oracle_pins
 MUTANTS = [
     ("warmup_drops_bias_correction_m", "const float mhat = m[i] / bc1;", "const float mhat = m[i];"),
     ("warmup_eps_inside_sqrt",
-     "const float root = sqrtf(vhat);\n        const float denom = root + eps;",
-     "const float root = sqrtf(vhat + eps);\n        const float denom = root;"),
+     "const float root = sqrtf(vhat);\n    const float denom = root + eps;",
+     "const float root = sqrtf(vhat + eps);\n    const float denom = root;"),
     ("warmup_sums_instead_of_averaging", "const float gbar = acc / wf;", "const float gbar = acc;"),
     ("warmup_variance_not_squared", "const float gsq = gbar * gbar;", "const float gsq = gbar;"),
     ("warmup_update_wrong_sign", "p[i] = p[i] - delta;\n    }\n}\n\n/* [1BA, Abstract; Proposed",
@@ -73,6 +73,21 @@ MUTANTS = [
      "const float m_old = c1 * m[i];\n        const float m_new = beta1 * g[i];"),
     ("warmup_variance_uses_beta1", "const float v_old = beta2 * v[i];", "const float v_old = beta1 * v[i];"),
     ("chunk_words_rounded_down", "const int64_t per = (nw + W - 1) / W;", "const int64_t per = nw / W;"),
+    # 1-bit LAMB
+    ("lamb_ratio_inverted", "return (float)sqrt(p_sq / u_sq);", "return (float)sqrt(u_sq / p_sq);"),
+    ("lamb_ratio_without_root", "return (float)sqrt(p_sq / u_sq);", "return (float)(p_sq / u_sq);"),
+    ("lamb_zero_norm_gives_zero_rate", "    return 1.0f;\n}", "    return 0.0f;\n}"),
+    ("lamb_warmup_ignores_ratio", "const float lr_t = lr * ratio;\n    for", "const float lr_t = lr;\n    for"),
+    ("lamb_warmup_ratio_of_momentum", "orc_sum_squares(n, r));", "orc_sum_squares(n, m));"),
+    ("lamb_warmup_ratio_of_variance", "trust_ratio(orc_sum_squares(n, p), orc_sum_squares(n, r))",
+     "trust_ratio(orc_sum_squares(n, v), orc_sum_squares(n, r))"),
+    ("lamb_compressed_ratio_of_d", "return trust_ratio(orc_sum_squares(n, p), u_sq);",
+     "return trust_ratio(orc_sum_squares(n, d), u_sq);"),
+    ("lamb_compressed_ratio_ignores_d", "/ (double)d[i];", "/ 1.0;"),
+    ("lamb_compressed_ratio_chunk0_scale", "signed_scale(get_bit(sbits, i), s_srv[j]) / (double)d[i]",
+     "signed_scale(get_bit(sbits, i), s_srv[0]) / (double)d[i]"),
+    ("lamb_apply_ignores_ratio", "const float lr_t = lr * ratio;\n    orc_apply_chunk",
+     "const float lr_t = lr + 0.0f * ratio;\n    orc_apply_chunk"),
 ]
 
 MUTANT_CFLAGS = [f for f in oracle.CFLAGS if f != "-Werror"]
