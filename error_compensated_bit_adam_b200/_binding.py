@@ -36,6 +36,7 @@ OB_STATE_S_SERVER = 7
 OB_STATE_BITS_WORKER = 8
 OB_STATE_BITS_SERVER = 9
 OB_STATE_STEP = 10
+OB_STATE_RATIO = 11
 
 OB_STATIC_MAX_ELEMENTS = 1 << 26
 
@@ -56,18 +57,18 @@ EXPORTS = (
     "ob_profile_enable", "ob_profile_read", "ob_kernel_name", "ob_test_fail_host_alloc",
     "ob_onebit_compress_static", "ob_set_lr", "ob_graph_enable",
     "ob_server_shard_range", "ob_set_server_shard", "ob_worker_stage", "ob_worker_exchange_buffers",
-    "ob_server_stage", "ob_server_exchange_buffers", "ob_apply_update",
+    "ob_server_stage", "ob_server_exchange_buffers", "ob_apply_update", "ob_set_layerwise",
 )
 
 
 __all__ = [name for name in EXPORTS] + [
-    "OnebitError", "lib", "status_name", "LIBRARY",
+    "OnebitError", "lib", "status_name", "LIBRARY", "pointer_array",
     "OB_ABI_VERSION", "OB_MAX_WORKERS", "OB_TENSOR_ALIGN", "OB_STATIC_MAX_ELEMENTS",
     "OB_OK", "OB_ERR_INVALID_ARG", "OB_ERR_PHASE", "OB_ERR_ALIGN", "OB_ERR_WORKSPACE",
     "OB_ERR_OOM", "OB_ERR_CUDA", "OB_ERR_DEVICE_TIMEOUT",
     "OB_STATE_P", "OB_STATE_M", "OB_STATE_V", "OB_STATE_D", "OB_STATE_E_WORKER",
     "OB_STATE_E_SERVER", "OB_STATE_S_WORKER", "OB_STATE_S_SERVER", "OB_STATE_BITS_WORKER",
-    "OB_STATE_BITS_SERVER", "OB_STATE_STEP",
+    "OB_STATE_BITS_SERVER", "OB_STATE_STEP", "OB_STATE_RATIO",
     "OB_K_WARMUP", "OB_K_FREEZE", "OB_K_PACK", "OB_K_PACK_SCALE", "OB_K_SERVER",
     "OB_K_SERVER_SCALE", "OB_K_APPLY", "OB_NUM_KERNELS",
 ]
@@ -127,6 +128,7 @@ def lib() -> ctypes.CDLL:
         "ob_server_exchange_buffers": (i32, [vp, ctypes.POINTER(vp), ctypes.POINTER(sz),
                                              ctypes.POINTER(vp), ctypes.POINTER(sz)]),
         "ob_apply_update": (i32, [vp]),
+        "ob_set_layerwise": (i32, [vp, i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -156,10 +158,18 @@ def _i64_array(values: Sequence[int]):
 
 
 def _ptrs(ptrs: Sequence[int]):
+    """A C array of pointers (a ctypes pointer array is passed through)."""
+    if isinstance(ptrs, ctypes.Array):
+        return ptrs
     arr = (ctypes.c_void_p * max(1, len(ptrs)))()
     for i, p in enumerate(ptrs):
         arr[i] = int(p)
     return arr
+
+
+def pointer_array(ptrs: Sequence[int]):
+    """A reusable C array of device pointers for the step calls."""
+    return _ptrs(list(ptrs))
 
 
 # --------------------------------------------------------------- host only
@@ -257,6 +267,10 @@ def ob_write_state(ctx: int, kind: int, index: int, host_src: int, nbytes: int) 
 
 def ob_set_lr(ctx: int, lr: float) -> None:
     _check(lib().ob_set_lr(ctx, float(lr)), "ob_set_lr")
+
+
+def ob_set_layerwise(ctx: int, on: bool) -> None:
+    _check(lib().ob_set_layerwise(ctx, 1 if on else 0), "ob_set_layerwise")
 
 
 def ob_graph_enable(ctx: int, on: bool) -> None:

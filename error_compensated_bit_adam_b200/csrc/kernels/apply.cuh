@@ -29,9 +29,11 @@ struct ApplyParams {
 // loads ahead of the previous slot's arithmetic, and holding all slots in
 // registers costs residency; so each thread first copies all its d and p
 // slots into shared memory (cp.async, 32 KiB per CTA), then computes.
-template <bool FULL>
-__device__ __forceinline__ void apply_tile(const ApplyParams &P, const Tile &tile, float4 (*sd)[kThreads],
-                                           float4 (*spp)[kThreads]) {
+// lr: the step's learning rate (P.lr, or 1-bit LAMB's layerwise rate).
+// With NORM the thread's sum of the new p^2 is returned (else 0).
+template <bool FULL, bool NORM>
+__device__ __forceinline__ double apply_tile(const ApplyParams &P, const Tile &tile, float4 (*sd)[kThreads],
+                                             float4 (*spp)[kThreads], float lr) {
     const int tid = threadIdx.x, lane = tid & 31;
     const uint32_t sb = __float_as_uint(P.sp[tile.tensor * P.W + tile.chunk]);
     const int shift = 4 * (lane & 7);
@@ -50,6 +52,7 @@ __device__ __forceinline__ void apply_tile(const ApplyParams &P, const Tile &til
     }
     cp_async_commit();
     cp_async_wait<0>();
+    double pp = 0.0;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
         const int off = 4 * (tid + kThreads * u);
@@ -63,24 +66,29 @@ __device__ __forceinline__ void apply_tile(const ApplyParams &P, const Tile &til
         for (int k = 0; k < 4; ++k) {
             if (FULL || k < real) {
                 const float m_hat = __uint_as_float(((inv[u] << (31 - k)) & 0x80000000u) | sb);
-                const float delta = __fmul_rn(P.lr, __fdiv_rn(m_hat, get(d, k)));
-                set(p, k, __fsub_rn(get(p, k), delta));
+                const float delta = __fmul_rn(lr, __fdiv_rn(m_hat, get(d, k)));
+                const float pk = __fsub_rn(get(p, k), delta);
+                set(p, k, pk);
                 set(m, k, m_hat);
+                if (NORM) pp = __fma_rn((double)pk, (double)pk, pp);
             }
         }
         st_stream(P.p + i, p);
         if (P.m) st_stream(P.m + i, m);
     }
+    return pp;
 }
 
 __global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constant__ ApplyParams P) {
     __shared__ float4 sd[kUnroll][kThreads];   // this thread's d slots
     __shared__ float4 spp[kUnroll][kThreads];  // and p slots
-    const Tile tile = P.tiles[blockIdx.x];
+    const Tile tile = P.tiles[blockIdx.x];  // the work list is written once, at create
+    grid_dependency_wait();
+    allow_dependent_launch();
     if (tile.count == kTile)
-        apply_tile<true>(P, tile, sd, spp);
+        apply_tile<true, false>(P, tile, sd, spp, P.lr);
     else
-        apply_tile<false>(P, tile, sd, spp);
+        apply_tile<false, false>(P, tile, sd, spp, P.lr);
 }
 
 }  // namespace onebit

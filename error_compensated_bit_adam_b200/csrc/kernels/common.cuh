@@ -152,6 +152,22 @@ __device__ __forceinline__ double block_sum(double v, double *smem) {
     return acc;
 }
 
+// Programmatic dependent launch (sm_90+).  A kernel launched with the
+// programmatic-serialization attribute may start while the kernel before
+// it on the stream is still finishing; grid_dependency_wait() blocks until
+// every earlier grid of the stream has completed and its memory is visible,
+// so each kernel calls it before reading anything an earlier kernel wrote.
+// In a kernel launched without the attribute it returns at once.
+// allow_dependent_launch() lets the next such kernel be scheduled once
+// every CTA of this grid has called it (or exited); it has no effect on
+// correctness, only on how early the next grid's CTAs are placed.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;\n" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+    asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // Real elements (0..4) of the float4 slot at tile offset off.
 __device__ __forceinline__ int slot_real(int count, int off) { return min(4, max(0, count - off)); }
 

@@ -4,6 +4,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "scale.cuh"
 
 namespace onebit {
 
@@ -15,8 +16,9 @@ struct PackParams {
     int n_tiles;                     // total tiles (row length of partial)
     const float *m;                  // [n_pad] dense momentum (when m_dense)
     const uint32_t *m_bits;          // [n_pad/32] last step's server signs (when !m_dense)
-    const float *m_scale;            // [T][W] last step's server scales (when !m_dense)
+    const float *m_scale;            // [T][chunks] last step's server scales (when !m_dense)
     int m_dense;
+    int chunks;                      // server chunks per tensor (the context's W, whatever W below is)
     const float *g[OB_MAX_WORKERS];  // element i of worker w at g[w][i - g_offset]
     int64_t g_offset;
     float *x;                        // [W][n_pad]: in x_prev (lazy e_w), out x
@@ -26,21 +28,29 @@ struct PackParams {
     int64_t n_pad;
     int W, T;
     float beta1, c1;
+    ScaleEpilogue scales;            // worker scales: ranges = tensors, one row per worker,
+                                     // out_prev = s_prev (read above, rewritten last)
 };
 
 // [1BA, Proposed method, 3; Abstract]: for every worker w of one tile,
 //   m_w = beta1 m + (1-beta1) g_w,  x = m_w + e_w (e_w decoded from the
-//   stored (x_prev, s_prev)), sign bits of x, partial sum of x^2.
-// x overwrites x_prev: with this step's scale it encodes the new e_w.
+//   stored (x_prev, s_prev)), sign bits of x, partial sum of x^2; the CTAs
+//   that finish a tensor's last tiles then form its scales
+//   s_w = ||x||_2 / sqrt(n_t) (finish_scales).
+// x overwrites x_prev: with this step's scale it encodes the new e_w.  The
+// scale s_prev[w][t] is rewritten only after every tile of tensor t has
+// arrived, so every CTA has read the old one by then.
 // m stays in registers across the W workers, so it is read once.  After a
 // compressed step m is exactly last step's decoded server momentum
 // sign' s'_j, so it is rebuilt from the server words (1/8 byte per
 // parameter) instead of read as fp32 (4 bytes).
 __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant__ PackParams P) {
     const int tile_id = P.tile_base + (int)blockIdx.x;
-    const Tile tile = P.tiles[tile_id];
+    const Tile tile = P.tiles[tile_id];  // the work list is written once, at create
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     __shared__ double red[kWarps][OB_MAX_WORKERS];
+    grid_dependency_wait();
+    allow_dependent_launch();
 
     float4 mv[kUnroll];
     int real[kUnroll];
@@ -52,7 +62,7 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
             mv[u] = real[u] > 0 ? ld_stream(P.m + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
     } else {
-        const uint32_t sb = __float_as_uint(P.m_scale[tile.tensor * P.W + tile.chunk]);
+        const uint32_t sb = __float_as_uint(P.m_scale[tile.tensor * P.chunks + tile.chunk]);
         const int shift = 4 * (lane & 7);
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
@@ -141,6 +151,7 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
         for (int k = 0; k < kWarps; ++k) acc += red[k][tid];
         P.partial[(int64_t)tid * P.n_tiles + tile_id] = acc;
     }
+    finish_scales(P.scales, P.partial, P.n_tiles, P.W, tile.tensor, tile_id);
 }
 
 }  // namespace onebit

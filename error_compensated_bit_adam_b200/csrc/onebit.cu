@@ -173,7 +173,8 @@ ob_status make_plan(int n_tensors, const int64_t *numel, int W, bool with_tiles,
 struct Carve {
     size_t m, v, x, y, bits, sbits, s_prev, s_last, sp_prev, sp_last, partial_w, partial_s,
         counters_w, counters_s, seg_w, seg_s, tiles, tensor_tile_begin, chunk_tile_begin, numel,
-        chunk_len, tensor_seg_base, chunk_seg_base, stage, total;
+        chunk_len, tensor_seg_base, chunk_seg_base, stage, ratio, pnorm, dnorm, partial_lamb,
+        seg_lamb, total;
 };
 
 Carve carve(const Plan &pl) {
@@ -198,8 +199,10 @@ Carve carve(const Plan &pl) {
     c.sp_last = take(T * W * 4);
     c.partial_w = take(W * nt * 8);
     c.partial_s = take(nt * 8);
-    c.counters_w = take(T * W * 4);
-    c.counters_s = take(T * W * 4);
+    // scale reductions: arrivals per segment slot, then finished segments
+    // per range (tensors for the workers, chunks for the servers)
+    c.counters_w = take(((size_t)pl.tensor_segs + T) * 4);
+    c.counters_s = take(((size_t)pl.chunk_segs + T * W) * 4);
     c.seg_w = take((size_t)pl.tensor_segs * W * 8);
     c.seg_s = take((size_t)pl.chunk_segs * 8);
     c.tiles = take(nt * sizeof(Tile));
@@ -210,6 +213,13 @@ Carve carve(const Plan &pl) {
     c.tensor_seg_base = take(T * 4);
     c.chunk_seg_base = take(T * W * 4);
     c.stage = take((size_t)kDecodeStage * 4);
+    // 1-bit LAMB: trust ratios, ||p||^2 per tensor, D_j per chunk, and the
+    // two-row reduction of the warmup's norms
+    c.ratio = take(T * 4);
+    c.pnorm = take(T * 8);
+    c.dnorm = take(T * W * 8);
+    c.partial_lamb = take(2 * nt * 8);
+    c.seg_lamb = take(2 * (size_t)pl.tensor_segs * 8);
     c.total = off;
     return c;
 }
@@ -272,11 +282,13 @@ const char *const kKernelNames[OB_NUM_KERNELS] = {
 // A compressed step recorded as a CUDA graph (graph mode).
 struct StepGraph {
     bool built = false;
+    bool lamb = false;           // built with the 1-bit LAMB update
     cudaGraph_t graph = nullptr;
     cudaGraphExec_t exec = nullptr;
     cudaGraphNode_t pack_node = nullptr, apply_node = nullptr;
     onebit::PackParams pack{};   // parameters last written into the nodes
     onebit::ApplyParams apply{};
+    onebit::LambApplyParams lamb_apply{};
 };
 
 struct ob_ctx {
@@ -300,6 +312,10 @@ struct ob_ctx {
     bool m_dense = true;
     bool use_graph = false;
     StepGraph graph;
+    // 1-bit LAMB (ob_set_layerwise): layerwise trust ratios; the norms the
+    // compressed update needs are valid unless p or d changed otherwise
+    bool lamb = false;
+    bool pnorm_valid = false, dnorm_valid = false;
     bool broken = false;
     // split step: 0 idle, 1 after ob_worker_stage, 2 after ob_server_stage
     int split_stage = 0;
@@ -339,6 +355,11 @@ struct ob_ctx {
     int *tensor_seg_base() const { return at<int>(cv.tensor_seg_base); }
     int *chunk_seg_base() const { return at<int>(cv.chunk_seg_base); }
     float *stage() const { return at<float>(cv.stage); }
+    float *ratio() const { return at<float>(cv.ratio); }
+    double *pnorm() const { return at<double>(cv.pnorm); }
+    double *dnorm() const { return at<double>(cv.dnorm); }
+    double *partial_lamb() const { return at<double>(cv.partial_lamb); }
+    double *seg_lamb() const { return at<double>(cv.seg_lamb); }
     int n_tiles() const { return (int)plan.tiles.size(); }
 };
 
@@ -411,9 +432,59 @@ dim3 grid1(int n) { return dim3((unsigned)n); }
 
 // ---------------------------------------------------------------- launches
 //
-// The five kernels of a compressed step, each with its parameters built by
+// The three kernels of a compressed step, each with its parameters built by
 // one function, so direct launches and the CUDA-graph nodes of graph mode
 // are the same launches.
+
+// Worker scales, finished by the worker-stage kernel: ranges = tensors,
+// one row per worker, scale (t, w) at s_prev[w * T + t].
+// Reductions over tensors (the worker stage's; also the LAMB norms, in
+// other kernels) and over server chunks (the server stage's).
+onebit::RangeSums tensor_sums(const ob_ctx *c) {
+    onebit::RangeSums E{};
+    E.range_begin = c->tensor_tile_begin();
+    E.seg_base = c->tensor_seg_base();
+    E.seg_counter = c->counters_w();
+    E.range_counter = c->counters_w() + c->plan.tensor_segs;
+    E.seg = c->seg_w();
+    E.seg_stride = c->plan.tensor_segs;
+    return E;
+}
+
+onebit::RangeSums chunk_sums(const ob_ctx *c) {
+    onebit::RangeSums E{};
+    E.range_begin = c->chunk_tile_begin();
+    E.seg_base = c->chunk_seg_base();
+    E.seg_counter = c->counters_s();
+    E.range_counter = c->counters_s() + c->plan.chunk_segs;
+    E.seg = c->seg_s();
+    E.seg_stride = c->plan.chunk_segs;
+    return E;
+}
+
+onebit::ScaleEpilogue worker_scale_epilogue(const ob_ctx *c) {
+    onebit::ScaleEpilogue E{};
+    E.sums = tensor_sums(c);
+    E.count = c->numel();
+    E.out_prev = c->s_prev();
+    E.out_last = c->s_last();
+    E.out_stride_r = 1;
+    E.out_stride_row = c->plan.T;
+    return E;
+}
+
+// Server scales, finished by the server-stage kernel: ranges = (tensor,
+// chunk) at t * W + j, one row, scale at sp_prev[t * W + j].
+onebit::ScaleEpilogue server_scale_epilogue(const ob_ctx *c) {
+    onebit::ScaleEpilogue E{};
+    E.sums = chunk_sums(c);
+    E.count = c->chunk_len();
+    E.out_prev = c->sp_prev();
+    E.out_last = c->sp_last();
+    E.out_stride_r = 1;
+    E.out_stride_row = 0;
+    return E;
+}
 
 onebit::PackParams pack_params(const ob_ctx *c, const float *const *g, int64_t g_offset,
                                int tile_lo) {
@@ -425,6 +496,7 @@ onebit::PackParams pack_params(const ob_ctx *c, const float *const *g, int64_t g
     P.m_bits = c->sbits();
     P.m_scale = c->sp_last();
     P.m_dense = c->m_dense ? 1 : 0;
+    P.chunks = c->plan.W;
     for (int w = 0; w < OB_MAX_WORKERS; ++w) P.g[w] = w < c->plan.W ? g[w] : nullptr;
     P.g_offset = g_offset;
     P.x = c->x();
@@ -436,24 +508,7 @@ onebit::PackParams pack_params(const ob_ctx *c, const float *const *g, int64_t g
     P.T = c->plan.T;
     P.beta1 = c->beta1;
     P.c1 = c->c1;
-    return P;
-}
-
-onebit::ScaleParams worker_scale_params(const ob_ctx *c) {
-    onebit::ScaleParams P{};  // zeroed, padding too: compared bytewise in graph mode
-    P.partial = c->partial_w();
-    P.n_tiles = c->n_tiles();
-    P.range_begin = c->tensor_tile_begin();
-    P.seg_base = c->tensor_seg_base();
-    P.count = c->numel();
-    P.seg = c->seg_w();
-    P.counter = c->counters_w();
-    P.out_prev = c->s_prev();
-    P.out_last = c->s_last();
-    P.rows = c->plan.W;
-    P.R = c->plan.T;
-    P.out_stride_r = 1;
-    P.out_stride_row = c->plan.T;
+    P.scales = worker_scale_epilogue(c);
     return P;
 }
 
@@ -472,24 +527,7 @@ onebit::ServerParams server_params(const ob_ctx *c) {
     P.T = c->plan.T;
     P.w_pow2 = (W & (W - 1)) == 0;
     P.inv_w = 1.0f / (float)W;  // exact for a power of two
-    return P;
-}
-
-onebit::ScaleParams server_scale_params(const ob_ctx *c) {
-    onebit::ScaleParams P{};  // zeroed, padding too: compared bytewise in graph mode
-    P.partial = c->partial_s();
-    P.n_tiles = c->n_tiles();
-    P.range_begin = c->chunk_tile_begin();
-    P.seg_base = c->chunk_seg_base();
-    P.count = c->chunk_len();
-    P.seg = c->seg_s();
-    P.counter = c->counters_s();
-    P.out_prev = c->sp_prev();
-    P.out_last = c->sp_last();
-    P.rows = 1;
-    P.R = c->plan.T * c->plan.W;
-    P.out_stride_r = 1;
-    P.out_stride_row = 0;
+    P.scales = server_scale_epilogue(c);
     return P;
 }
 
@@ -506,71 +544,123 @@ onebit::ApplyParams apply_params(const ob_ctx *c) {
     return P;
 }
 
+// The 1-bit LAMB update: apply_params with the layerwise rates, and the
+// new ||p||^2 reduced per tensor (in the worker stage's tensor-range
+// buffers, free once the worker stage is done).
+onebit::LambApplyParams lamb_apply_params(const ob_ctx *c) {
+    onebit::LambApplyParams P{};  // zeroed, padding too: compared bytewise in graph mode
+    P.a = apply_params(c);
+    P.tensor_tile_begin = c->tensor_tile_begin();
+    P.pnorm = c->pnorm();
+    P.dnorm = c->dnorm();
+    P.ratio = c->ratio();
+    P.partial = c->partial_w();
+    P.n_tiles = c->n_tiles();
+    P.sums = tensor_sums(c);
+    return P;
+}
+
 // Launch geometry of each kernel: grid, block, dynamic shared memory.
 struct Geometry {
     dim3 grid, block;
     size_t smem;
 };
 Geometry pack_geometry(int tiles) { return {grid1(tiles), dim3(kThreads), (size_t)onebit::kPackSmemBytes}; }
-Geometry worker_scale_geometry(const ob_ctx *c) {
-    return {dim3((unsigned)c->plan.T, (unsigned)c->plan.W, (unsigned)c->plan.tensor_max_seg),
-            dim3(kScaleThreads), 0};
-}
-Geometry server_geometry(const ob_ctx *c) {
-    return {grid1(c->n_tiles()), dim3(kThreads),
-            (size_t)c->plan.W * onebit::kTileWords * sizeof(uint32_t)};
-}
-Geometry server_scale_geometry(const ob_ctx *c) {
-    return {dim3((unsigned)(c->plan.T * c->plan.W), 1u, (unsigned)c->plan.chunk_max_seg),
-            dim3(kScaleThreads), 0};
+Geometry server_geometry(int tiles, int W) {
+    return {grid1(tiles), dim3(kThreads), (size_t)W * onebit::kTileWords * sizeof(uint32_t)};
 }
 Geometry apply_geometry(const ob_ctx *c) { return {grid1(c->n_tiles()), dim3(kThreads), 0}; }
+
+// One kernel launch on the context's stream, allowed to start while the
+// stream's previous kernel finishes (programmatic dependent launch: every
+// kernel of the step waits for its predecessors' results inside, with
+// grid_dependency_wait, before it reads them).  Returns this launch's own
+// status.
+template <class Params>
+cudaError_t launch(void (*kernel)(Params), const Geometry &G, const Params &P, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = G.grid;
+    cfg.blockDim = G.block;
+    cfg.dynamicSmemBytes = G.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, P);
+}
 
 ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int tile_lo, int tile_hi) {
     if (tile_hi <= tile_lo) return OB_OK;
     const onebit::PackParams P = pack_params(c, g, g_offset, tile_lo);
-    const Geometry G = pack_geometry(tile_hi - tile_lo);
-    onebit::ob_pack_kernel<<<G.grid, G.block, G.smem, c->stream>>>(P);
-    return fail_cuda(c, cudaGetLastError());
+    return fail_cuda(c, launch(onebit::ob_pack_kernel, pack_geometry(tile_hi - tile_lo), P, c->stream));
 }
 
-// Everything of a compressed step after the worker stage's tile kernels.
+// The gather and update (1-bit LAMB's with layerwise rates when on).
+ob_status launch_apply(ob_ctx *c) {
+    if (c->n_tiles() == 0) return OB_OK;
+    KernelTimer k(c, OB_K_APPLY);
+    const cudaError_t e =
+        c->lamb ? launch(onebit::ob_lamb_apply_kernel, apply_geometry(c), lamb_apply_params(c), c->stream)
+                : launch(onebit::ob_apply_kernel, apply_geometry(c), apply_params(c), c->stream);
+    k.stop();
+    return fail_cuda(c, e);
+}
+
+// 1-bit LAMB: recompute D_j (want_d) and ||p||^2 (want_p) from d and p.
+ob_status launch_lamb_norms(ob_ctx *c, bool want_d, bool want_p) {
+    if (!want_d && !want_p) return OB_OK;
+    if (c->n_tiles() > 0) {
+        onebit::LambNormsParams P{};
+        P.tiles = c->tiles();
+        P.tile_base = 0;
+        P.d = c->v();
+        P.p = c->params;
+        P.partial_d = c->partial_s();
+        P.partial_p = c->partial_w();
+        P.n_tiles = c->n_tiles();
+        P.W = c->plan.W;
+        P.chunks = chunk_sums(c);
+        P.tensors = tensor_sums(c);
+        P.dnorm = c->dnorm();
+        P.pnorm = c->pnorm();
+        P.want_d = want_d ? 1 : 0;
+        P.want_p = want_p ? 1 : 0;
+        KernelTimer k(c, OB_K_FREEZE);
+        const cudaError_t e = launch(onebit::ob_lamb_norms_kernel, Geometry{grid1(c->n_tiles()), dim3(kThreads), 0},
+                                     P, c->stream);
+        k.stop();
+        ob_status st = fail_cuda(c, e);
+        if (st != OB_OK) return st;
+    }
+    if (want_d) c->dnorm_valid = true;
+    if (want_p) c->pnorm_valid = true;
+    return OB_OK;
+}
+
+// Before a 1-bit LAMB compressed step: the norms its update reads.
+ob_status ensure_lamb_norms(ob_ctx *c) {
+    if (!c->lamb) return OB_OK;
+    return launch_lamb_norms(c, !c->dnorm_valid, !c->pnorm_valid);
+}
+
+// Everything of a compressed step after the worker stage's tile kernels
+// (which finish the worker scales themselves): the server stage, which
+// finishes the server scales, then the update.
 ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
     const int nt = c->n_tiles();
     pack_timer.stop();
+    if (nt == 0) return OB_OK;
     {
-        KernelTimer k(c, OB_K_PACK_SCALE);
-        const Geometry G = worker_scale_geometry(c);
-        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(worker_scale_params(c));
-        k.stop();
-        ob_status st = fail_cuda(c, cudaGetLastError());
-        if (st != OB_OK) return st;
-    }
-    if (nt > 0) {
         KernelTimer k(c, OB_K_SERVER);
-        const Geometry G = server_geometry(c);
-        onebit::ob_server_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_params(c));
+        const cudaError_t e =
+            launch(onebit::ob_server_kernel, server_geometry(nt, c->plan.W), server_params(c), c->stream);
         k.stop();
-        ob_status st = fail_cuda(c, cudaGetLastError());
+        ob_status st = fail_cuda(c, e);
         if (st != OB_OK) return st;
     }
-    {
-        KernelTimer k(c, OB_K_SERVER_SCALE);
-        const Geometry G = server_scale_geometry(c);
-        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(server_scale_params(c));
-        k.stop();
-        ob_status st = fail_cuda(c, cudaGetLastError());
-        if (st != OB_OK) return st;
-    }
-    if (nt > 0) {
-        KernelTimer k(c, OB_K_APPLY);
-        const Geometry G = apply_geometry(c);
-        onebit::ob_apply_kernel<<<G.grid, G.block, G.smem, c->stream>>>(apply_params(c));
-        k.stop();
-        ob_status st = fail_cuda(c, cudaGetLastError());
-        if (st != OB_OK) return st;
-    }
-    return OB_OK;
+    return launch_apply(c);
 }
 
 // ------------------------------------------------------------- graph mode
@@ -609,14 +699,18 @@ ob_status build_graph(ob_ctx *c, const float *const *g) {
     const int nt = c->n_tiles();
     sg.pack = pack_params(c, g, 0, 0);
     sg.apply = apply_params(c);
-    onebit::ScaleParams ws = worker_scale_params(c), ss = server_scale_params(c);
+    sg.lamb_apply = lamb_apply_params(c);
+    sg.lamb = c->lamb;
     onebit::ServerParams sv = server_params(c);
-    cudaGraphNode_t n_ws, n_sv, n_ss;
-    if (nt > 0) add((void *)onebit::ob_pack_kernel, pack_geometry(nt), &sg.pack, &sg.pack_node);
-    add((void *)onebit::ob_scale_kernel, worker_scale_geometry(c), &ws, &n_ws);
-    if (nt > 0) add((void *)onebit::ob_server_kernel, server_geometry(c), &sv, &n_sv);
-    add((void *)onebit::ob_scale_kernel, server_scale_geometry(c), &ss, &n_ss);
-    if (nt > 0) add((void *)onebit::ob_apply_kernel, apply_geometry(c), &sg.apply, &sg.apply_node);
+    cudaGraphNode_t n_sv;
+    if (nt > 0) {
+        add((void *)onebit::ob_pack_kernel, pack_geometry(nt), &sg.pack, &sg.pack_node);
+        add((void *)onebit::ob_server_kernel, server_geometry(nt, c->plan.W), &sv, &n_sv);
+        if (sg.lamb)
+            add((void *)onebit::ob_lamb_apply_kernel, apply_geometry(c), &sg.lamb_apply, &sg.apply_node);
+        else
+            add((void *)onebit::ob_apply_kernel, apply_geometry(c), &sg.apply, &sg.apply_node);
+    }
     if (e == cudaSuccess) e = cudaGraphInstantiate(&sg.exec, sg.graph, 0);
     if (e != cudaSuccess) {
         destroy_graph(c);
@@ -651,13 +745,24 @@ ob_status graph_step(ob_ctx *c, const float *const *g) {
                 node_params((void *)onebit::ob_pack_kernel, pack_geometry(nt), &sg.pack, args);
             e = cudaGraphExecKernelNodeSetParams(sg.exec, sg.pack_node, &kp);
         }
-        onebit::ApplyParams A = apply_params(c);
-        if (e == cudaSuccess && std::memcmp(&A, &sg.apply, sizeof A) != 0) {
-            sg.apply = A;
-            void *args[1];
-            const cudaKernelNodeParams kp =
-                node_params((void *)onebit::ob_apply_kernel, apply_geometry(c), &sg.apply, args);
-            e = cudaGraphExecKernelNodeSetParams(sg.exec, sg.apply_node, &kp);
+        if (sg.lamb) {
+            onebit::LambApplyParams A = lamb_apply_params(c);
+            if (e == cudaSuccess && std::memcmp(&A, &sg.lamb_apply, sizeof A) != 0) {
+                sg.lamb_apply = A;
+                void *args[1];
+                const cudaKernelNodeParams kp = node_params((void *)onebit::ob_lamb_apply_kernel,
+                                                            apply_geometry(c), &sg.lamb_apply, args);
+                e = cudaGraphExecKernelNodeSetParams(sg.exec, sg.apply_node, &kp);
+            }
+        } else {
+            onebit::ApplyParams A = apply_params(c);
+            if (e == cudaSuccess && std::memcmp(&A, &sg.apply, sizeof A) != 0) {
+                sg.apply = A;
+                void *args[1];
+                const cudaKernelNodeParams kp =
+                    node_params((void *)onebit::ob_apply_kernel, apply_geometry(c), &sg.apply, args);
+                e = cudaGraphExecKernelNodeSetParams(sg.exec, sg.apply_node, &kp);
+            }
         }
     }
     if (e == cudaSuccess) e = cudaGraphLaunch(sg.exec, c->stream);
@@ -686,6 +791,8 @@ size_t state_bytes(const ob_ctx *c, int kind) {
         return (n / 32) * 4;
     case OB_STATE_STEP:
         return 3 * sizeof(int64_t);
+    case OB_STATE_RATIO:
+        return T * 4;
     default:
         return 0;
     }
@@ -990,12 +1097,33 @@ ob_status ob_warmup_adam_step(ob_ctx *c, const float *const *d_grads) {
     P.bc2 = (float)(1.0 - std::pow((double)c->beta2, (double)t));
     P.eps = c->eps;
     P.lr = c->lr;
-    if (c->n_tiles() > 0) {
+    if (c->n_tiles() > 0 && !c->lamb) {
         KernelTimer k(c, OB_K_WARMUP);
         onebit::ob_warmup_kernel<<<grid1(c->n_tiles()), kThreads, 0, c->stream>>>(P);
         k.stop();
         if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
     }
+    if (c->n_tiles() > 0 && c->lamb) {
+        // 1-bit LAMB's warmup: the moments and each tensor's trust ratio,
+        // then the step with the layerwise rates
+        onebit::LambWarmupParams L{};
+        L.w = P;
+        L.partial = c->partial_lamb();
+        L.n_tiles = c->n_tiles();
+        L.sums = tensor_sums(c);
+        L.sums.seg = c->seg_lamb();
+        L.ratio = c->ratio();
+        KernelTimer k(c, OB_K_WARMUP);
+        onebit::ob_lamb_moments_kernel<<<grid1(c->n_tiles()), kThreads, 0, c->stream>>>(L);
+        cudaError_t e = cudaGetLastError();
+        if (e == cudaSuccess) {
+            onebit::ob_lamb_step_kernel<<<grid1(c->n_tiles()), kThreads, 0, c->stream>>>(L);
+            e = cudaGetLastError();
+        }
+        k.stop();
+        if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    }
+    c->pnorm_valid = false;
     c->t_warmup = t;
     return OB_OK;
 }
@@ -1022,6 +1150,8 @@ ob_status ob_freeze_variance(ob_ctx *c) {
     if (e == cudaSuccess) e = cudaMemsetAsync(c->bits(), 0, cv.partial_w - cv.bits, c->stream);
     if ((st = fail_cuda(c, e)) != OB_OK) return st;
     c->frozen = true;
+    c->dnorm_valid = false;
+    if (c->lamb && (st = launch_lamb_norms(c, true, true)) != OB_OK) return st;
     return OB_OK;
 }
 
@@ -1033,6 +1163,7 @@ ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
     if ((st = check_grads(c, d_grads)) != OB_OK) return st;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    if ((st = ensure_lamb_norms(c)) != OB_OK) return st;
     if (c->use_graph && !c->profiling) {
         if ((st = graph_step(c, d_grads)) != OB_OK) return st;
     } else {
@@ -1066,13 +1197,12 @@ ob_status ob_worker_stage(ob_ctx *c, const float *const *d_grads, int w_begin, i
         }
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
-    // The worker stage's lazy momentum decode reads the server scale of
-    // (tensor t, chunk j) at t * W + j with W the launch's worker count,
-    // which the view changes; with one tensor that index is j whatever W
-    // is, otherwise the momentum is decoded densely first.
-    if (c->plan.T > 1 && (st = materialize_momentum(c)) != OB_OK) return st;
+    if ((st = ensure_lamb_norms(c)) != OB_OK) return st;
     const size_t n = (size_t)c->plan.n_pad, T = (size_t)c->plan.T, nt = (size_t)c->n_tiles();
     if (w_count > 0 && nt > 0) {
+        // the step's worker-stage kernel on a view of the worker rows: the
+        // rows [w_begin, w_begin + w_count) of x, bits, the scales, the
+        // partial sums and the segment sums, as if they were all workers
         onebit::PackParams P = pack_params(c, d_grads, 0, 0);
         for (int i = 0; i < OB_MAX_WORKERS; ++i) P.g[i] = i < w_count ? d_grads[w_begin + i] : nullptr;
         P.x = c->x() + (size_t)w_begin * n;
@@ -1080,23 +1210,13 @@ ob_status ob_worker_stage(ob_ctx *c, const float *const *d_grads, int w_begin, i
         P.s_prev = c->s_prev() + (size_t)w_begin * T;
         P.partial = c->partial_w() + (size_t)w_begin * nt;
         P.W = w_count;
+        P.scales.sums.seg = c->seg_w() + (size_t)w_begin * c->plan.tensor_segs;
+        P.scales.out_prev = c->s_prev() + (size_t)w_begin * T;
+        P.scales.out_last = c->s_last() + (size_t)w_begin * T;
         KernelTimer k(c, OB_K_PACK);
-        const Geometry G = pack_geometry((int)nt);
-        onebit::ob_pack_kernel<<<G.grid, G.block, G.smem, c->stream>>>(P);
+        const cudaError_t e = launch(onebit::ob_pack_kernel, pack_geometry((int)nt), P, c->stream);
         k.stop();
-        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
-    }
-    if (w_count > 0) {
-        onebit::ScaleParams S = worker_scale_params(c);
-        S.partial = c->partial_w() + (size_t)w_begin * nt;
-        S.out_prev = c->s_prev() + (size_t)w_begin * T;
-        S.out_last = c->s_last() + (size_t)w_begin * T;
-        S.rows = w_count;
-        KernelTimer k(c, OB_K_PACK_SCALE);
-        const dim3 grid((unsigned)T, (unsigned)w_count, (unsigned)c->plan.tensor_max_seg);
-        onebit::ob_scale_kernel<<<grid, dim3(kScaleThreads), 0, c->stream>>>(S);
-        k.stop();
-        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
+        if ((st = fail_cuda(c, e)) != OB_OK) return st;
     }
     c->split_stage = 1;
     return OB_OK;
@@ -1156,36 +1276,18 @@ ob_status ob_server_stage(ob_ctx *c) {
     cudaError_t e = cudaMemcpyAsync(c->s_last(), c->s_prev(), (size_t)pl.W * pl.T * 4,
                                     cudaMemcpyDeviceToDevice, c->stream);
     if ((st = fail_cuda(c, e)) != OB_OK) return st;
-    // The server stage and its scales on the served chunks only: the
-    // kernels index their tiles and chunks from the pointers they are
-    // given, so a contiguous range is launched through offset pointers.
+    // The server stage (which finishes its chunks' scales) on the served
+    // chunks only: their tiles are one contiguous range of the work list,
+    // launched from its first tile.  Empty served chunks have no tile and
+    // keep their scale, 0.
     const int t_lo = pl.chunk_tile_begin[lo], t_hi = pl.chunk_tile_begin[hi];
     if (t_hi > t_lo) {
         onebit::ServerParams P = server_params(c);
-        P.tiles = c->tiles() + t_lo;
-        P.partial = c->partial_s() + t_lo;
-        Geometry G = server_geometry(c);
-        G.grid = grid1(t_hi - t_lo);
+        P.tile_base = t_lo;
         KernelTimer k(c, OB_K_SERVER);
-        onebit::ob_server_kernel<<<G.grid, G.block, G.smem, c->stream>>>(P);
+        e = launch(onebit::ob_server_kernel, server_geometry(t_hi - t_lo, pl.W), P, c->stream);
         k.stop();
-        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
-    }
-    if (hi > lo) {
-        onebit::ScaleParams S = server_scale_params(c);
-        S.range_begin = c->chunk_tile_begin() + lo;
-        S.seg_base = c->chunk_seg_base() + lo;
-        S.count = c->chunk_len() + lo;
-        S.counter = c->counters_s() + lo;  // one row
-        S.out_prev = c->sp_prev() + lo;
-        S.out_last = c->sp_last() + lo;
-        S.R = hi - lo;
-        Geometry G = server_scale_geometry(c);
-        G.grid.x = (unsigned)(hi - lo);
-        KernelTimer k(c, OB_K_SERVER_SCALE);
-        onebit::ob_scale_kernel<<<G.grid, G.block, G.smem, c->stream>>>(S);
-        k.stop();
-        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
+        if ((st = fail_cuda(c, e)) != OB_OK) return st;
     }
     // The words and scales of the chunks served elsewhere are zero here, so
     // that summing every process's buffers gives every chunk its server's.
@@ -1226,16 +1328,32 @@ ob_status ob_apply_update(ob_ctx *c) {
     cudaError_t e = cudaMemcpyAsync(c->sp_prev(), c->sp_last(), (size_t)c->plan.T * c->plan.W * 4,
                                     cudaMemcpyDeviceToDevice, c->stream);
     if ((st = fail_cuda(c, e)) != OB_OK) return st;
-    if (c->n_tiles() > 0) {
-        KernelTimer k(c, OB_K_APPLY);
-        const Geometry G = apply_geometry(c);
-        onebit::ob_apply_kernel<<<G.grid, G.block, G.smem, c->stream>>>(apply_params(c));
-        k.stop();
-        if ((st = fail_cuda(c, cudaGetLastError())) != OB_OK) return st;
-    }
+    if ((st = launch_apply(c)) != OB_OK) return st;
     c->split_stage = 0;
     c->m_dense = false;
     c->t_compressed += 1;
+    return OB_OK;
+}
+
+ob_status ob_set_layerwise(ob_ctx *c, int on) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (c->t_warmup != 0 || c->t_compressed != 0 || c->frozen || c->split_stage != 0)
+        return OB_ERR_PHASE;
+    DeviceGuard dg(c->device);
+    if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    try {
+        host_alloc_point();
+        const std::vector<float> ones((size_t)c->plan.T, 1.0f);  // empty tensors keep ratio 1
+        cudaError_t e = cudaMemcpyAsync(c->ratio(), ones.data(), ones.size() * 4,
+                                        cudaMemcpyHostToDevice, c->stream);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(c->stream);
+        if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    } catch (const std::bad_alloc &) {
+        return OB_ERR_OOM;
+    }
+    c->lamb = on != 0;
+    c->pnorm_valid = c->dnorm_valid = false;
     return OB_OK;
 }
 
@@ -1276,6 +1394,7 @@ ob_status ob_compressed_step_host(ob_ctx *c, const float *const *h_grads, void *
     if (staging_bytes < (size_t)2 * W * kHostSlice * sizeof(float)) return OB_ERR_WORKSPACE;
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
+    if ((st = ensure_lamb_norms(c)) != OB_OK) return st;
     float *stage = static_cast<float *>(d_staging);
     // The copy stream must not overwrite staging still read by earlier work.
     cudaError_t e = cudaEventRecord(c->ev_start, c->stream);
@@ -1352,6 +1471,7 @@ ob_status ob_read_state(ob_ctx *c, int kind, int index, void *host_dst, size_t b
     case OB_STATE_S_SERVER: src = c->sp_last(); break;
     case OB_STATE_BITS_WORKER: src = c->bits() + (size_t)index * (n / 32); break;
     case OB_STATE_BITS_SERVER: src = c->sbits(); break;
+    case OB_STATE_RATIO: src = c->ratio(); break;
     default: return OB_ERR_INVALID_ARG;
     }
     cudaError_t e = cudaMemcpyAsync(host_dst, src, bytes, cudaMemcpyDeviceToHost, c->stream);
@@ -1387,9 +1507,10 @@ ob_status ob_write_state(ob_ctx *c, int kind, int index, const void *host_src, s
     void *dst = nullptr;
     cudaError_t e = cudaSuccess;
     switch (kind) {
-    case OB_STATE_P: dst = c->params; break;
+    case OB_STATE_P: dst = c->params; c->pnorm_valid = false; break;
     case OB_STATE_M: dst = c->m(); c->m_dense = true; break;
-    case OB_STATE_V: case OB_STATE_D: dst = c->v(); break;
+    case OB_STATE_V: dst = c->v(); break;
+    case OB_STATE_D: dst = c->v(); c->dnorm_valid = false; break;
     case OB_STATE_E_WORKER:
         // stored as (x, s) with s = 0, which decodes to x exactly
         dst = c->x() + (size_t)index * n;

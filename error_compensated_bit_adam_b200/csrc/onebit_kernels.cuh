@@ -2,17 +2,19 @@
 //
 // The compression-phase step of 1-bit Adam ("1-bit Adam: Communication
 // Efficient Large-Scale Training with Adam's Convergence Speed", review
-// page, sections "Abstract" and "Proposed method") as five HBM-streaming
-// kernels over a list of 4096-element tiles:
+// page, sections "Abstract" and "Proposed method") as three HBM-streaming
+// kernels over a list of 4096-element tiles, each launched so that it may
+// start while the one before it finishes (programmatic dependent launch):
 //
-//   ob_pack_kernel          worker stage, all W workers of a tile per CTA
-//   ob_scale_kernel         worker scales per (tensor, worker)
-//   ob_server_kernel        server stage of a tile
-//   ob_scale_kernel         server scales per (tensor, chunk)
+//   ob_pack_kernel          worker stage, all W workers of a tile per CTA;
+//                           its last CTAs per tensor finish the worker scales
+//   ob_server_kernel        server stage of a tile; its last CTAs per chunk
+//                           finish the server scales
 //   ob_apply_kernel         gather, decode, preconditioned update
 //
 // plus the warmup Adam step, the freeze and an error decoder used when the
-// host reads state.  No step is a dense contraction, so no tensor cores:
+// host reads state, and the 1-bit LAMB variants (kernels/lamb.cuh: the
+// warmup in two passes, the norms, the update with layerwise rates).  No step is a dense contraction, so no tensor cores:
 // every kernel is a stream of coalesced 16-byte loads and stores, bound by
 // HBM bandwidth.
 //
@@ -37,5 +39,6 @@
 #include "kernels/scale.cuh"
 #include "kernels/server.cuh"
 #include "kernels/apply.cuh"
+#include "kernels/lamb.cuh"
 #include "kernels/state.cuh"
 #include "kernels/compress_static.cuh"

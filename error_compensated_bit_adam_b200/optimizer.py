@@ -17,7 +17,7 @@ _STATE_DTYPE = {
     B.OB_STATE_D: np.float32, B.OB_STATE_E_WORKER: np.float32, B.OB_STATE_E_SERVER: np.float32,
     B.OB_STATE_S_WORKER: np.float32, B.OB_STATE_S_SERVER: np.float32,
     B.OB_STATE_BITS_WORKER: np.uint32, B.OB_STATE_BITS_SERVER: np.uint32,
-    B.OB_STATE_STEP: np.int64,
+    B.OB_STATE_STEP: np.int64, B.OB_STATE_RATIO: np.float32,
 }
 
 Grads = Union[torch.Tensor, Sequence[torch.Tensor]]
@@ -30,12 +30,14 @@ class OneBitAdam:
     n_padded elements in the padded layout (see ``layout``), updated in
     place; a zero tensor is made if omitted.  Gradients are passed as a
     [W, n_padded] float32 CUDA tensor or a list of W such vectors.
+    layerwise=True runs 1-bit LAMB instead (ob_set_layerwise): every
+    tensor's step scaled by its trust ratio ||p|| / ||u||.
     """
 
     def __init__(self, numel: Sequence[int], W: int, *, beta1: float = 0.9, beta2: float = 0.999,
                  eps: float = 1e-8, lr: float = 1e-4, params: Optional[torch.Tensor] = None,
                  device: Union[str, torch.device, None] = None,
-                 stream: Optional[torch.cuda.Stream] = None):
+                 stream: Optional[torch.cuda.Stream] = None, layerwise: bool = False):
         self.numel = [int(n) for n in numel]
         self.W = int(W)
         self.offsets, self.n_padded = B.ob_layout(self.numel)
@@ -52,18 +54,38 @@ class OneBitAdam:
         self.workspace = torch.empty(self.workspace_bytes, dtype=torch.uint8, device=self.device)
         self.stream = stream if stream is not None else torch.cuda.current_stream(self.device)
         self._staging: Optional[torch.Tensor] = None
+        self._ptr_cache = {}
         self.ctx = 0
         with torch.cuda.device(self.device):
             self.ctx = B.ob_create(self.numel, self.W, beta1, beta2, eps, lr, params.data_ptr(),
                                    self.workspace.data_ptr(), self.workspace_bytes,
                                    self.stream.cuda_stream)
+            if layerwise:
+                B.ob_set_layerwise(self.ctx, True)
 
     # ------------------------------------------------------------ helpers
     def layout(self):
         return self.offsets, self.n_padded
 
-    def _ptrs(self, grads: Grads) -> List[int]:
-        rows = [grads[w] for w in range(self.W)] if isinstance(grads, torch.Tensor) else list(grads)
+    def _ptrs(self, grads: Grads):
+        """The W gradient pointers as a C array.  A [W, n_padded] tensor is
+        checked once and its rows' addresses computed from its base; the
+        array is kept per base address, so stepping on the same gradient
+        buffers again costs no marshalling."""
+        if isinstance(grads, torch.Tensor):
+            if (grads.dtype != torch.float32 or not grads.is_cuda or not grads.is_contiguous()
+                    or tuple(grads.shape) != (self.W, self.n_padded)):
+                raise ValueError(f"gradients must be a contiguous float32 CUDA tensor of shape "
+                                 f"({self.W}, {self.n_padded}) or a list of {self.W} vectors")
+            base = grads.data_ptr()
+            arr = self._ptr_cache.get(base)
+            if arr is None:
+                if len(self._ptr_cache) >= 8:
+                    self._ptr_cache.clear()
+                row = self.n_padded * 4
+                arr = self._ptr_cache[base] = B.pointer_array([base + w * row for w in range(self.W)])
+            return arr
+        rows = list(grads)
         if len(rows) != self.W:
             raise ValueError(f"expected {self.W} gradients")
         for g in rows:
@@ -110,6 +132,8 @@ class OneBitAdam:
             return (n // 32,)
         if kind == B.OB_STATE_STEP:
             return (3,)
+        if kind == B.OB_STATE_RATIO:
+            return (T,)
         return (n,)
 
     def read(self, kind: int, index: int = 0) -> np.ndarray:

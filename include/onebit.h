@@ -93,17 +93,20 @@ typedef enum ob_state_kind {
     OB_STATE_S_SERVER = 7,    /* last step's server chunk scales, float[n_tensors][W]           r  */
     OB_STATE_BITS_WORKER = 8, /* index w: last step's packed worker signs, uint32[n_padded/32]  r  */
     OB_STATE_BITS_SERVER = 9, /* last step's packed server signs, uint32[n_padded/32]           r  */
-    OB_STATE_STEP = 10        /* int64[3]: {warmup steps taken, compressed steps taken, frozen} rw */
+    OB_STATE_STEP = 10,       /* int64[3]: {warmup steps taken, compressed steps taken, frozen} rw */
+    OB_STATE_RATIO = 11       /* last step's 1-bit LAMB trust ratios, float[n_tensors] (1 while
+                                 layerwise rates are off, before the first step, for empty
+                                 tensors)                                                       r  */
 } ob_state_kind;
 
 /* Kernels timed by the profiling counters (ob_profile_read). */
 typedef enum ob_kernel_id {
     OB_K_WARMUP = 0,          /* ob_warmup_adam_step */
     OB_K_FREEZE = 1,          /* ob_freeze_variance */
-    OB_K_PACK = 2,            /* worker stage: momentum, error, signs, partial sums of squares */
-    OB_K_PACK_SCALE = 3,      /* worker scales from the partial sums (ob_scale_kernel) */
-    OB_K_SERVER = 4,          /* server stage: average, server error, signs, partial sums */
-    OB_K_SERVER_SCALE = 5,    /* server chunk scales from the partial sums (ob_scale_kernel) */
+    OB_K_PACK = 2,            /* worker stage: momentum, error, signs and the worker scales */
+    OB_K_PACK_SCALE = 3,      /* no longer launched: the worker stage finishes its scales (0 launches) */
+    OB_K_SERVER = 4,          /* server stage: average, server error, signs and the chunk scales */
+    OB_K_SERVER_SCALE = 5,    /* no longer launched: the server stage finishes its scales (0 launches) */
     OB_K_APPLY = 6,           /* gather, decode and preconditioned update */
     OB_NUM_KERNELS = 7
 } ob_kernel_id;
@@ -297,13 +300,31 @@ OB_API ob_status ob_read_state(ob_ctx *ctx, int kind, int index, void *host_dst,
  * Waits for the copy to finish. */
 OB_API ob_status ob_write_state(ob_ctx *ctx, int kind, int index, const void *host_src, size_t bytes);
 
+/* 1-bit LAMB: layerwise adaptive learning rates on (on != 0) or off (the
+ * default, 1-bit Adam).  The 1-bit LAMB review page ("1-bit LAMB:
+ * Communication Efficient Large-Scale Large-Batch Training with LAMB's
+ * Convergence Speed", Abstract) keeps LAMB's layerwise rates while the
+ * momentum is exchanged compressed; it prints no update rule, and the
+ * reading taken is LAMB's trust ratio per tensor,
+ *   ratio_t = ||p_t|| / ||u_t||   (1 when either norm is 0),
+ * recomputed every step, scaling that tensor's step: p -= (lr ratio_t) u.
+ * In the warmup u is Adam's direction m_hat / (sqrt(v_hat) + eps); in the
+ * compression phase u = m_hat / d, m_hat the momentum decoded from the
+ * compressed exchange (the same on every worker) and d the frozen
+ * denominator.  Everything else (the compressed exchange, the errors, the
+ * freeze) is 1-bit Adam's.  The trust ratios are read as OB_STATE_RATIO.
+ * Only before the first step: OB_ERR_PHASE afterwards.  The ratios are
+ * rounded from fp64 sums of squares taken in an order of the GPU's own, so
+ * they can differ from a sequential evaluation in the last place. */
+OB_API ob_status ob_set_layerwise(ob_ctx *ctx, int on);
+
 /* Set the learning rate used by the following warmup and compressed steps
  * (learning-rate schedules).  OB_ERR_INVALID_ARG for a non-finite lr. */
 OB_API ob_status ob_set_lr(ob_ctx *ctx, float lr);
 
 /* Graph mode on or off (default off).  While on (and profiling is off),
- * ob_compressed_step replays the step's five kernels as one CUDA graph,
- * built at the first such call: one launch instead of five, which matters
+ * ob_compressed_step replays the step's three kernels as one CUDA graph,
+ * built at the first such call: one launch instead of three, which matters
  * for small tensor lists where each kernel runs a few microseconds.
  * Changed gradient pointers, the dense/lazy state of m and the learning
  * rate are written into the graph before each replay; the results are
