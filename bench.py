@@ -11,8 +11,12 @@ BERT-Large-sized flat fp32 vector, n = 335,544,320, W = 8 simulated
 workers, after 100 full-precision Adam warmup steps and the freeze.
 
 Prints one JSON line (rank 0).  value = parameters updated per second per
-simulated worker, summed over the N GPUs (each GPU runs an independent
-replica: the method's exchange lives inside one GPU's HBM).
+worker.  With one GPU all W workers are simulated in its HBM and the
+exchange is addressing inside it.  With N > 1 GPUs (torchrun, one process
+per GPU) the W workers are spread over the GPUs, W/N each, and every step
+runs the split step with its per-chunk NCCL exchange between them (value =
+n / the slowest rank's step time, "strong" scaling); --multi replicas runs
+N independent one-GPU steps instead ("weak").
 
 --impl reference times the CPU oracle (single-threaded C) on a bounded
 sample of the same workload instead.
@@ -454,6 +458,127 @@ def measure_overlap(wl, args, dev, world) -> dict:
             "hidden_fraction_of_shorter": (t_b + t_s - t_o) / min(t_b, t_s)}
 
 
+def run_split(args, world: int, rank: int, dev) -> None:
+    """The workload's W workers spread over the `world` processes, one per
+    GPU, through the split step (distributed.DistributedOneBitAdam): each
+    process runs the worker stage of its W/world workers, exchanges chunks
+    of the worker words with the others (NCCL point-to-point), serves its
+    share of the server chunks, exchanges the server words and scales, and
+    updates.  The whole job updates n parameters per step for each of the
+    W workers, so value = n / step time (the slowest rank's), the total
+    work fixed as the GPUs grow ("strong")."""
+    from error_compensated_bit_adam_b200.distributed import DistributedOneBitAdam
+
+    wl = pick_workload(args)
+    if wl.W % world:
+        raise SystemExit(f"W = {wl.W} workers do not split over {world} GPUs")
+    offsets, n_pad = B.ob_layout(wl.numels)
+    params = WL.make_params(wl, offsets, n_pad, device=dev)
+    scale = WL.grad_scale_vector(wl, offsets, n_pad, device=dev)
+    D = DistributedOneBitAdam(wl.numels, wl.W, rank=rank, world=world, device=dev, **WL.HYPER)
+    D.params.copy_(params)
+    del params
+    wl_local, w0 = D.w_local, D.w_begin
+    full = torch.empty((wl.W, n_pad), dtype=torch.float32, device=dev)
+    step = 0
+    D.opt.profile(True)
+    for _ in range(wl.warmup_steps):           # Adam on all-reduced gradients, outside the step
+        WL.fill_grads(wl, step, scale, full)
+        step += 1
+        D.warmup_step_allreduce([full[w0 + i] for i in range(wl_local)])
+    D.freeze()
+    pre_prof = D.opt.profile_read(reset=True)
+    D.opt.profile(False)
+    grads = []
+    for _ in range(GRAD_SETS):                 # this process's workers' rows of fresh draws
+        WL.fill_grads(wl, step, scale, full)
+        step += 1
+        grads.append(full[w0:w0 + wl_local].clone())
+    del full, scale
+    local_rows = [[g[i] for i in range(wl_local)] for g in grads]
+    for k in range(args.warmup):
+        D.step(local_rows[k % len(grads)])
+    torch.cuda.synchronize(dev)
+
+    stream = D.opt.stream
+    D.opt.profile(True)
+    D.opt.profile_read(reset=True)
+    sampler = ClockSampler()
+    if rank == 0:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        D.step(local_rows[k % len(grads)])
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clocks = sampler.stop() if rank == 0 else None
+    prof = D.opt.profile_read(reset=True)
+    D.opt.profile(False)
+    ms_per_step = max_over_ranks(t0.elapsed_time(t1), world) / args.steps
+    launches = sum(prof[B.ob_kernel_name(k)][1] for k in range(B.OB_K_PACK, B.OB_K_APPLY + 1))
+    launches = int(max_over_ranks(float(launches), world)) * world
+
+    # end to end: every step copies this process's gradients in from pinned
+    # host memory and reads the step's server scales back
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    host = [torch.empty((wl_local, n_pad), dtype=torch.float32, pin_memory=True) for _ in range(1)]
+    host[0].copy_(grads[0])
+    scales_out = torch.empty(D.server_scales.numel(), dtype=torch.float32, pin_memory=True)
+    dev_rows = grads[0]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    w_start = time.perf_counter()
+    for _ in range(e2e_steps):
+        with torch.cuda.stream(stream):
+            dev_rows.copy_(host[0], non_blocking=True)
+        D.step(local_rows[0])
+        with torch.cuda.stream(stream):
+            scales_out.copy_(D.server_scales, non_blocking=True)
+        stream.synchronize()
+    e2e_s = max_over_ranks(time.perf_counter() - w_start, world) / e2e_steps
+    e2e = {"value": wl.n / e2e_s, "unit": UNIT, "h2d_bytes_per_step": int(host[0].numel() * 4 * world),
+           "d2h_bytes_per_step": int(scales_out.numel() * 4 * world), "ms_per_step": e2e_s * 1e3,
+           "steps": e2e_steps, "call": "DistributedOneBitAdam.step after a pinned host copy"}
+
+    peak = measured_peaks()
+    n_real = wl.n
+    pack_bytes = n_real * (1 / 8 + 12 * wl_local + wl_local / 8)
+    pack_ms, pack_n = prof["ob_pack_kernel"]
+    pack_avg_s = pack_ms / 1e3 / max(1, pack_n)
+    achieved = pack_bytes / pack_avg_s / 1e9
+    per_kernel = {name: {"ms_per_step": kms / args.steps, "launches_per_step": cnt / args.steps}
+                  for name, (kms, cnt) in prof.items() if cnt}
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": wl.n / (ms_per_step / 1e3), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": workload_config(wl, n_pad, f"dp{world}: split step, {wl_local} of the W={wl.W} "
+                                                 "workers per GPU, per-chunk NCCL exchange",
+                                      len(grads)),
+            "exchange_bytes_in_per_rank_per_step": D.exchange_bytes(),
+            "roofline": {"bound": "hbm", "kernel": "ob_pack_kernel", "achieved": achieved,
+                         "peak": peak["hbm_gbs"], "peak_source": peak["source"], "unit": "GB/s",
+                         "frac": achieved / peak["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes_per_launch": pack_bytes,
+                         "avg_launch_ms": pack_avg_s * 1e3, "rank": 0},
+            "kernels_rank0": per_kernel,
+            "pre_path_rank0": {k: v for k, v in pre_prof.items() if v[1]},
+            "cpu_baseline": None, "e2e": e2e, "gpu_launches": launches, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    D.close()
+    if world > 1:
+        import torch.distributed as dist
+        barrier(world)
+        dist.destroy_process_group()
+
+
 def run_b200(args) -> None:
     from error_compensated_bit_adam_b200.optimizer import OneBitAdam
 
@@ -469,6 +594,10 @@ def run_b200(args) -> None:
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
+    multi = args.multi or ("split" if world > 1 else "single")
+    if multi == "split":
+        run_split(args, world, rank, dev)
+        return
 
     wl = pick_workload(args)
     offsets, n_pad = B.ob_layout(wl.numels)
@@ -546,9 +675,9 @@ def run_b200(args) -> None:
     achieved = algo["ob_pack_kernel"] / pack_avg_s / 1e9
     step_gbs = algo["step"] / (ms_per_step / 1e3) / 1e9
     model_gbs = algo["model"] / (ms_per_step / 1e3) / 1e9
-    # per kernel, per step (the server stage, its scales and the update run in
-    # chunk groups, the update of one group overlapping the next group's
-    # server stage, so their times can add up to more than the step)
+    # per kernel, per step, from the library's event pairs around each
+    # launch (three kernels in sequence; the worker and server stages finish
+    # their own scales)
     per_kernel = {}
     for name, (kms, cnt) in prof.items():
         if cnt:
@@ -602,7 +731,8 @@ def run_b200(args) -> None:
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(wl, n_pad, "replicas" if world > 1 else "single GPU", n_sets),
+            "config": workload_config(wl, n_pad, f"replicas{world}" if world > 1 else "single GPU",
+                                      n_sets),
             "params_per_s_aggregate_all_workers": value * wl.W,
             "hbm_gbs_step": step_gbs,
             "hbm_frac_of_measured_peak_step": step_gbs / peak["hbm_gbs"],
@@ -646,6 +776,11 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-gradient end-to-end leg")
+    ap.add_argument("--multi", choices=["split", "replicas"], default=None,
+                    help="with --gpus N > 1: 'split' (default) spreads the W workers over the N "
+                         "GPUs through the split step and its NCCL exchange; 'replicas' runs N "
+                         "independent copies of the one-GPU step.  '--multi split' with one GPU "
+                         "runs the split step's calls without an exchange")
     ap.add_argument("--graph", action="store_true",
                     help="also time the steps replayed as one CUDA graph each")
     ap.add_argument("--overlap", action="store_true",

@@ -6,24 +6,29 @@ method", 4) has a worker stage (every worker compresses its momentum and
 sends server j the part of its words that chunk j covers) and a server
 stage (server j averages its chunk, compresses it again and sends the
 result to every worker).  Here process r of G computes workers
-[r W/G, (r+1) W/G) and serves one contiguous range of the server chunks
-(ob_server_shard_range); between the library's three calls
+[r W/G, (r+1) W/G) and serves one contiguous range of the server chunks,
+whose words are one contiguous range [wb_r, we_r) of the padded layout
+(ob_server_shard_range).  Between the library's three calls
 (ob_worker_stage, ob_server_stage, ob_apply_update) the process exchanges
 
-  * the worker rows (sign words and scales) by an all-gather, and
-  * the server words and scales by a sum-all-reduce: every process holds
-    zeros in the chunks it does not serve, so the sums are exact.
+  * chunks of the worker words: process r sends words [wb_q, we_q) of each
+    of its workers' rows to process q and receives words [wb_r, we_r) of
+    every other worker's row (grouped point-to-point sends and receives:
+    about (W - W/G) n / (8 G) bytes in per process), plus an all-gather of
+    the worker scales (W x T floats);
+  * the server results: process r sends its words [wb_r, we_r) and its
+    chunks' scales to every other process and receives theirs (about n/8
+    bytes in per process).
 
-The all-gather sends every worker's whole row to every process, where the
-pages send each server only its chunk: W/G times more bytes, for one
-collective over the library's own layout.  Every process ends the step
-with the same parameters, bit for bit equal to one ob_compressed_step over
-all W workers.
+Every process ends the step with the same parameters, bit for bit equal to
+one ob_compressed_step over all W workers.  A process's rows of the other
+workers hold only the words of the chunks it serves (the rest is stale),
+and its server error only the chunks it serves.
 
 LocalRanks runs the same split step for G ranks inside one process on one
 GPU, each rank a context of its own, with the exchanges done by device
-copies and sums: the single-GPU form of the path, used to check it against
-one context and to time each rank's share of the work.
+copies of the same ranges: the single-GPU form of the path, used to check
+it against one context and to time each rank's share of the work.
 """
 from __future__ import annotations
 
@@ -43,9 +48,9 @@ def _view(workspace: torch.Tensor, ptr: int, nbytes: int, dtype: torch.dtype) ->
 
 
 class TorchExchange:
-    """The split step's two exchanges over a torch.distributed group (NCCL
-    for CUDA tensors, gloo for CPU tensors).  Collectives run on the current
-    stream; every rank calls them in the same order."""
+    """The split step's exchanges over a torch.distributed group (NCCL for
+    CUDA tensors, gloo for CPU tensors).  They run on the current stream;
+    every rank calls them in the same order with the same ranges."""
 
     def __init__(self, group=None):
         import torch.distributed as dist
@@ -53,6 +58,14 @@ class TorchExchange:
         self.group = group
         self.rank = dist.get_rank(group)
         self.world = dist.get_world_size(group)
+
+    def _peer(self, q: int) -> int:
+        return q if self.group is None else self.dist.get_global_rank(self.group, q)
+
+    def _run(self, ops) -> None:
+        if ops:
+            for req in self.dist.batch_isend_irecv(ops):
+                req.wait()
 
     def gather_rows(self, rows: torch.Tensor, begin: int, count: int) -> None:
         """rows: [R, k], rank q's block at rows [q count, (q+1) count); this
@@ -62,8 +75,50 @@ class TorchExchange:
         mine = rows[begin:begin + count].view(-1)
         self.dist.all_gather_into_tensor(flat, mine, group=self.group)
 
+    def send_worker_chunks(self, rows: torch.Tensor, count: int, ranges) -> None:
+        """Worker stage: rows [W, words], rank q's workers at rows
+        [q count, (q+1) count), rank q serving columns ranges[q] = (a, b).
+        Afterwards every rank holds columns ranges[rank] of every row."""
+        P2P = self.dist.P2POp
+        r, ops = self.rank, []
+        for q in range(self.world):
+            if q == r:
+                continue
+            a, b = ranges[q]
+            if b > a:        # my workers' words of q's chunks, to q
+                ops += [P2P(self.dist.isend, rows[w, a:b], self._peer(q), self.group)
+                        for w in range(r * count, (r + 1) * count)]
+            a, b = ranges[r]
+            if b > a:        # q's workers' words of my chunks, from q
+                ops += [P2P(self.dist.irecv, rows[w, a:b], self._peer(q), self.group)
+                        for w in range(q * count, (q + 1) * count)]
+        self._run(ops)
+
+    def gather_ranges(self, buf: torch.Tensor, ranges) -> None:
+        """Server stage: buf is 1-D, rank q holding the entries ranges[q] =
+        (a, b).  Afterwards every rank holds all of them."""
+        P2P = self.dist.P2POp
+        r, ops = self.rank, []
+        a_r, b_r = ranges[r]
+        for q in range(self.world):
+            if q == r:
+                continue
+            if b_r > a_r:
+                ops.append(P2P(self.dist.isend, buf[a_r:b_r], self._peer(q), self.group))
+            a, b = ranges[q]
+            if b > a:
+                ops.append(P2P(self.dist.irecv, buf[a:b], self._peer(q), self.group))
+        self._run(ops)
+
     def sum_(self, buf: torch.Tensor) -> None:
         self.dist.all_reduce(buf, op=self.dist.ReduceOp.SUM, group=self.group)
+
+
+def exchange_plan(numel: Sequence[int], W: int, world: int):
+    """Per rank (chunk_begin, chunk_end) and (word_begin, word_end) of the
+    server shard it serves (ob_server_shard_range)."""
+    shards = [B.ob_server_shard_range(numel, W, world, q) for q in range(world)]
+    return [(s[0], s[1]) for s in shards], [(s[2], s[3]) for s in shards]
 
 
 class DistributedOneBitAdam:
@@ -88,7 +143,9 @@ class DistributedOneBitAdam:
         self.opt = OneBitAdam(numel, W, device=device, stream=stream, **hyper)
         ctx, ws = self.opt.ctx, self.opt.workspace
         B.ob_set_server_shard(ctx, self.world, self.rank)
-        self.chunk_begin, self.chunk_end, _, _ = B.ob_server_shard_range(numel, W, self.world, self.rank)
+        # every rank's served chunks and their words, for the exchanges
+        self.chunk_ranges, self.word_ranges = exchange_plan(numel, W, self.world)
+        self.chunk_begin, self.chunk_end = self.chunk_ranges[self.rank]
         bits, bits_row, scales, scales_row = B.ob_worker_exchange_buffers(ctx)
         self.worker_bits = _view(ws, bits, self.W * bits_row, torch.int32).view(self.W, -1)
         self.worker_scales = _view(ws, scales, self.W * scales_row, torch.float32).view(self.W, -1)
@@ -166,27 +223,40 @@ class DistributedOneBitAdam:
             self.exchange_impl = TorchExchange()
         return self.exchange_impl
 
+    def exchange_worker_stage(self, ex) -> None:
+        """The worker stage's exchange: each rank's chunks of every worker's
+        words, and all worker scales."""
+        ex.send_worker_chunks(self.worker_bits, self.w_local, self.word_ranges)
+        ex.gather_rows(self.worker_scales, self.w_begin, self.w_local)
+
+    def exchange_server_stage(self, ex) -> None:
+        """The server stage's exchange: every rank's server words and chunk
+        scales to every rank."""
+        ex.gather_ranges(self.server_bits, self.word_ranges)
+        ex.gather_ranges(self.server_scales, self.chunk_ranges)
+
     def step(self, local_grads: Sequence[torch.Tensor]) -> None:
         ex = self._exchange()
         with torch.cuda.stream(self.opt.stream):
             self.worker_stage(local_grads)
-            ex.gather_rows(self.worker_bits, self.w_begin, self.w_local)
-            ex.gather_rows(self.worker_scales, self.w_begin, self.w_local)
+            if self.world > 1:
+                self.exchange_worker_stage(ex)
             self.server_stage()
             if self.world > 1:
-                ex.sum_(self.server_bits)
-                ex.sum_(self.server_scales)
+                self.exchange_server_stage(ex)
             self.apply_update()
 
     def exchange_bytes(self) -> dict:
-        """Bytes each exchange moves into this process per step (the sum's
-        figure is its buffer size; the bytes on the wire depend on NCCL's
-        algorithm)."""
+        """Bytes each exchange brings into this process per step."""
         others = self.W - self.w_local
-        return {"worker_rows_all_gather": others * (self.worker_bits.shape[1]
-                                                    + self.worker_scales.shape[1]) * 4,
-                "server_words_and_scales_sum": (self.server_bits.numel() + self.server_scales.numel()) * 4
-                if self.world > 1 else 0}
+        wb, we = self.word_ranges[self.rank]
+        T = self.worker_scales.shape[1]
+        theirs = [q for q in range(self.world) if q != self.rank]
+        return {"worker_words": others * (we - wb) * 4,
+                "worker_scales": others * T * 4,
+                "server_words": sum(self.word_ranges[q][1] - self.word_ranges[q][0] for q in theirs) * 4,
+                "server_scales": sum(self.chunk_ranges[q][1] - self.chunk_ranges[q][0]
+                                     for q in theirs) * 4}
 
     def read(self, kind: int, index: int = 0):
         return self.opt.read(kind, index)
@@ -229,6 +299,18 @@ class LocalRanks:
         for r in self.ranks:
             r.freeze()
 
+    def _send_worker_chunks(self) -> None:
+        """Rank dst receives, in every other rank's worker rows, the words
+        of the chunks dst serves."""
+        for dst in self.ranks:
+            a, b = dst.word_ranges[dst.rank]
+            if b <= a:
+                continue
+            for src in self.ranks:
+                if src is not dst:
+                    rows = slice(src.w_begin, src.w_begin + src.w_local)
+                    dst.worker_bits[rows, a:b].copy_(src.worker_bits[rows, a:b])
+
     def _gather_rows(self, attr: str) -> None:
         for dst in self.ranks:
             for src in self.ranks:
@@ -236,24 +318,27 @@ class LocalRanks:
                     rows = slice(src.w_begin, src.w_begin + src.w_local)
                     getattr(dst, attr)[rows].copy_(getattr(src, attr)[rows])
 
-    def _sum(self, attr: str) -> None:
-        total = getattr(self.ranks[0], attr).clone()
-        for r in self.ranks[1:]:
-            total += getattr(r, attr)
-        for r in self.ranks:
-            getattr(r, attr).copy_(total)
+    def _gather_ranges(self, attr: str, ranges_attr: str) -> None:
+        for src in self.ranks:
+            a, b = getattr(src, ranges_attr)[src.rank]
+            if b <= a:
+                continue
+            for dst in self.ranks:
+                if dst is not src:
+                    getattr(dst, attr)[a:b].copy_(getattr(src, attr)[a:b])
 
     def step(self, all_grads: torch.Tensor) -> None:
         """all_grads: [W, n_padded]; rank r gets its workers' rows."""
         for r in self.ranks:
             r.worker_stage([all_grads[r.w_begin + i] for i in range(r.w_local)])
-        self._gather_rows("worker_bits")
-        self._gather_rows("worker_scales")
+        if self.G > 1:
+            self._send_worker_chunks()
+            self._gather_rows("worker_scales")
         for r in self.ranks:
             r.server_stage()
         if self.G > 1:
-            self._sum("server_bits")
-            self._sum("server_scales")
+            self._gather_ranges("server_bits", "word_ranges")
+            self._gather_ranges("server_scales", "chunk_ranges")
         for r in self.ranks:
             r.apply_update()
 

@@ -132,7 +132,18 @@ def _rank_main(rank, world, port, out):
         sp = torch.zeros(4, dtype=torch.float32)
         sp[rank::world] = torch.tensor([0.1 + rank, 3e-7])
         ex.sum_(sp)
-        out[rank] = (rows.tolist(), scales.tolist(), words.tolist(), sp.tolist())
+        # per-chunk worker words: rank 0 serves columns [0, 6), rank 1 none
+        chunk_rows = torch.full((W, 8), -1, dtype=torch.int32)
+        chunk_rows[2 * rank:2 * rank + 2] = (torch.arange(16, dtype=torch.int32).view(2, 8)
+                                             + 1000 * rank)
+        ex.send_worker_chunks(chunk_rows, 2, [(0, 6), (6, 6)])
+        # server ranges: rank 0 holds [0, 3), rank 1 [3, 7); [7, 9) is nobody's
+        srv = torch.full((9,), -5.0)
+        a, b = [(0, 3), (3, 7)][rank]
+        srv[a:b] = torch.arange(a, b, dtype=torch.float32) + 0.25
+        ex.gather_ranges(srv, [(0, 3), (3, 7)])
+        out[rank] = (rows.tolist(), scales.tolist(), words.tolist(), sp.tolist(),
+                     chunk_rows.tolist(), srv.tolist())
     finally:
         dist.destroy_process_group()
 
@@ -143,8 +154,21 @@ def test_torch_exchange_on_two_gloo_ranks():
         out = mgr.dict()
         mp.spawn(_rank_main, args=(world, _free_port(), out), nprocs=world, join=True)
         res = dict(out)
-    assert res[0] == res[1]
-    rows, scales, words, sp = res[0]
+    assert res[0][:4] == res[1][:4]
+    rows, scales, words, sp, _, _ = res[0]
+    for r in range(world):
+        chunk_rows, srv = res[r][4], res[r][5]
+        assert srv == [0.25, 1.25, 2.25, 3.25, 4.25, 5.25, 6.25, -5.0, -5.0]
+        for q in range(world):
+            for i in range(2):
+                w = 2 * q + i
+                want = [v + 1000 * q for v in range(8 * i, 8 * i + 8)]
+                if q == r:
+                    assert chunk_rows[w] == want            # own rows untouched
+                elif r == 0:
+                    assert chunk_rows[w] == want[:6] + [-1, -1]   # only rank 0's columns came
+                else:
+                    assert chunk_rows[w] == [-1] * 8       # rank 1 serves nothing
     assert words == [-7, -8, 2**30, 2**30 + 1, -(2**31), -(2**31), 5, 5]
     assert sp == [np.float32(0.1).item(), np.float32(1.1).item(),
                   np.float32(3e-7).item(), np.float32(3e-7).item()]
@@ -200,13 +224,15 @@ def _grads(numel, W, step):
 
 
 def _protocol_rank(rank, world, port, out, numel, W, steps):
-    """One process of the split step with the oracle doing its arithmetic:
-    worker stage of its workers, all-gather of the worker rows, server stage
-    of its shard, sum of the server words and scales, update of everything."""
+    """One process of the split step with the oracle doing its arithmetic,
+    on buffers in the library's padded layout: worker stage of its workers,
+    the per-chunk exchange of the worker words (plus the worker scales),
+    server stage of its shard, the exchange of the server words and scales,
+    update of everything."""
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     import datetime
     import oracle
-    from error_compensated_bit_adam_b200.distributed import TorchExchange
+    from error_compensated_bit_adam_b200.distributed import TorchExchange, exchange_plan
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
     try:
@@ -217,51 +243,61 @@ def _protocol_rank(rank, world, port, out, numel, W, steps):
         run = oracle.OracleRun(params, W, hp)          # this process's state
         o, T, wl = run.o, len(numel), W // world
         mine = range(rank * wl, (rank + 1) * wl)
-        cb, ce, _, _ = B.ob_server_shard_range(numel, W, world, rank)
+        offsets, n_pad = B.ob_layout(numel)
+        chunk_ranges, word_ranges = exchange_plan(numel, W, world)
+        cb, ce = chunk_ranges[rank]
+        first = [off // 32 for off in offsets]
+        nw = [o.num_words(n) for n in numel]
+        received = 0
         for step in range(2):
             run.warmup_step(_grads(numel, W, step))    # every process, every worker
         run.freeze()
         for step in range(2, 2 + steps):
             g = _grads(numel, W, step)
-            words = [torch.zeros((W, o.num_words(n)), dtype=torch.int32) for n in numel]
+            bits = torch.zeros((W, n_pad // 32), dtype=torch.int32)   # stale rows stay 0
             scales = torch.zeros((W, T), dtype=torch.float32)
             for w in mine:
                 for t in range(T):
                     b, s = run.worker_stage(w, t, g[w][t])
-                    words[t][w] = torch.from_numpy(b.view(np.int32))
+                    bits[w, first[t]:first[t] + nw[t]] = torch.from_numpy(b.view(np.int32))
                     scales[w, t] = float(s)
-            for t in range(T):
-                ex.gather_rows(words[t], rank * wl, wl)
+            ex.send_worker_chunks(bits, wl, word_ranges)
             ex.gather_rows(scales, rank * wl, wl)
-            sbits = [np.zeros(o.num_words(n), np.uint32) for n in numel]
-            s_srv = np.zeros((T, W), np.float32)
+            sbits = torch.zeros(n_pad // 32, dtype=torch.int32)
+            s_srv = torch.zeros(T * W, dtype=torch.float32)
             for t in range(T):
-                rows = [words[t][w].numpy().view(np.uint32).copy() for w in range(W)]
+                rows = [bits[w, first[t]:first[t] + nw[t]].numpy().view(np.uint32).copy()
+                        for w in range(W)]
+                words_t = np.zeros(nw[t], np.uint32)
                 for j in range(W):
                     if cb <= t * W + j < ce:
-                        s_srv[t, j] = o.server_compress_chunk(j, rows, scales[:, t].numpy(),
-                                                              run.e_s[t], sbits[t])
-            sw = [torch.from_numpy(sb.view(np.int32)) for sb in sbits]
+                        s_srv[t * W + j] = float(o.server_compress_chunk(
+                            j, rows, scales[:, t].numpy(), run.e_s[t], words_t))
+                sbits[first[t]:first[t] + nw[t]] = torch.from_numpy(words_t.view(np.int32))
+            mine_words = sbits[slice(*word_ranges[rank])].clone()
+            ex.gather_ranges(sbits, word_ranges)
+            ex.gather_ranges(s_srv, chunk_ranges)
+            assert torch.equal(sbits[slice(*word_ranges[rank])], mine_words)
+            received += sum(b - a for q, (a, b) in enumerate(word_ranges) if q != rank)
             for t in range(T):
-                ex.sum_(sw[t])
-            st_ = torch.from_numpy(s_srv)
-            ex.sum_(st_)
-            for t in range(T):
-                full = sw[t].numpy().view(np.uint32)
+                full = sbits[first[t]:first[t] + nw[t]].numpy().view(np.uint32)
                 for j in range(W):
-                    o.apply_chunk(j, W, hp["lr"], full, st_[t, j].item(), run.d[t], run.p[t], run.m[t])
+                    o.apply_chunk(j, W, hp["lr"], full, s_srv[t * W + j].item(), run.d[t], run.p[t],
+                                  run.m[t])
         served = {(t, j) for t in range(T) for j in range(W) if cb <= t * W + j < ce}
         out[rank] = ([p.tobytes() for p in run.p], [m.tobytes() for m in run.m],
                      {w: [e.tobytes() for e in run.e_w[w]] for w in mine},
                      {(t, j): run.e_s[t][slice(*o.chunk_range(numel[t], W, j))].tobytes()
-                      for (t, j) in served})
+                      for (t, j) in served}, received)
     finally:
         dist.destroy_process_group()
 
 
-def test_split_protocol_on_gloo_ranks_equals_one_process():
+@pytest.mark.parametrize("numel,W,world", [([5_001, 64, 0, 777], 4, 2), ([70_000, 33], 6, 3),
+                                           ([100, 33, 5000], 8, 4)])
+def test_split_protocol_on_gloo_ranks_equals_one_process(numel, W, world):
     import oracle
-    numel, W, world, steps = [5_001, 64, 0, 777], 4, 2, 3
+    steps = 3
     with mp.Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_protocol_rank, args=(world, _free_port(), out, numel, W, steps), nprocs=world,
@@ -277,8 +313,10 @@ def test_split_protocol_on_gloo_ranks_equals_one_process():
     for step in range(2, 2 + steps):
         ref.compressed_step(_grads(numel, W, step))
     o = ref.o
+    n_words = B.ob_layout(numel)[1] // 32
     for r in range(world):
-        p, m, e_w, e_s = res[r]
+        p, m, e_w, e_s, received = res[r]
+        assert received < steps * n_words      # only the other ranks' words came in
         assert p == [a.tobytes() for a in ref.p] and m == [a.tobytes() for a in ref.m]
         for w, rows in e_w.items():
             assert rows == [e.tobytes() for e in ref.e_w[w]]

@@ -3,11 +3,13 @@ the exchanges between them) against one ob_compressed_step context.
 
 G ranks run in one process on one GPU (distributed.LocalRanks), each with
 its own context and its own range of server chunks, the exchanges done by
-device copies and sums.  The bar is bit for bit: parameters, momentum, the
-server words and scales, and every worker's words and scales on every
-rank, the worker errors on their rank and the server error on the rank
-serving each chunk, after warmup, freeze and several compressed steps with
-fresh gradients."""
+device copies of the ranges the processes would send each other.  The bar
+is bit for bit: parameters, momentum, the server words and scales, every
+worker scale on every rank, each rank's own workers' words whole and the
+other workers' words over the chunks the rank serves, the worker errors on
+their rank and the server error on the rank serving each chunk, after
+warmup, freeze and several compressed steps with fresh gradients.  The
+same runs are also compared with the CPU oracle."""
 import numpy as np
 import pytest
 import torch
@@ -16,6 +18,7 @@ from error_compensated_bit_adam_b200 import _binding as B
 from error_compensated_bit_adam_b200 import workloads as WL
 from error_compensated_bit_adam_b200.distributed import DistributedOneBitAdam, LocalRanks
 from error_compensated_bit_adam_b200.optimizer import OneBitAdam
+import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -27,10 +30,12 @@ CASES = {
     "ragged-W6-G3": ((50_001, 129, 12_345), 6, 3),
     "empty-chunks-W16-G4": ((100, 33, 5000), 16, 4),
     "W4-G1": ((30_000, 7), 4, 1),
+    "ragged-W8-G8": ((100_003, 31, 0, 4097, 70_000, 1 << 16), 8, 8),
+    "two-tensors-W4-G2": ((4096 * 5 + 17, 4096 * 3), 4, 2),
 }
 
 
-def _run(sizes, W, G, warmup=2, compressed=4, seed=31):
+def _run(sizes, W, G, warmup=2, compressed=4, seed=31, orc=False):
     wl = WL.Workload(f"split-{W}-{G}", tuple((n,) for n in sizes), W, warmup, compressed, seed=seed,
                      zero_fraction=0.2)
     offsets, n_pad = B.ob_layout(wl.numels)
@@ -38,24 +43,37 @@ def _run(sizes, W, G, warmup=2, compressed=4, seed=31):
     scale = WL.grad_scale_vector(wl, offsets, n_pad, device="cuda")
     ref = OneBitAdam(wl.numels, W, params=params.clone(), **WL.HYPER)
     ranks = LocalRanks(wl.numels, W, G, **WL.HYPER)
+    run = (oracle.OracleRun(WL.split(params.cpu().numpy(), offsets, wl.numels), W, WL.HYPER)
+           if orc else None)
     for r in ranks.ranks:
         r.params.copy_(params)
     g = torch.empty((W, n_pad), device="cuda")
+
+    def host(g):
+        h = g.cpu().numpy()
+        return [WL.split(h[w], offsets, wl.numels) for w in range(W)]
+
     step = 0
     for _ in range(warmup):
         WL.fill_grads(wl, step, scale, g)
         step += 1
         ref.warmup_step(g)
         ranks.warmup_step(g)
+        if run:
+            run.warmup_step(host(g))
     ref.freeze()
     ranks.freeze()
+    if run:
+        run.freeze()
     for _ in range(compressed):
         WL.fill_grads(wl, step, scale, g)
         step += 1
         ref.step(g)
         ranks.step(g)
+        if run:
+            run.compressed_step(host(g))
     torch.cuda.synchronize()
-    return ref, ranks
+    return (ref, ranks, run) if orc else (ref, ranks)
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -69,8 +87,13 @@ def test_split_step_equals_one_context(name):
         for r in ranks.ranks:
             for k, v in want.items():
                 np.testing.assert_array_equal(r.read(k), v, err_msg=f"{name} rank {r.rank} kind {k}")
+            a, b = r.word_ranges[r.rank]             # the words of the chunks r serves
             for w in range(W):
-                np.testing.assert_array_equal(r.read(B.OB_STATE_BITS_WORKER, w), want_bits[w])
+                got = r.read(B.OB_STATE_BITS_WORKER, w)
+                if r.w_begin <= w < r.w_begin + r.w_local:
+                    np.testing.assert_array_equal(got, want_bits[w])
+                else:
+                    np.testing.assert_array_equal(got[a:b], want_bits[w][a:b])
             for w in range(r.w_begin, r.w_begin + r.w_local):  # errors live with their worker
                 np.testing.assert_array_equal(r.read(B.OB_STATE_E_WORKER, w),
                                               ref.read(B.OB_STATE_E_WORKER, w))
@@ -88,6 +111,36 @@ def test_split_step_equals_one_context(name):
                         np.testing.assert_array_equal(e[offsets[t] + b:offsets[t] + end],
                                                       e_ref[offsets[t] + b:offsets[t] + end])
         assert served == len(sizes) * W
+    finally:
+        ref.close()
+        ranks.close()
+
+
+@pytest.mark.parametrize("sizes,W,G", [((1 << 18,), 8, 2), ((100_003, 31, 0, 4097, 70_000), 8, 4),
+                                       ((100, 33, 5000), 16, 8), ((50_001, 129, 12_345), 6, 3)])
+def test_split_step_follows_the_oracle(sizes, W, G):
+    """The split step against the CPU oracle over the same schedule: worker
+    and server scales within 1e-6 relative, the server words bit for bit
+    while every scale has matched the oracle's exactly (else at most 1e-3
+    of the bits), parameters within 1e-5 relative L2 after 4 free-running
+    compressed steps."""
+    ref, ranks, run = _run(sizes, W, G, orc=True)
+    try:
+        offsets, _ = ref.layout()
+        for r in ranks.ranks:
+            s_w = r.read(B.OB_STATE_S_WORKER)
+            s_s = r.read(B.OB_STATE_S_SERVER)
+            np.testing.assert_allclose(s_w, run.s_w, rtol=1e-6, atol=0)
+            np.testing.assert_allclose(s_s, run.s_srv, rtol=1e-6, atol=0)
+            words = r.read(B.OB_STATE_BITS_SERVER)
+            exact = np.array_equal(s_w, run.s_w) and np.array_equal(s_s, run.s_srv)
+            for t, n in enumerate(sizes):
+                got = words[offsets[t] // 32:offsets[t] // 32 + (n + 31) // 32]
+                diff = int(np.unpackbits((got ^ run.sbits[t]).view(np.uint8)).sum())
+                assert diff == 0 or (not exact and diff <= max(1, 1e-3 * 32 * got.size)), (t, diff)
+            p = np.concatenate(WL.split(r.read(B.OB_STATE_P), offsets, list(sizes))).astype(np.float64)
+            want = np.concatenate(run.p).astype(np.float64)
+            assert np.linalg.norm(p - want) <= 1e-5 * np.linalg.norm(want)
     finally:
         ref.close()
         ranks.close()
