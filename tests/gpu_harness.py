@@ -39,8 +39,10 @@ def words_of(flat_words: np.ndarray, offsets, numels):
 class Pair:
     """A GPU context and an oracle run over the same workload."""
 
-    def __init__(self, wl: WL.Workload, device="cuda", threads: int = 1, hp: Optional[dict] = None):
+    def __init__(self, wl: WL.Workload, device="cuda", threads: int = 1, hp: Optional[dict] = None,
+                 lamb: bool = False):
         self.wl = wl
+        self.lamb = lamb
         self.hp = dict(hp or WL.HYPER)
         self.W = wl.W
         self.numels = wl.numels
@@ -48,9 +50,9 @@ class Pair:
         self.dev = torch.device(device)
         params = WL.make_params(wl, self.offsets, self.n_pad, device=self.dev)
         self.scale = WL.grad_scale_vector(wl, self.offsets, self.n_pad, device=self.dev)
-        self.gpu = OneBitAdam(self.numels, wl.W, params=params.clone(), **self.hp)
+        self.gpu = OneBitAdam(self.numels, wl.W, params=params.clone(), layerwise=lamb, **self.hp)
         self.orc = oracle.OracleRun(WL.split(params.cpu().numpy(), self.offsets, self.numels), wl.W,
-                                    self.hp, threads=threads)
+                                    self.hp, threads=threads, lamb=lamb)
         del params
         self.grads = torch.empty((wl.W, self.n_pad), dtype=torch.float32, device=self.dev)
         self.step_index = 0
