@@ -186,16 +186,21 @@ def workload_config(wl: WL.Workload, n_pad: int, parallelism: str, grad_sets: in
 
 # ------------------------------------------------------------ oracle timing
 
-def oracle_sample_rate(W: int, n_sample: int, steps: int, warm: int = 1):
-    """Time the oracle's compressed step (single-threaded C) on a flat
-    n_sample vector with W workers; returns (params/s per worker, seconds
-    per step).  Inputs come from the shared generator, on the CPU."""
+ORACLE_SAMPLE = 1 << 21  # elements of the flat vector the oracle is timed on (both legs)
+
+
+def oracle_sample_rate(W: int, n_sample: int, steps: int, warm: int = 1, threads: int = 1):
+    """Time the oracle's compressed step (single-threaded C calls; with
+    threads > 1 its independent per-worker and per-chunk calls run
+    concurrently) on a flat n_sample vector with W workers; returns
+    (params/s per worker, seconds per step).  Inputs come from the shared
+    generator, on the CPU."""
     import oracle
     wl = WL.flat(n_sample, W, warmup=1, compressed=steps, seed=41, name="oracle-sample")
     offs = [0]
     p = WL.make_params(wl, offs, n_sample).numpy()
     scale = WL.grad_scale_vector(wl, offs, n_sample)
-    run = oracle.OracleRun([p], W, WL.HYPER)
+    run = oracle.OracleRun([p], W, WL.HYPER, threads=threads)
     g = torch.empty((W, n_sample), dtype=torch.float32)
     WL.fill_grads(wl, 0, scale, g)
     run.warmup_step([[g[w].numpy()] for w in range(W)])
@@ -213,11 +218,20 @@ def oracle_sample_rate(W: int, n_sample: int, steps: int, warm: int = 1):
     return n_sample / t, t
 
 
-def cpu_baseline(W: int, n_sample: int = 1 << 23, steps: int = 4) -> dict:
+def cpu_baseline(W: int, n_sample: int = ORACLE_SAMPLE, steps: int = 8) -> dict:
     rate, t = oracle_sample_rate(W, n_sample, steps)
-    return {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"flat fp32 n={n_sample}, W={W}: {steps} timed oracle compressed steps "
-                      f"({t:.2f} s each) after 1 Adam step and the freeze; single-threaded C"}
+    out = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"flat fp32 n={n_sample}, W={W}: {steps} timed oracle compressed steps "
+                     f"({t:.2f} s each) after 1 Adam step and the freeze; single-threaded C"}
+    cores = os.cpu_count() or 1
+    if cores > 1 and W > 1:  # a second, separately labelled figure: the same calls on every core
+        threads = min(cores, W)
+        trate, tt = oracle_sample_rate(W, n_sample, steps, threads=threads)
+        out["threaded"] = {"value": trate, "unit": UNIT, "cores": threads, "kind": "oracle",
+                           "sample": f"the same sample, its {W} worker stages and {W} server "
+                                     f"chunks run as concurrent single-threaded calls "
+                                     f"({tt:.2f} s per step)"}
+    return out
 
 
 # ------------------------------------------------------------- reference arm
@@ -227,7 +241,7 @@ def run_reference(args) -> None:
     if rank != 0:
         return
     wl = pick_workload(args)
-    n_sample = min(wl.n, 1 << 21)
+    n_sample = min(wl.n, ORACLE_SAMPLE)
     rate, t = oracle_sample_rate(wl.W, n_sample, args.steps, warm=args.warmup)
     line = {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
@@ -603,7 +617,7 @@ def run_b200(args) -> None:
     offsets, n_pad = B.ob_layout(wl.numels)
     params = WL.make_params(wl, offsets, n_pad, device=dev)
     scale = WL.grad_scale_vector(wl, offsets, n_pad, device=dev)
-    opt = OneBitAdam(wl.numels, wl.W, params=params, device=dev, **WL.HYPER)
+    opt = OneBitAdam(wl.numels, wl.W, params=params, device=dev, layerwise=args.lamb, **WL.HYPER)
     set_bytes = 4 * wl.W * n_pad
     free_bytes = torch.cuda.mem_get_info(dev)[0]
     n_sets = GRAD_SETS if free_bytes > GRAD_SETS * set_bytes + 2 * 4 * n_pad + (1 << 30) else 1
@@ -731,8 +745,9 @@ def run_b200(args) -> None:
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": workload_config(wl, n_pad, f"replicas{world}" if world > 1 else "single GPU",
-                                      n_sets),
+            "config": dict(workload_config(wl, n_pad, f"replicas{world}" if world > 1 else "single GPU",
+                                           n_sets),
+                           optimizer="1-bit LAMB (layerwise trust ratios)" if args.lamb else "1-bit Adam"),
             "params_per_s_aggregate_all_workers": value * wl.W,
             "hbm_gbs_step": step_gbs,
             "hbm_frac_of_measured_peak_step": step_gbs / peak["hbm_gbs"],
@@ -781,6 +796,8 @@ def main(argv=None):
                          "GPUs through the split step and its NCCL exchange; 'replicas' runs N "
                          "independent copies of the one-GPU step.  '--multi split' with one GPU "
                          "runs the split step's calls without an exchange")
+    ap.add_argument("--lamb", action="store_true",
+                    help="time 1-bit LAMB (layerwise trust ratios, ob_set_layerwise) instead of 1-bit Adam")
     ap.add_argument("--graph", action="store_true",
                     help="also time the steps replayed as one CUDA graph each")
     ap.add_argument("--overlap", action="store_true",
