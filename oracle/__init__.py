@@ -339,11 +339,10 @@ class OracleRun:
             self.d[t][a:b] = self.o.freeze(self.t_warmup, self.hp, self.v[t][a:b])
         self._run([lambda t=t, a=a, b=b: job(t, a, b)
                    for t in range(self.T) for a, b in self._slices(self.numel[t])])
-        for w in range(self.W):
-            for t in range(self.T):
-                self.e_w[w][t][:] = 0
-        for t in range(self.T):
-            self.e_s[t][:] = 0
+        # e_w = 0, e_s = 0 (fresh zero arrays: their pages are only touched
+        # when the first compressed step writes them)
+        self.e_w = [[np.zeros(n, np.float32) for n in self.numel] for _ in range(self.W)]
+        self.e_s = [np.zeros(n, np.float32) for n in self.numel]
 
     def worker_stage(self, w: int, t: int, g: np.ndarray):
         """Worker stage of one worker on one tensor; returns (bits, s)."""

@@ -58,12 +58,12 @@ FULL = {
     WL.ENCODER_24L_W16.name: shortened(WL.ENCODER_24L_W16, 2, 10),
     WL.RAGGED_2000_W8.name: shortened(WL.RAGGED_2000_W8, 2, 10),
 }
-# sweep points: the whole oracle up to W*n = 2^30 worker elements; above
-# that (up to 2^34, minutes of single-core oracle time each) sampled
-# elements and any-size properties
-SAMPLED = {}
+# sweep points: one Adam step and two compressed steps each, against the
+# whole oracle whenever the host has the RAM for it (test_full_size_...
+# routes by oracle_host_bytes), else sampled elements and any-size
+# properties
 for _w in WL.sweep():
-    (FULL if _w.W * _w.n <= (1 << 30) else SAMPLED)[_w.name] = shortened(_w, 1, 2)
+    FULL[_w.name] = shortened(_w, 1, 2)
 
 
 def run_with_oracle(wl: WL.Workload):
@@ -156,18 +156,16 @@ def device_room(wl: WL.Workload):
 
 @pytest.mark.parametrize("name", list(FULL))
 def test_full_size_against_oracle(name):
+    """The whole oracle when the host has 1.25x the RAM it needs (every
+    sweep point but (2^29, 32) on a host of about 200 GB), else the
+    sampled check for a flat vector."""
     wl = FULL[name]
     device_room(wl)
     if host_available() >= 1.25 * oracle_host_bytes(wl):
         run_with_oracle(wl)
     elif wl.n_tensors == 1:
+        print(f"{name}: host RAM {host_available() / 1e9:.0f} GB < 1.25 x the oracle's "
+              f"{oracle_host_bytes(wl) / 1e9:.0f} GB; sampled check")
         run_sampled(wl)
     else:
         pytest.skip(f"host RAM: the oracle needs ~{oracle_host_bytes(wl) / 1e9:.0f} GB")
-
-
-@pytest.mark.parametrize("name", list(SAMPLED))
-def test_full_size_sampled(name):
-    wl = SAMPLED[name]
-    device_room(wl)
-    run_sampled(wl)
