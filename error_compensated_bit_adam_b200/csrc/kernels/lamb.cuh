@@ -17,7 +17,9 @@
 // so D_j is computed once (ob_lamb_norms_kernel, at the freeze) and every
 // step needs only the chunk scales.  ||p||^2 is summed by the update kernel
 // as it writes p (for the next step), and by ob_lamb_norms_kernel whenever
-// p was changed otherwise (warmup, freeze, a state write).
+// p was changed otherwise (warmup, freeze, a state write).  Every kernel
+// here leaves per-tile partial sums; ob_scale_kernel (scale.cuh) adds them
+// per tensor or chunk in its fixed order.
 #pragma once
 
 #include "common.cuh"
@@ -56,15 +58,17 @@ __device__ __forceinline__ void block_sum2(double &a, double &b, double (*red)[2
 
 struct LambWarmupParams {
     WarmupParams w;
-    double *partial;    // [2][n_tiles]: per tile, sum of p^2 (before the step) and of r^2
+    double *partial;      // [2][n_tiles]: per tile, sum of p^2 (before the step) and of r^2
     int64_t n_tiles;
-    RangeSums sums;     // ranges = tensors
-    float *ratio;       // [T] out: the tensors' trust ratios
+    const double *sums;   // [2][T]: the tensors' ||p||^2 and ||r||^2 (for the step kernel)
+    int T;
+    const int *tensor_tile_begin;  // [T+1]
+    float *ratio;         // [T] out: the tensors' trust ratios
 };
 
-// First half of a LAMB warmup step: Adam's moments (written back) and, per
-// tensor, ||p||^2 of the parameters before the step and ||r||^2 of Adam's
-// direction, reduced to the tensor's trust ratio by its last CTA.
+// First half of a LAMB warmup step: Adam's moments (written back) and the
+// tile's partial sums of p^2 (the parameters before the step) and of r^2
+// (Adam's direction).
 __global__ void __launch_bounds__(kThreads) ob_lamb_moments_kernel(const __grid_constant__ LambWarmupParams P) {
     const int tile_id = (int)blockIdx.x;
     const Tile tile = P.w.tiles[tile_id];
@@ -97,17 +101,18 @@ __global__ void __launch_bounds__(kThreads) ob_lamb_moments_kernel(const __grid_
         P.partial[tile_id] = pp;
         P.partial[P.n_tiles + tile_id] = rr;
     }
-    reduce_ranges(P.sums, P.partial, P.n_tiles, 2, tile.tensor, tile_id,
-                  [&](int t, const double *s) {
-                      if (threadIdx.x == 0) P.ratio[t] = trust_ratio(s[0], s[1]);
-                  });
 }
 
-// Second half: p -= (lr * ratio_t) * r, r recomputed from the stored
+// Second half, once the sums are reduced per tensor: ratio_t =
+// ||p|| / ||r||, then p -= (lr * ratio_t) * r, r recomputed from the stored
 // moments with the same operations (so the same values).
 __global__ void __launch_bounds__(kThreads) ob_lamb_step_kernel(const __grid_constant__ LambWarmupParams P) {
-    const Tile tile = P.w.tiles[blockIdx.x];
-    const float lr_t = __fmul_rn(P.w.lr, P.ratio[tile.tensor]);
+    const int tile_id = (int)blockIdx.x;
+    const Tile tile = P.w.tiles[tile_id];
+    const int t = tile.tensor;
+    const float ratio = trust_ratio(P.sums[t], P.sums[P.T + t]);
+    if (threadIdx.x == 0 && tile_id == P.tensor_tile_begin[t]) P.ratio[t] = ratio;
+    const float lr_t = __fmul_rn(P.w.lr, ratio);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
         const int off = 4 * ((int)threadIdx.x + kThreads * u);
@@ -130,21 +135,15 @@ __global__ void __launch_bounds__(kThreads) ob_lamb_step_kernel(const __grid_con
 
 struct LambNormsParams {
     const Tile *tiles;
-    int tile_base;
     const float *d, *p;
-    double *partial_d;  // [n_tiles] per tile, sum of (1/d)^2
-    double *partial_p;  // [n_tiles] per tile, sum of p^2
-    int64_t n_tiles;
-    int W;
-    RangeSums chunks, tensors;
-    double *dnorm;      // [T][W] out: D_j of every server chunk (when want_d)
-    double *pnorm;      // [T] out: ||p||^2 of every tensor (when want_p)
+    double *partial_d;  // [n_tiles] per tile, sum of (1/d)^2 (when want_d)
+    double *partial_p;  // [n_tiles] per tile, sum of p^2 (when want_p)
     int want_d, want_p;
 };
 
-// D_j = sum over chunk j of (1/d)^2 and ||p||^2 per tensor, as asked.
+// Per-tile sums for D_j = sum over chunk j of (1/d)^2 and for ||p||^2.
 __global__ void __launch_bounds__(kThreads) ob_lamb_norms_kernel(const __grid_constant__ LambNormsParams P) {
-    const int tile_id = P.tile_base + (int)blockIdx.x;
+    const int tile_id = (int)blockIdx.x;
     const Tile tile = P.tiles[tile_id];
     __shared__ double red[kWarps][2];
     grid_dependency_wait();
@@ -167,19 +166,9 @@ __global__ void __launch_bounds__(kThreads) ob_lamb_norms_kernel(const __grid_co
     }
     block_sum2(dd, pp, red);
     if (threadIdx.x == 0) {
-        P.partial_d[tile_id] = dd;
-        P.partial_p[tile_id] = pp;
+        if (P.want_d) P.partial_d[tile_id] = dd;
+        if (P.want_p) P.partial_p[tile_id] = pp;
     }
-    if (P.want_d)
-        reduce_ranges(P.chunks, P.partial_d, P.n_tiles, 1, tile.tensor * P.W + tile.chunk, tile_id,
-                      [&](int c, const double *s) {
-                          if (threadIdx.x == 0) P.dnorm[c] = s[0];
-                      });
-    if (P.want_p)
-        reduce_ranges(P.tensors, P.partial_p, P.n_tiles, 1, tile.tensor, tile_id,
-                      [&](int t, const double *s) {
-                          if (threadIdx.x == 0) P.pnorm[t] = s[0];
-                      });
 }
 
 // ------------------------------------------------- the compressed update
@@ -187,20 +176,17 @@ __global__ void __launch_bounds__(kThreads) ob_lamb_norms_kernel(const __grid_co
 struct LambApplyParams {
     ApplyParams a;
     const int *tensor_tile_begin;  // [T+1]
-    double *pnorm;      // [T]: ||p||^2 before this step; rewritten with the new p's
+    const double *pnorm;  // [T]: ||p||^2 before this step
     const double *dnorm;  // [T][W]: D_j
-    float *ratio;       // [T] out
-    double *partial;    // [n_tiles]: per tile, sum of the new p^2
-    int64_t n_tiles;
-    RangeSums sums;     // ranges = tensors
+    float *ratio;         // [T] out
+    double *partial;      // [n_tiles]: per tile, sum of the new p^2 (the next step's ||p||^2)
 };
 
 // [1BA, Proposed method, 1-2] with the 1-bit LAMB page's layerwise rates:
 // the gather and update of ob_apply_kernel with lr_t = lr * ratio_t, where
 // ratio_t = ||p|| / ||m_hat / d|| is formed by every CTA of tensor t from
-// the tensor's W chunk scales (in chunk order) and ||p||^2.  The CTA that
-// completes the tensor rewrites ||p||^2 with the new parameters' (every
-// CTA of the tensor has read the old value by then).
+// the tensor's W chunk scales (in chunk order) and ||p||^2; and the tile's
+// partial sum of the new p^2.
 __global__ void __launch_bounds__(kThreads) ob_lamb_apply_kernel(const __grid_constant__ LambApplyParams P) {
     __shared__ float4 sd[kUnroll][kThreads];
     __shared__ float4 spp[kUnroll][kThreads];
@@ -226,9 +212,6 @@ __global__ void __launch_bounds__(kThreads) ob_lamb_apply_kernel(const __grid_co
     double unused = 0.0;
     block_sum2(pp, unused, red);
     if (threadIdx.x == 0) P.partial[tile_id] = pp;
-    reduce_ranges(P.sums, P.partial, P.n_tiles, 1, t, tile_id, [&](int r, const double *s) {
-        if (threadIdx.x == 0) P.pnorm[r] = s[0];
-    });
 }
 
 }  // namespace onebit

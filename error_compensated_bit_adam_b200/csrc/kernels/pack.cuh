@@ -4,7 +4,6 @@
 #pragma once
 
 #include "common.cuh"
-#include "scale.cuh"
 
 namespace onebit {
 
@@ -28,18 +27,12 @@ struct PackParams {
     int64_t n_pad;
     int W, T;
     float beta1, c1;
-    ScaleEpilogue scales;            // worker scales: ranges = tensors, one row per worker,
-                                     // out_prev = s_prev (read above, rewritten last)
 };
 
 // [1BA, Proposed method, 3; Abstract]: for every worker w of one tile,
 //   m_w = beta1 m + (1-beta1) g_w,  x = m_w + e_w (e_w decoded from the
-//   stored (x_prev, s_prev)), sign bits of x, partial sum of x^2; the CTAs
-//   that finish a tensor's last tiles then form its scales
-//   s_w = ||x||_2 / sqrt(n_t) (finish_scales).
-// x overwrites x_prev: with this step's scale it encodes the new e_w.  The
-// scale s_prev[w][t] is rewritten only after every tile of tensor t has
-// arrived, so every CTA has read the old one by then.
+//   stored (x_prev, s_prev)), sign bits of x, partial sum of x^2.
+// x overwrites x_prev: with this step's scale it encodes the new e_w.
 // m stays in registers across the W workers, so it is read once.  After a
 // compressed step m is exactly last step's decoded server momentum
 // sign' s'_j, so it is rebuilt from the server words (1/8 byte per
@@ -151,7 +144,6 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
         for (int k = 0; k < kWarps; ++k) acc += red[k][tid];
         P.partial[(int64_t)tid * P.n_tiles + tile_id] = acc;
     }
-    finish_scales(P.scales, P.partial, P.n_tiles, P.W, tile.tensor, tile_id);
 }
 
 }  // namespace onebit

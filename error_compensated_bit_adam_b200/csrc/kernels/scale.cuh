@@ -1,4 +1,4 @@
-// kernels/scale.cuh -- Worker and server scales, finished inside the kernels that produce their partial sums.
+// kernels/scale.cuh -- Range sums of per-tile partial sums: the worker and server scales, and 1-bit LAMB's norms.
 //
 // Part of libonebit (sm_100a); see onebit_kernels.cuh for the overview.
 #pragma once
@@ -10,132 +10,116 @@ namespace onebit {
 // ------------------------------------------------------------- scales
 //
 // A scale is sqrt(S / count) ([1BA, Proposed method, 3]: the 1-bit code's
-// magnitude, the RMS of what it compresses), with S the sum of squares of
-// one range of tiles: a tensor for the worker scales (one row per worker),
-// a server chunk for the server scales (one row).  Every tile CTA writes
-// its per-row partial sums, then takes part in a two-level reduction that
-// needs no kernel of its own and never waits:
-//   * a range is cut into segments of kScaleSegTiles tiles; the CTA that
-//     arrives last at a segment (thread fence, then an atomic counter) sums
-//     the segment's partials for every row;
-//   * a range of one segment has its scales then; otherwise the CTA that
-//     finishes the range's last segment sums the segment results and
-//     writes the scales.
-// Every addition's order is fixed by the layout alone (sum_rows), so the
-// scales repeat run to run whatever the CTAs' timing.  The last arriver
-// resets each counter to 0 for the next launch.  Ranges with no tiles (an
-// empty tensor or server chunk) keep the scale they were given, 0.
+// magnitude, the RMS of what it compresses), with S the sum of the per-tile
+// partial sums of one range of tiles (a tensor for the worker scales, a
+// server chunk for the server scales).  A range is cut into segments of
+// kScaleSegTiles tiles; one CTA sums one segment, and the CTA that finishes
+// last for the range sums the segment results in segment order.  The order
+// of every addition is fixed by the layout, so the scales repeat run to
+// run.  The last CTA is found with a per-range counter (thread fence, then
+// atomic increment; it resets the counter), so nothing ever waits.
+//
+// The same kernel also returns plain range sums (out_sum), for 1-bit
+// LAMB's norms.
+//
+// The reduction is a kernel of its own on purpose: finishing it in the
+// tail of the tile kernels that produce the partial sums (fence, atomic
+// arrival, barrier at the end of every CTA) held each CTA and its shared
+// memory past its last store and cost 15% of the worker stage and 20% of
+// the server stage on the B200, against about 20 us for these launches.
 
-constexpr int kScaleSegTiles = 512;
+constexpr int kScaleSegTiles = 2048;
 
-// Row sums of rows x [lo, hi) doubles, row r at base + r * row_stride,
-// into out[r].  Warp g sums rows g, g + kWarps, ...: lane l adds entries
-// lo + l, lo + l + 32, ... into four accumulators in turn, the accumulators
-// are added pairwise and the lanes by a butterfly.  Ends with a barrier.
-__device__ __forceinline__ void sum_rows(const double *base, int64_t row_stride, int rows, int lo,
-                                         int hi, double *out) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int r = warp; r < rows; r += kWarps) {
-        const double *v = base + (int64_t)r * row_stride;
-        double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
-        int k = lo + lane;
-        for (; k + 96 < hi; k += 128) {
-            a0 += __ldcg(v + k);
-            a1 += __ldcg(v + k + 32);
-            a2 += __ldcg(v + k + 64);
-            a3 += __ldcg(v + k + 96);
-        }
-        for (; k < hi; k += 32) a0 += __ldcg(v + k);
-        const double s = warp_sum((a0 + a1) + (a2 + a3));
-        if (lane == 0) out[r] = s;
+__device__ __forceinline__ double segment_sum(const double *v, int lo, int hi, double *smem) {
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+    int k = lo + (int)threadIdx.x;
+    for (; k + 3 * kScaleThreads < hi; k += 4 * kScaleThreads) {
+        a0 += __ldcg(v + k);
+        a1 += __ldcg(v + k + kScaleThreads);
+        a2 += __ldcg(v + k + 2 * kScaleThreads);
+        a3 += __ldcg(v + k + 3 * kScaleThreads);
+    }
+    for (; k < hi; k += kScaleThreads) a0 += __ldcg(v + k);
+    return block_sum((a0 + a1) + (a2 + a3), smem);
+}
+
+// One segment of range r; returns (in thread 0, with *done = true) the
+// range's total when this CTA is the last of the range's nseg CTAs.
+__device__ __forceinline__ bool range_sum(const double *v, int lo, int hi, int seg, int nseg,
+                                          double *seg_out, unsigned *counter, double *total) {
+    __shared__ double smem[kScaleThreads / 32];
+    __shared__ bool last;
+    const int a = lo + seg * kScaleSegTiles;
+    const int b = min(hi, a + kScaleSegTiles);
+    const double part = segment_sum(v, a, b, smem);
+    if (nseg == 1) {
+        *total = part;
+        return true;
+    }
+    if (threadIdx.x == 0) {
+        seg_out[seg] = part;
+        __threadfence();
+        last = atomicAdd(counter, 1u) == (unsigned)(nseg - 1);
     }
     __syncthreads();
+    if (!last) return false;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        double acc = 0.0;
+        for (int k = 0; k < nseg; ++k) acc += __ldcg(seg_out + k);
+        *counter = 0u;
+        *total = acc;
+    }
+    return true;
+}
+
+__device__ __forceinline__ int num_segments(int tiles) {
+    return tiles <= kScaleSegTiles ? 1 : (tiles + kScaleSegTiles - 1) / kScaleSegTiles;
 }
 
 __device__ __forceinline__ float rms(double sum_sq, int64_t count) {
     return count > 0 ? __double2float_rn(__dsqrt_rn(__ddiv_rn(sum_sq, (double)count))) : 0.0f;
 }
 
-// The ranges a producing kernel reduces over, and where the segment sums
-// and counters live.
-struct RangeSums {
-    const int *range_begin;    // [R+1] first tile of each range (absolute tile indices)
+struct ScaleParams {
+    const double *partial;     // per-tile sums
+    int n_tiles;               // row length of partial (worker scales: one row per worker)
+    const int *range_begin;    // [R+1] tile ranges
     const int *seg_base;       // [R] first segment slot of each range
-    unsigned *seg_counter;     // [segment slots] arrivals, 0 between launches
-    unsigned *range_counter;   // [R] finished segments, 0 between launches
-    double *seg;               // segment sums: row r, slot q at seg[r * seg_stride + q]
-    int seg_stride;
-};
-
-// Where a producing kernel finishes its scales: the reduction, then
-// scale (range, row) = sqrt(sum / count[range]) at
-// out[range * stride_r + row * stride_row].
-struct ScaleEpilogue {
-    RangeSums sums;
     const int64_t *count;      // [R] elements of each range
-    float *out_prev, *out_last;
-    int out_stride_r, out_stride_row;
+    double *seg;               // segment results, [segments][rows]
+    unsigned *counter;         // [R][rows], zero between launches
+    float *out_prev, *out_last;  // scales, when out_sum is NULL
+    double *out_sum;           // plain range sums instead, when not NULL
+    int rows;                  // workers (worker scales) or 1 (server scales)
+    int R;
+    int out_stride_r, out_stride_row;  // out[r * stride_r + row * stride_row]
 };
 
-// Called by every thread of a tile CTA once threads [0, rows) have stored
-// the tile's partial sums partial[row * n_tiles + tile_id].  `range` is the
-// tile's range; rows <= OB_MAX_WORKERS; kThreads threads.  The CTA that
-// completes the range calls done(range, sums) in every thread, sums[r]
-// being row r's total (shared memory); every other CTA returns without
-// calling it.  The ranges' rows are summed in an order fixed by the layout.
-template <class Done>
-__device__ __forceinline__ void reduce_ranges(const RangeSums &E, const double *partial,
-                                              int64_t n_tiles, int rows, int range, int tile_id,
-                                              Done done) {
-    __shared__ double sums[OB_MAX_WORKERS];
-    __shared__ int last;
-    const int tid = threadIdx.x;
-    const int lo = E.range_begin[range], hi = E.range_begin[range + 1];
-    const int nseg = (hi - lo + kScaleSegTiles - 1) / kScaleSegTiles;
-    const int s = (tile_id - lo) / kScaleSegTiles;
-    const int a = lo + s * kScaleSegTiles, b = min(hi, a + kScaleSegTiles);
-    const int slot = E.seg_base[range] + s;
-    __threadfence();  // this thread's partial sums before the arrival below
-    __syncthreads();
-    if (tid == 0) {
-        __threadfence();
-        last = atomicAdd(&E.seg_counter[slot], 1u) == (unsigned)(b - a - 1);
-    }
-    __syncthreads();
-    if (!last) return;
-    __threadfence();  // the other CTAs' partial sums are visible from here
-    sum_rows(partial, n_tiles, rows, a, b, sums);
-    if (nseg > 1) {
-        if (tid < rows) E.seg[(int64_t)tid * E.seg_stride + slot] = sums[tid];
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) {
-            E.seg_counter[slot] = 0u;
-            last = atomicAdd(&E.range_counter[range], 1u) == (unsigned)(nseg - 1);
+// Grid (R, rows, segments): worker scales use ranges = tensors and one row
+// per worker; server scales use ranges = (tensor, chunk) and one row.
+__global__ void __launch_bounds__(kScaleThreads) ob_scale_kernel(const __grid_constant__ ScaleParams P) {
+    const int r = blockIdx.x, row = blockIdx.y, seg = blockIdx.z;
+    grid_dependency_wait();
+    allow_dependent_launch();
+    const int lo = P.range_begin[r], hi = P.range_begin[r + 1];
+    const int nseg = num_segments(hi - lo);
+    if (seg >= nseg) return;
+    double total = 0.0;
+    const double *v = P.partial + (int64_t)row * P.n_tiles;
+    double *seg_out = P.seg + ((int64_t)P.seg_base[r] * P.rows + (int64_t)row * nseg);
+    if (!range_sum(v, lo, hi, seg, nseg, seg_out, P.counter + (int64_t)r * P.rows + row, &total))
+        return;
+    if (threadIdx.x == 0) {
+        const int64_t o = (int64_t)r * P.out_stride_r + (int64_t)row * P.out_stride_row;
+        if (P.out_sum) {
+            P.out_sum[o] = total;
+        } else {
+            const float s = rms(total, P.count[r]);
+            P.out_prev[o] = s;
+            P.out_last[o] = s;
         }
-        __syncthreads();
-        if (!last) return;
-        __threadfence();
-        sum_rows(E.seg + E.seg_base[range], E.seg_stride, rows, 0, nseg, sums);
-        if (tid == 0) E.range_counter[range] = 0u;
-    } else if (tid == 0) {
-        E.seg_counter[slot] = 0u;
     }
-    done(range, (const double *)sums);
-}
-
-__device__ __forceinline__ void finish_scales(const ScaleEpilogue &E, const double *partial,
-                                              int64_t n_tiles, int rows, int range, int tile_id) {
-    reduce_ranges(E.sums, partial, n_tiles, rows, range, tile_id,
-                  [&](int r, const double *sums) {
-                      const int tid = threadIdx.x;
-                      if (tid < rows) {
-                          const float sc = rms(sums[tid], E.count[r]);
-                          const int64_t o = (int64_t)r * E.out_stride_r + (int64_t)tid * E.out_stride_row;
-                          E.out_prev[o] = sc;
-                          E.out_last[o] = sc;
-                      }
-                  });
 }
 
 }  // namespace onebit

@@ -4,7 +4,6 @@
 #pragma once
 
 #include "common.cuh"
-#include "scale.cuh"
 
 namespace onebit {
 
@@ -14,7 +13,7 @@ constexpr int kTileWords = kTile / 32;  // sign words of one worker in a full ti
 
 struct ServerParams {
     const Tile *tiles;
-    int tile_base;          // tile of blockIdx.x == 0
+    int tile_base;          // tile of blockIdx.x == 0 (partial sums indexed by the absolute tile)
     const uint32_t *bits;   // [W][n_pad/32] this step's worker signs
     const float *s_w;       // [W][T] this step's worker scales
     float *y;               // [n_pad]: in y_prev (lazy e_s), out y
@@ -25,8 +24,6 @@ struct ServerParams {
     int W, T;
     float inv_w;            // 1/W when W is a power of two (then acc*inv_w == acc/W exactly)
     int w_pow2;
-    ScaleEpilogue scales;   // server scales: ranges = (tensor, chunk), one row,
-                            // out_prev = sp_prev (read above, rewritten last)
 };
 
 // Two independent IEEE round-to-nearest additions in one instruction
@@ -44,9 +41,7 @@ __device__ __forceinline__ void add2_rn(float &a0, float &a1, float b0, float b1
 // index into [W][words]) and forms
 //   y = (sum over w in order of sign_w s_w) / W + e_s,
 // with e_s decoded from (y_prev, s'_prev); then the sign bits of y and the
-// tile's partial sum of y^2, and the chunk's scale s'_j = ||y||_2 /
-// sqrt(len_j) once its last tile is in (finish_scales; s'_prev of the chunk
-// is rewritten only after every tile of the chunk has read it).  The tile's W word rows are staged in shared
+// tile's partial sum of y^2.  The tile's W word rows are staged in shared
 // memory with one 16-byte load per thread, so the W-long sequential sum
 // never waits on global memory.  FULL tiles (all 4096 elements real, the
 // rule) skip every per-element bound check.
@@ -156,7 +151,6 @@ __global__ void __launch_bounds__(kThreads) ob_server_kernel(const __grid_consta
         server_tile<true>(P, tile, tile_id, staged, scale_bits, red);
     else
         server_tile<false>(P, tile, tile_id, staged, scale_bits, red);
-    finish_scales(P.scales, P.partial, 0, 1, tile.tensor * P.W + tile.chunk, tile_id);
 }
 
 }  // namespace onebit

@@ -174,7 +174,7 @@ struct Carve {
     size_t m, v, x, y, bits, sbits, s_prev, s_last, sp_prev, sp_last, partial_w, partial_s,
         counters_w, counters_s, seg_w, seg_s, tiles, tensor_tile_begin, chunk_tile_begin, numel,
         chunk_len, tensor_seg_base, chunk_seg_base, stage, ratio, pnorm, dnorm, partial_lamb,
-        seg_lamb, total;
+        seg_lamb, counters_lamb, lamb_sums, total;
 };
 
 Carve carve(const Plan &pl) {
@@ -199,10 +199,8 @@ Carve carve(const Plan &pl) {
     c.sp_last = take(T * W * 4);
     c.partial_w = take(W * nt * 8);
     c.partial_s = take(nt * 8);
-    // scale reductions: arrivals per segment slot, then finished segments
-    // per range (tensors for the workers, chunks for the servers)
-    c.counters_w = take(((size_t)pl.tensor_segs + T) * 4);
-    c.counters_s = take(((size_t)pl.chunk_segs + T * W) * 4);
+    c.counters_w = take(T * W * 4);
+    c.counters_s = take(T * W * 4);
     c.seg_w = take((size_t)pl.tensor_segs * W * 8);
     c.seg_s = take((size_t)pl.chunk_segs * 8);
     c.tiles = take(nt * sizeof(Tile));
@@ -220,6 +218,8 @@ Carve carve(const Plan &pl) {
     c.dnorm = take(T * W * 8);
     c.partial_lamb = take(2 * nt * 8);
     c.seg_lamb = take(2 * (size_t)pl.tensor_segs * 8);
+    c.counters_lamb = take(2 * T * 4);
+    c.lamb_sums = take(2 * T * 8);
     c.total = off;
     return c;
 }
@@ -310,7 +310,7 @@ struct ob_ctx {
     // m is held densely in the m region (after create / warmup / a write),
     // or, after a compressed step, only as the server words and scales.
     bool m_dense = true;
-    bool use_graph = false;
+    bool use_graph = true;  // graph mode (ob_graph_enable); used while the stream is not captured
     StepGraph graph;
     // 1-bit LAMB (ob_set_layerwise): layerwise trust ratios; the norms the
     // compressed update needs are valid unless p or d changed otherwise
@@ -360,6 +360,8 @@ struct ob_ctx {
     double *dnorm() const { return at<double>(cv.dnorm); }
     double *partial_lamb() const { return at<double>(cv.partial_lamb); }
     double *seg_lamb() const { return at<double>(cv.seg_lamb); }
+    unsigned *counters_lamb() const { return at<unsigned>(cv.counters_lamb); }
+    double *lamb_sums() const { return at<double>(cv.lamb_sums); }
     int n_tiles() const { return (int)plan.tiles.size(); }
 };
 
@@ -438,52 +440,71 @@ dim3 grid1(int n) { return dim3((unsigned)n); }
 
 // Worker scales, finished by the worker-stage kernel: ranges = tensors,
 // one row per worker, scale (t, w) at s_prev[w * T + t].
-// Reductions over tensors (the worker stage's; also the LAMB norms, in
-// other kernels) and over server chunks (the server stage's).
-onebit::RangeSums tensor_sums(const ob_ctx *c) {
-    onebit::RangeSums E{};
-    E.range_begin = c->tensor_tile_begin();
-    E.seg_base = c->tensor_seg_base();
-    E.seg_counter = c->counters_w();
-    E.range_counter = c->counters_w() + c->plan.tensor_segs;
-    E.seg = c->seg_w();
-    E.seg_stride = c->plan.tensor_segs;
-    return E;
+// Range sums of per-tile partial sums (ob_scale_kernel): the worker and
+// server scales, and plain sums for 1-bit LAMB's norms.
+onebit::ScaleParams worker_scale_params(const ob_ctx *c) {
+    onebit::ScaleParams P{};  // zeroed, padding too: compared bytewise in graph mode
+    P.partial = c->partial_w();
+    P.n_tiles = c->n_tiles();
+    P.range_begin = c->tensor_tile_begin();
+    P.seg_base = c->tensor_seg_base();
+    P.count = c->numel();
+    P.seg = c->seg_w();
+    P.counter = c->counters_w();
+    P.out_prev = c->s_prev();
+    P.out_last = c->s_last();
+    P.rows = c->plan.W;
+    P.R = c->plan.T;
+    P.out_stride_r = 1;
+    P.out_stride_row = c->plan.T;
+    return P;
 }
 
-onebit::RangeSums chunk_sums(const ob_ctx *c) {
-    onebit::RangeSums E{};
-    E.range_begin = c->chunk_tile_begin();
-    E.seg_base = c->chunk_seg_base();
-    E.seg_counter = c->counters_s();
-    E.range_counter = c->counters_s() + c->plan.chunk_segs;
-    E.seg = c->seg_s();
-    E.seg_stride = c->plan.chunk_segs;
-    return E;
+onebit::ScaleParams server_scale_params(const ob_ctx *c) {
+    onebit::ScaleParams P{};  // zeroed, padding too: compared bytewise in graph mode
+    P.partial = c->partial_s();
+    P.n_tiles = c->n_tiles();
+    P.range_begin = c->chunk_tile_begin();
+    P.seg_base = c->chunk_seg_base();
+    P.count = c->chunk_len();
+    P.seg = c->seg_s();
+    P.counter = c->counters_s();
+    P.out_prev = c->sp_prev();
+    P.out_last = c->sp_last();
+    P.rows = 1;
+    P.R = c->plan.T * c->plan.W;
+    P.out_stride_r = 1;
+    P.out_stride_row = 0;
+    return P;
 }
 
-onebit::ScaleEpilogue worker_scale_epilogue(const ob_ctx *c) {
-    onebit::ScaleEpilogue E{};
-    E.sums = tensor_sums(c);
-    E.count = c->numel();
-    E.out_prev = c->s_prev();
-    E.out_last = c->s_last();
-    E.out_stride_r = 1;
-    E.out_stride_row = c->plan.T;
-    return E;
+// Plain sums per tensor of `rows` rows of per-tile partials (rows <= 2):
+// out[row * T + t].  Uses the worker scales' buffers for one row and the
+// 1-bit LAMB ones for two.
+onebit::ScaleParams tensor_sum_params(const ob_ctx *c, const double *partial, int rows, double *out) {
+    onebit::ScaleParams P{};  // zeroed, padding too: compared bytewise in graph mode
+    P.partial = partial;
+    P.n_tiles = c->n_tiles();
+    P.range_begin = c->tensor_tile_begin();
+    P.seg_base = c->tensor_seg_base();
+    P.count = c->numel();
+    P.seg = rows == 1 ? c->seg_w() : c->seg_lamb();
+    P.counter = rows == 1 ? c->counters_w() : c->counters_lamb();
+    P.out_sum = out;
+    P.rows = rows;
+    P.R = c->plan.T;
+    P.out_stride_r = 1;
+    P.out_stride_row = c->plan.T;
+    return P;
 }
 
-// Server scales, finished by the server-stage kernel: ranges = (tensor,
-// chunk) at t * W + j, one row, scale at sp_prev[t * W + j].
-onebit::ScaleEpilogue server_scale_epilogue(const ob_ctx *c) {
-    onebit::ScaleEpilogue E{};
-    E.sums = chunk_sums(c);
-    E.count = c->chunk_len();
-    E.out_prev = c->sp_prev();
-    E.out_last = c->sp_last();
-    E.out_stride_r = 1;
-    E.out_stride_row = 0;
-    return E;
+// Plain sums per server chunk of one row of per-tile partials: out[t * W + j].
+onebit::ScaleParams chunk_sum_params(const ob_ctx *c, const double *partial, double *out) {
+    onebit::ScaleParams P = server_scale_params(c);
+    P.partial = partial;
+    P.out_prev = P.out_last = nullptr;
+    P.out_sum = out;
+    return P;
 }
 
 onebit::PackParams pack_params(const ob_ctx *c, const float *const *g, int64_t g_offset,
@@ -508,7 +529,6 @@ onebit::PackParams pack_params(const ob_ctx *c, const float *const *g, int64_t g
     P.T = c->plan.T;
     P.beta1 = c->beta1;
     P.c1 = c->c1;
-    P.scales = worker_scale_epilogue(c);
     return P;
 }
 
@@ -527,7 +547,6 @@ onebit::ServerParams server_params(const ob_ctx *c) {
     P.T = c->plan.T;
     P.w_pow2 = (W & (W - 1)) == 0;
     P.inv_w = 1.0f / (float)W;  // exact for a power of two
-    P.scales = server_scale_epilogue(c);
     return P;
 }
 
@@ -544,9 +563,10 @@ onebit::ApplyParams apply_params(const ob_ctx *c) {
     return P;
 }
 
-// The 1-bit LAMB update: apply_params with the layerwise rates, and the
-// new ||p||^2 reduced per tensor (in the worker stage's tensor-range
-// buffers, free once the worker stage is done).
+// The 1-bit LAMB update: apply_params with the layerwise rates; its
+// per-tile sums of the new p^2 go to the worker stage's partial-sum row 0
+// (free once the worker scales are done) and are reduced per tensor into
+// pnorm by a range-sum launch after it.
 onebit::LambApplyParams lamb_apply_params(const ob_ctx *c) {
     onebit::LambApplyParams P{};  // zeroed, padding too: compared bytewise in graph mode
     P.a = apply_params(c);
@@ -555,8 +575,6 @@ onebit::LambApplyParams lamb_apply_params(const ob_ctx *c) {
     P.dnorm = c->dnorm();
     P.ratio = c->ratio();
     P.partial = c->partial_w();
-    P.n_tiles = c->n_tiles();
-    P.sums = tensor_sums(c);
     return P;
 }
 
@@ -566,8 +584,17 @@ struct Geometry {
     size_t smem;
 };
 Geometry pack_geometry(int tiles) { return {grid1(tiles), dim3(kThreads), (size_t)onebit::kPackSmemBytes}; }
+Geometry range_sum_geometry(int ranges, int rows, int max_seg) {
+    return {dim3((unsigned)ranges, (unsigned)rows, (unsigned)max_seg), dim3(kScaleThreads), 0};
+}
+Geometry worker_scale_geometry(const ob_ctx *c) {
+    return range_sum_geometry(c->plan.T, c->plan.W, c->plan.tensor_max_seg);
+}
 Geometry server_geometry(int tiles, int W) {
     return {grid1(tiles), dim3(kThreads), (size_t)W * onebit::kTileWords * sizeof(uint32_t)};
+}
+Geometry server_scale_geometry(const ob_ctx *c) {
+    return range_sum_geometry(c->plan.T * c->plan.W, 1, c->plan.chunk_max_seg);
 }
 Geometry apply_geometry(const ob_ctx *c) { return {grid1(c->n_tiles()), dim3(kThreads), 0}; }
 
@@ -597,13 +624,17 @@ ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int ti
     return fail_cuda(c, launch(onebit::ob_pack_kernel, pack_geometry(tile_hi - tile_lo), P, c->stream));
 }
 
-// The gather and update (1-bit LAMB's with layerwise rates when on).
+// The gather and update (1-bit LAMB's with layerwise rates when on; then
+// its new ||p||^2 summed per tensor for the next step).
 ob_status launch_apply(ob_ctx *c) {
     if (c->n_tiles() == 0) return OB_OK;
     KernelTimer k(c, OB_K_APPLY);
-    const cudaError_t e =
+    cudaError_t e =
         c->lamb ? launch(onebit::ob_lamb_apply_kernel, apply_geometry(c), lamb_apply_params(c), c->stream)
                 : launch(onebit::ob_apply_kernel, apply_geometry(c), apply_params(c), c->stream);
+    if (e == cudaSuccess && c->lamb)
+        e = launch(onebit::ob_scale_kernel, range_sum_geometry(c->plan.T, 1, c->plan.tensor_max_seg),
+                   tensor_sum_params(c, c->partial_w(), 1, c->pnorm()), c->stream);
     k.stop();
     return fail_cuda(c, e);
 }
@@ -614,22 +645,21 @@ ob_status launch_lamb_norms(ob_ctx *c, bool want_d, bool want_p) {
     if (c->n_tiles() > 0) {
         onebit::LambNormsParams P{};
         P.tiles = c->tiles();
-        P.tile_base = 0;
         P.d = c->v();
         P.p = c->params;
         P.partial_d = c->partial_s();
         P.partial_p = c->partial_w();
-        P.n_tiles = c->n_tiles();
-        P.W = c->plan.W;
-        P.chunks = chunk_sums(c);
-        P.tensors = tensor_sums(c);
-        P.dnorm = c->dnorm();
-        P.pnorm = c->pnorm();
         P.want_d = want_d ? 1 : 0;
         P.want_p = want_p ? 1 : 0;
         KernelTimer k(c, OB_K_FREEZE);
-        const cudaError_t e = launch(onebit::ob_lamb_norms_kernel, Geometry{grid1(c->n_tiles()), dim3(kThreads), 0},
-                                     P, c->stream);
+        cudaError_t e = launch(onebit::ob_lamb_norms_kernel, Geometry{grid1(c->n_tiles()), dim3(kThreads), 0},
+                               P, c->stream);
+        if (e == cudaSuccess && want_d)
+            e = launch(onebit::ob_scale_kernel, server_scale_geometry(c),
+                       chunk_sum_params(c, c->partial_s(), c->dnorm()), c->stream);
+        if (e == cudaSuccess && want_p)
+            e = launch(onebit::ob_scale_kernel, range_sum_geometry(c->plan.T, 1, c->plan.tensor_max_seg),
+                       tensor_sum_params(c, c->partial_w(), 1, c->pnorm()), c->stream);
         k.stop();
         ob_status st = fail_cuda(c, e);
         if (st != OB_OK) return st;
@@ -645,17 +675,31 @@ ob_status ensure_lamb_norms(ob_ctx *c) {
     return launch_lamb_norms(c, !c->dnorm_valid, !c->pnorm_valid);
 }
 
-// Everything of a compressed step after the worker stage's tile kernels
-// (which finish the worker scales themselves): the server stage, which
-// finishes the server scales, then the update.
+// Everything of a compressed step after the worker stage's tile kernels:
+// the worker scales, the server stage, the server scales, the update.
 ob_status launch_after_pack(ob_ctx *c, KernelTimer &pack_timer) {
     const int nt = c->n_tiles();
     pack_timer.stop();
-    if (nt == 0) return OB_OK;
     {
+        KernelTimer k(c, OB_K_PACK_SCALE);
+        const cudaError_t e =
+            launch(onebit::ob_scale_kernel, worker_scale_geometry(c), worker_scale_params(c), c->stream);
+        k.stop();
+        ob_status st = fail_cuda(c, e);
+        if (st != OB_OK) return st;
+    }
+    if (nt > 0) {
         KernelTimer k(c, OB_K_SERVER);
         const cudaError_t e =
             launch(onebit::ob_server_kernel, server_geometry(nt, c->plan.W), server_params(c), c->stream);
+        k.stop();
+        ob_status st = fail_cuda(c, e);
+        if (st != OB_OK) return st;
+    }
+    {
+        KernelTimer k(c, OB_K_SERVER_SCALE);
+        const cudaError_t e =
+            launch(onebit::ob_scale_kernel, server_scale_geometry(c), server_scale_params(c), c->stream);
         k.stop();
         ob_status st = fail_cuda(c, e);
         if (st != OB_OK) return st;
@@ -702,14 +746,21 @@ ob_status build_graph(ob_ctx *c, const float *const *g) {
     sg.lamb_apply = lamb_apply_params(c);
     sg.lamb = c->lamb;
     onebit::ServerParams sv = server_params(c);
-    cudaGraphNode_t n_sv;
+    onebit::ScaleParams ws = worker_scale_params(c), ss = server_scale_params(c);
+    onebit::ScaleParams pn = tensor_sum_params(c, c->partial_w(), 1, c->pnorm());
+    cudaGraphNode_t n_ws, n_sv, n_ss, n_pn;
+    if (nt > 0) add((void *)onebit::ob_pack_kernel, pack_geometry(nt), &sg.pack, &sg.pack_node);
+    add((void *)onebit::ob_scale_kernel, worker_scale_geometry(c), &ws, &n_ws);
+    if (nt > 0) add((void *)onebit::ob_server_kernel, server_geometry(nt, c->plan.W), &sv, &n_sv);
+    add((void *)onebit::ob_scale_kernel, server_scale_geometry(c), &ss, &n_ss);
     if (nt > 0) {
-        add((void *)onebit::ob_pack_kernel, pack_geometry(nt), &sg.pack, &sg.pack_node);
-        add((void *)onebit::ob_server_kernel, server_geometry(nt, c->plan.W), &sv, &n_sv);
-        if (sg.lamb)
+        if (sg.lamb) {
             add((void *)onebit::ob_lamb_apply_kernel, apply_geometry(c), &sg.lamb_apply, &sg.apply_node);
-        else
+            add((void *)onebit::ob_scale_kernel, range_sum_geometry(c->plan.T, 1, c->plan.tensor_max_seg),
+                &pn, &n_pn);
+        } else {
             add((void *)onebit::ob_apply_kernel, apply_geometry(c), &sg.apply, &sg.apply_node);
+        }
     }
     if (e == cudaSuccess) e = cudaGraphInstantiate(&sg.exec, sg.graph, 0);
     if (e != cudaSuccess) {
@@ -1110,12 +1161,16 @@ ob_status ob_warmup_adam_step(ob_ctx *c, const float *const *d_grads) {
         L.w = P;
         L.partial = c->partial_lamb();
         L.n_tiles = c->n_tiles();
-        L.sums = tensor_sums(c);
-        L.sums.seg = c->seg_lamb();
+        L.sums = c->lamb_sums();
+        L.T = c->plan.T;
+        L.tensor_tile_begin = c->tensor_tile_begin();
         L.ratio = c->ratio();
         KernelTimer k(c, OB_K_WARMUP);
         onebit::ob_lamb_moments_kernel<<<grid1(c->n_tiles()), kThreads, 0, c->stream>>>(L);
         cudaError_t e = cudaGetLastError();
+        if (e == cudaSuccess)  // ||p||^2 and ||r||^2 per tensor
+            e = launch(onebit::ob_scale_kernel, range_sum_geometry(c->plan.T, 2, c->plan.tensor_max_seg),
+                       tensor_sum_params(c, c->partial_lamb(), 2, c->lamb_sums()), c->stream);
         if (e == cudaSuccess) {
             onebit::ob_lamb_step_kernel<<<grid1(c->n_tiles()), kThreads, 0, c->stream>>>(L);
             e = cudaGetLastError();
@@ -1164,7 +1219,13 @@ ob_status ob_compressed_step(ob_ctx *c, const float *const *d_grads) {
     DeviceGuard dg(c->device);
     if (!dg.ok) return fail_cuda(c, cudaErrorInvalidDevice);
     if ((st = ensure_lamb_norms(c)) != OB_OK) return st;
-    if (c->use_graph && !c->profiling) {
+    // graph replay unless profiling, or unless the caller is capturing the
+    // stream into a graph of its own (then the launches are captured)
+    cudaStreamCaptureStatus capture = cudaStreamCaptureStatusNone;
+    if (c->use_graph && !c->profiling &&
+        (st = fail_cuda(c, cudaStreamIsCapturing(c->stream, &capture))) != OB_OK)
+        return st;
+    if (c->use_graph && !c->profiling && capture == cudaStreamCaptureStatusNone) {
         if ((st = graph_step(c, d_grads)) != OB_OK) return st;
     } else {
         KernelTimer pack(c, OB_K_PACK);
@@ -1202,7 +1263,7 @@ ob_status ob_worker_stage(ob_ctx *c, const float *const *d_grads, int w_begin, i
     if (w_count > 0 && nt > 0) {
         // the step's worker-stage kernel on a view of the worker rows: the
         // rows [w_begin, w_begin + w_count) of x, bits, the scales, the
-        // partial sums and the segment sums, as if they were all workers
+        // partial sums and the scales, as if they were all workers
         onebit::PackParams P = pack_params(c, d_grads, 0, 0);
         for (int i = 0; i < OB_MAX_WORKERS; ++i) P.g[i] = i < w_count ? d_grads[w_begin + i] : nullptr;
         P.x = c->x() + (size_t)w_begin * n;
@@ -1210,11 +1271,21 @@ ob_status ob_worker_stage(ob_ctx *c, const float *const *d_grads, int w_begin, i
         P.s_prev = c->s_prev() + (size_t)w_begin * T;
         P.partial = c->partial_w() + (size_t)w_begin * nt;
         P.W = w_count;
-        P.scales.sums.seg = c->seg_w() + (size_t)w_begin * c->plan.tensor_segs;
-        P.scales.out_prev = c->s_prev() + (size_t)w_begin * T;
-        P.scales.out_last = c->s_last() + (size_t)w_begin * T;
         KernelTimer k(c, OB_K_PACK);
         const cudaError_t e = launch(onebit::ob_pack_kernel, pack_geometry((int)nt), P, c->stream);
+        k.stop();
+        if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    }
+    if (w_count > 0) {
+        onebit::ScaleParams S = worker_scale_params(c);
+        S.partial = c->partial_w() + (size_t)w_begin * nt;
+        S.out_prev = c->s_prev() + (size_t)w_begin * T;
+        S.out_last = c->s_last() + (size_t)w_begin * T;
+        S.rows = w_count;
+        KernelTimer k(c, OB_K_PACK_SCALE);
+        const cudaError_t e = launch(onebit::ob_scale_kernel,
+                                     range_sum_geometry((int)T, w_count, c->plan.tensor_max_seg), S,
+                                     c->stream);
         k.stop();
         if ((st = fail_cuda(c, e)) != OB_OK) return st;
     }
@@ -1276,16 +1347,30 @@ ob_status ob_server_stage(ob_ctx *c) {
     cudaError_t e = cudaMemcpyAsync(c->s_last(), c->s_prev(), (size_t)pl.W * pl.T * 4,
                                     cudaMemcpyDeviceToDevice, c->stream);
     if ((st = fail_cuda(c, e)) != OB_OK) return st;
-    // The server stage (which finishes its chunks' scales) on the served
-    // chunks only: their tiles are one contiguous range of the work list,
-    // launched from its first tile.  Empty served chunks have no tile and
-    // keep their scale, 0.
+    // The server stage and its scales on the served chunks only: their
+    // tiles are one contiguous range of the work list, launched from its
+    // first tile (every index inside the kernels stays absolute), and their
+    // scales one contiguous range of the chunk arrays.
     const int t_lo = pl.chunk_tile_begin[lo], t_hi = pl.chunk_tile_begin[hi];
     if (t_hi > t_lo) {
         onebit::ServerParams P = server_params(c);
         P.tile_base = t_lo;
         KernelTimer k(c, OB_K_SERVER);
         e = launch(onebit::ob_server_kernel, server_geometry(t_hi - t_lo, pl.W), P, c->stream);
+        k.stop();
+        if ((st = fail_cuda(c, e)) != OB_OK) return st;
+    }
+    if (hi > lo) {
+        onebit::ScaleParams S = server_scale_params(c);
+        S.range_begin = c->chunk_tile_begin() + lo;
+        S.seg_base = c->chunk_seg_base() + lo;
+        S.count = c->chunk_len() + lo;
+        S.counter = c->counters_s() + lo;  // one row
+        S.out_prev = c->sp_prev() + lo;
+        S.out_last = c->sp_last() + lo;
+        S.R = hi - lo;
+        KernelTimer k(c, OB_K_SERVER_SCALE);
+        e = launch(onebit::ob_scale_kernel, range_sum_geometry(hi - lo, 1, pl.chunk_max_seg), S, c->stream);
         k.stop();
         if ((st = fail_cuda(c, e)) != OB_OK) return st;
     }

@@ -103,11 +103,12 @@ typedef enum ob_state_kind {
 typedef enum ob_kernel_id {
     OB_K_WARMUP = 0,          /* ob_warmup_adam_step */
     OB_K_FREEZE = 1,          /* ob_freeze_variance */
-    OB_K_PACK = 2,            /* worker stage: momentum, error, signs and the worker scales */
-    OB_K_PACK_SCALE = 3,      /* no longer launched: the worker stage finishes its scales (0 launches) */
-    OB_K_SERVER = 4,          /* server stage: average, server error, signs and the chunk scales */
-    OB_K_SERVER_SCALE = 5,    /* no longer launched: the server stage finishes its scales (0 launches) */
-    OB_K_APPLY = 6,           /* gather, decode and preconditioned update */
+    OB_K_PACK = 2,            /* worker stage: momentum, error, signs, partial sums of squares */
+    OB_K_PACK_SCALE = 3,      /* worker scales from the partial sums (ob_scale_kernel) */
+    OB_K_SERVER = 4,          /* server stage: average, server error, signs, partial sums */
+    OB_K_SERVER_SCALE = 5,    /* server chunk scales from the partial sums (ob_scale_kernel) */
+    OB_K_APPLY = 6,           /* gather, decode and preconditioned update (1-bit LAMB: with its
+                                 norm sums) */
     OB_NUM_KERNELS = 7
 } ob_kernel_id;
 
@@ -322,15 +323,20 @@ OB_API ob_status ob_set_layerwise(ob_ctx *ctx, int on);
  * (learning-rate schedules).  OB_ERR_INVALID_ARG for a non-finite lr. */
 OB_API ob_status ob_set_lr(ob_ctx *ctx, float lr);
 
-/* Graph mode on or off (default off).  While on (and profiling is off),
- * ob_compressed_step replays the step's three kernels as one CUDA graph,
- * built at the first such call: one launch instead of three, which matters
- * for small tensor lists where each kernel runs a few microseconds.
- * Changed gradient pointers, the dense/lazy state of m and the learning
- * rate are written into the graph before each replay; the results are
- * those of the ordinary launches.  ob_compressed_step_host never uses the
- * graph.  The first call in graph mode must not be made while the stream is
- * being captured. */
+/* Graph mode on (the default) or off.  While on, profiling is off and the
+ * context's stream is not being captured by the caller, ob_compressed_step
+ * replays the step's kernels as one CUDA graph, built at the first such
+ * call: one launch instead of five, which matters for small tensor lists
+ * where each kernel runs a few microseconds.  Changed gradient pointers,
+ * the dense/lazy state of m and the learning rate are written into the
+ * graph before each replay; the results are those of the ordinary
+ * launches.  While the caller captures the stream (or with graph mode or
+ * profiling off) the kernels are launched one by one, so they become part
+ * of the caller's capture; a captured step keeps the launch parameters of
+ * the step it was captured from (gradient pointers, learning rate, and
+ * whether m is read densely, as only the first step after the warmup or a
+ * write of M does), so capture a step after the first compressed one.
+ * ob_compressed_step_host and the split step never use the graph. */
 OB_API ob_status ob_graph_enable(ob_ctx *ctx, int on);
 
 /* Turn per-kernel timing on or off.  While on, every step records CUDA

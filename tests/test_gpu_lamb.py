@@ -139,6 +139,7 @@ def test_lamb_graph_mode_equals_direct_launches():
     wl = WL.Workload("lamb-graph", ((70_000,), (33,), (4096 * 3,)), 4, 2, 4, seed=66)
     a = OneBitAdam(wl.numels, wl.W, layerwise=True, **WL.HYPER)
     b = OneBitAdam(wl.numels, wl.W, layerwise=True, **WL.HYPER)
+    a.graph(False)
     b.graph(True)
     try:
         _lamb_pair_steps([a, b], wl, 7)

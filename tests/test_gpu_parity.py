@@ -319,6 +319,46 @@ def test_graph_mode_matches_direct_launches():
         assert np.array_equal(a.view(np.uint8), b.view(np.uint8))
 
 
+def test_steps_captured_by_the_caller_replay_like_direct_launches():
+    """With graph mode on (the default) a step queued while the caller
+    captures the context's stream is launched kernel by kernel into the
+    caller's graph; replaying that graph takes the same steps as direct
+    launches, bit for bit."""
+    wl = small_ragged(W=4, count=20)
+    offs, n_pad = B.ob_layout(wl.numels)
+    params = WL.make_params(wl, offs, n_pad, device="cuda")
+    scale = WL.grad_scale_vector(wl, offs, n_pad, device="cuda")
+    g = torch.empty((wl.W, n_pad), device="cuda")
+    s = torch.cuda.Stream()
+    cap = OneBitAdam(wl.numels, wl.W, params=params.clone(), stream=s, **WL.HYPER)
+    ref = OneBitAdam(wl.numels, wl.W, params=params.clone(), **WL.HYPER)
+    ref.graph(False)
+    try:
+        WL.fill_grads(wl, 0, scale, g)
+        torch.cuda.synchronize()
+        for o in (cap, ref):
+            o.warmup_step(g)
+            o.freeze()
+        torch.cuda.synchronize()
+        WL.fill_grads(wl, 1, scale, g)
+        torch.cuda.synchronize()
+        for o in (cap, ref):  # the first compressed step reads m densely, later ones lazily
+            o.step(g)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            cap.step(g)
+        for _ in range(3):
+            graph.replay()
+            ref.step(g)
+        torch.cuda.synchronize()
+        for kind in (B.OB_STATE_P, B.OB_STATE_BITS_SERVER, B.OB_STATE_S_SERVER, B.OB_STATE_S_WORKER):
+            assert np.array_equal(cap.read(kind).view(np.uint8), ref.read(kind).view(np.uint8)), kind
+    finally:
+        cap.close()
+        ref.close()
+
+
 def test_set_lr_rejects_non_finite():
     opt = OneBitAdam([100], 2, **WL.HYPER)
     with pytest.raises(B.OnebitError) as ei:
