@@ -37,3 +37,39 @@ def test_reference_arm_other_ranks_exit_without_work():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr
     assert not [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+
+
+import pytest  # noqa: E402
+
+
+def _b200_line(args):
+    r = subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600, env=dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0"))
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    return json.loads(lines[0])
+
+
+@pytest.mark.gpu
+def test_b200_arm_small_case_prints_the_contract_keys():
+    d = _b200_line(["--n", "1048576", "--workers", "4", "--steps", "5", "--warmup", "3",
+                    "--adam-steps", "2", "--no-cpu-baseline", "--e2e-steps", "1"])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config", "roofline",
+                "e2e", "gpu_launches", "clocks"):
+        assert key in d, key
+    assert d["n_gpus"] == 1 and d["value"] > 0 and d["gpu_launches"] == 5 * 5
+    assert d["roofline"]["kernel"] == "ob_pack_kernel" and d["roofline"]["frac"] > 0
+    assert d["e2e"]["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 4 * 1048576 * 4
+
+
+@pytest.mark.gpu
+def test_b200_arm_split_step_mode_on_one_gpu():
+    """--multi split runs the split step's calls through the bench's
+    multi-GPU path (with one process there is no exchange)."""
+    d = _b200_line(["--n", "1048576", "--workers", "4", "--steps", "5", "--warmup", "3",
+                    "--adam-steps", "2", "--multi", "split", "--e2e-steps", "1"])
+    assert d["scaling"] == "strong" and d["value"] > 0 and d["gpu_launches"] == 5 * 5
+    assert "split step" in d["config"]["parallelism"]
+    assert d["e2e"]["value"] > 0
