@@ -28,7 +28,7 @@ Every step of both 1-bit arms runs the library's kernels.  The result is
 reported as it comes out, whatever it shows.
 
     python -m error_compensated_bit_adam_b200.ablation [--n N] [--workers W]
-        [--steps T] [--warmup Tw] [--noise SIGMA ...] [--seed S]
+        [--steps T] [--warmup Tw] [--noise SIGMA ...] [--lr LR ...] [--h-min H ...] [--seed S]
 """
 from __future__ import annotations
 
@@ -122,18 +122,23 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=400)
     ap.add_argument("--noise", type=float, nargs="+", default=[0.01, 0.1, 1.0])
-    ap.add_argument("--lr", type=float, default=1e-2)
+    ap.add_argument("--lr", type=float, nargs="+", default=[1e-2, 1e-3])
+    ap.add_argument("--h-min", type=float, nargs="+", default=[1e-3, 1e-1],
+                    help="smallest curvature (the largest is --h-max): 1e-3 is ill-conditioned")
+    ap.add_argument("--h-max", type=float, default=10.0)
     ap.add_argument("--every", type=int, default=50)
     ap.add_argument("--seed", type=int, default=7)
     args = ap.parse_args(argv)
-    for noise in args.noise:
-        t0 = time.time()
-        curves = run(args.n, args.workers, args.steps, args.warmup, noise, args.lr, args.seed,
-                     every=args.every)
-        print(json.dumps({"n": args.n, "W": args.workers, "steps": args.steps,
-                          "warmup": args.warmup, "noise": noise, "lr": args.lr, "seed": args.seed,
-                          "every": args.every, "seconds": time.time() - t0, "loss": curves}),
-              flush=True)
+    for h_min in args.h_min:
+        for lr in args.lr:
+            for noise in args.noise:
+                t0 = time.time()
+                curves = run(args.n, args.workers, args.steps, args.warmup, noise, lr, args.seed,
+                             h_min=h_min, h_max=args.h_max, every=args.every)
+                print(json.dumps({"n": args.n, "W": args.workers, "steps": args.steps,
+                                  "warmup": args.warmup, "noise": noise, "lr": lr, "h_min": h_min,
+                                  "h_max": args.h_max, "seed": args.seed, "every": args.every,
+                                  "seconds": time.time() - t0, "loss": curves}), flush=True)
 
 
 if __name__ == "__main__":

@@ -177,10 +177,11 @@ class DistributedOneBitAdam:
         additions inside the all-reduce."""
         if len(local_grads) != self.w_local:
             raise ValueError(f"expected {self.w_local} local gradients")
-        ex = self._exchange()
         with torch.cuda.stream(self.opt.stream):
-            for g in local_grads:
-                ex.sum_(g)
+            if self.world > 1:  # one process: the sums are its own gradients
+                ex = self._exchange()
+                for g in local_grads:
+                    ex.sum_(g)
             self.warmup_from_sums(local_grads)
 
     def warmup_from_sums(self, sums: Sequence[torch.Tensor]) -> None:
