@@ -237,13 +237,13 @@ class DistributedOneBitAdam:
         ex.gather_ranges(self.server_scales, self.chunk_ranges)
 
     def step(self, local_grads: Sequence[torch.Tensor]) -> None:
-        ex = self._exchange()
+        ex = self._exchange() if self.world > 1 else None  # one process: nothing to exchange
         with torch.cuda.stream(self.opt.stream):
             self.worker_stage(local_grads)
-            if self.world > 1:
+            if ex is not None:
                 self.exchange_worker_stage(ex)
             self.server_stage()
-            if self.world > 1:
+            if ex is not None:
                 self.exchange_server_stage(ex)
             self.apply_update()
 
