@@ -58,6 +58,7 @@ EXPORTS = (
     "ob_onebit_compress_static", "ob_set_lr", "ob_graph_enable",
     "ob_server_shard_range", "ob_set_server_shard", "ob_worker_stage", "ob_worker_exchange_buffers",
     "ob_server_stage", "ob_server_exchange_buffers", "ob_apply_update", "ob_set_layerwise",
+    "ob_set_peer_words",
 )
 
 
@@ -129,6 +130,7 @@ def lib() -> ctypes.CDLL:
                                              ctypes.POINTER(vp), ctypes.POINTER(sz)]),
         "ob_apply_update": (i32, [vp]),
         "ob_set_layerwise": (i32, [vp, i32]),
+        "ob_set_peer_words": (i32, [vp, i32, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -332,6 +334,14 @@ def ob_server_exchange_buffers(ctx: int) -> Tuple[int, int, int, int]:
 
 def ob_apply_update(ctx: int) -> None:
     _check(lib().ob_apply_update(ctx), "ob_apply_update")
+
+
+def ob_set_peer_words(ctx: int, d_worker_bits: Sequence[int], d_server_bits: Sequence[int]) -> None:
+    """Fused word exchanges of the split step (empty lists turn them off)."""
+    n = len(d_worker_bits)
+    assert len(d_server_bits) == n
+    _check(lib().ob_set_peer_words(ctx, n, _ptrs(d_worker_bits) if n else None,
+                                   _ptrs(d_server_bits) if n else None), "ob_set_peer_words")
 
 
 # ------------------------------------------------------ allocation-free call

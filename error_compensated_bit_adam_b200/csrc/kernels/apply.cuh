@@ -18,6 +18,14 @@ struct ApplyParams {
     float *m;               // [n_pad] dense momentum, or NULL to keep it as (sbits, sp)
     int W;
     float lr;
+    // Split step with peer memory (n_shards > 0): the words of the tiles of
+    // shard q (shard_end as in PackParams) are read from src_sbits[q], the
+    // server words of the process serving it, and copied into sbits_copy
+    // (this process's server words, which then hold every chunk's).
+    int n_shards;
+    int shard_end[OB_MAX_WORKERS];
+    const uint32_t *src_sbits[OB_MAX_WORKERS];
+    uint32_t *sbits_copy;
 };
 
 // [1BA, Proposed method, 1-2]: every worker decodes the gathered server
@@ -31,9 +39,13 @@ struct ApplyParams {
 // slots into shared memory (cp.async, 32 KiB per CTA), then computes.
 // lr: the step's learning rate (P.lr, or 1-bit LAMB's layerwise rate).
 // With NORM the thread's sum of the new p^2 is returned (else 0).
+// sbits: where the tile's server words are read (P.sbits, or the serving
+// process's with peer memory); copy: where lane 8k of each group stores
+// the word it read (NULL: nowhere).
 template <bool FULL, bool NORM>
 __device__ __forceinline__ double apply_tile(const ApplyParams &P, const Tile &tile, float4 (*sd)[kThreads],
-                                             float4 (*spp)[kThreads], float lr) {
+                                             float4 (*spp)[kThreads], float lr, const uint32_t *sbits,
+                                             uint32_t *copy) {
     const int tid = threadIdx.x, lane = tid & 31;
     const uint32_t sb = __float_as_uint(P.sp[tile.tensor * P.W + tile.chunk]);
     const int shift = 4 * (lane & 7);
@@ -47,7 +59,9 @@ __device__ __forceinline__ double apply_tile(const ApplyParams &P, const Tile &t
             const int64_t i = tile.begin + off;
             cp_async16(&sd[u][tid], P.d + i, pol);
             cp_async16(&spp[u][tid], P.p + i, pol);
-            inv[u] = ~(__ldg(P.sbits + (i >> 5)) >> shift);
+            const uint32_t word = __ldg(sbits + (i >> 5));
+            if (copy && (lane & 7) == 0) copy[i >> 5] = word;
+            inv[u] = ~(word >> shift);
         }
     }
     cp_async_commit();
@@ -85,10 +99,13 @@ __global__ void __launch_bounds__(kThreads) ob_apply_kernel(const __grid_constan
     const Tile tile = P.tiles[blockIdx.x];  // the work list is written once, at create
     grid_dependency_wait();
     allow_dependent_launch();
+    const bool peer = P.n_shards > 0;
+    const uint32_t *sbits = peer ? P.src_sbits[shard_of(blockIdx.x, P.n_shards, P.shard_end)] : P.sbits;
+    uint32_t *copy = peer ? P.sbits_copy : nullptr;
     if (tile.count == kTile)
-        apply_tile<true, false>(P, tile, sd, spp, P.lr);
+        apply_tile<true, false>(P, tile, sd, spp, P.lr, sbits, copy);
     else
-        apply_tile<false, false>(P, tile, sd, spp, P.lr);
+        apply_tile<false, false>(P, tile, sd, spp, P.lr, sbits, copy);
 }
 
 }  // namespace onebit

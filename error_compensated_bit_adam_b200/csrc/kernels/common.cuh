@@ -168,6 +168,15 @@ __device__ __forceinline__ void allow_dependent_launch() {
     asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 }
 
+// The shard of the split step serving tile `tile_id`: the first q with
+// tile_id < shard_end[q] (n_shards > 0; shard_end ascending, its last entry
+// the number of tiles).
+__device__ __forceinline__ int shard_of(int tile_id, int n_shards, const int *shard_end) {
+    int q = 0;
+    while (q < n_shards - 1 && tile_id >= shard_end[q]) ++q;
+    return q;
+}
+
 // Real elements (0..4) of the float4 slot at tile offset off.
 __device__ __forceinline__ int slot_real(int count, int off) { return min(4, max(0, count - off)); }
 

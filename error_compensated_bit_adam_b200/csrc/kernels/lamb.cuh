@@ -205,10 +205,13 @@ __global__ void __launch_bounds__(kThreads) ob_lamb_apply_kernel(const __grid_co
     if (threadIdx.x == 0 && tile_id == P.tensor_tile_begin[t]) P.ratio[t] = ratio;
     const float lr_t = __fmul_rn(P.a.lr, ratio);
     double pp;
+    const bool peer = P.a.n_shards > 0;
+    const uint32_t *sbits = peer ? P.a.src_sbits[shard_of(tile_id, P.a.n_shards, P.a.shard_end)] : P.a.sbits;
+    uint32_t *copy = peer ? P.a.sbits_copy : nullptr;
     if (tile.count == kTile)
-        pp = apply_tile<true, true>(P.a, tile, sd, spp, lr_t);
+        pp = apply_tile<true, true>(P.a, tile, sd, spp, lr_t, sbits, copy);
     else
-        pp = apply_tile<false, true>(P.a, tile, sd, spp, lr_t);
+        pp = apply_tile<false, true>(P.a, tile, sd, spp, lr_t, sbits, copy);
     double unused = 0.0;
     block_sum2(pp, unused, red);
     if (threadIdx.x == 0) P.partial[tile_id] = pp;

@@ -27,7 +27,15 @@ struct PackParams {
     int64_t n_pad;
     int W, T;
     float beta1, c1;
+    // Split step with peer memory (n_shards > 0): the words of the tiles
+    // below shard_end[q] (absolute tile ids, ascending) and not below
+    // shard_end[q-1] go to dest[q] -- the worker rows of the process serving
+    // shard q, offset to this launch's first worker -- instead of `bits`.
+    int n_shards;
+    int shard_end[OB_MAX_WORKERS];
+    uint32_t *dest[OB_MAX_WORKERS];
 };
+
 
 // [1BA, Proposed method, 3; Abstract]: for every worker w of one tile,
 //   m_w = beta1 m + (1-beta1) g_w,  x = m_w + e_w (e_w decoded from the
@@ -70,6 +78,7 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
         }
     }
     const int64_t words_per_worker = P.n_pad >> 5;
+    uint32_t *const bits = P.n_shards > 0 ? P.dest[shard_of(tile_id, P.n_shards, P.shard_end)] : P.bits;
     // Pipeline over the workers: the gradient and x_prev slots of worker
     // w + kPackStages - 1 are copied into shared memory (cp.async) while
     // worker w is computed, so HBM stays busy whatever the arithmetic's
@@ -101,7 +110,7 @@ __global__ void __launch_bounds__(kThreads) ob_pack_kernel(const __grid_constant
         const int st = w % kPackStages;
         const float s_prev = P.s_prev[w * P.T + tile.tensor];
         float *xw = P.x + (int64_t)w * P.n_pad + tile.begin;
-        uint32_t *bw = P.bits + (int64_t)w * words_per_worker + (tile.begin >> 5);
+        uint32_t *bw = bits + (int64_t)w * words_per_worker + (tile.begin >> 5);
         double ss[kUnroll];
         uint32_t words[kUnroll];
 #pragma unroll

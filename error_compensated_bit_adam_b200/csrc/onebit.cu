@@ -321,8 +321,15 @@ struct ob_ctx {
     int split_stage = 0;
     // the server chunks this context serves in a split step: flat chunk
     // indices t * W + j in [chunk_lo, chunk_hi), contiguous in layout order
-    // (ob_set_server_shard; all of them by default)
+    // (ob_set_server_shard; all of them by default), shard `shard` of
+    // n_shards
     int chunk_lo = 0, chunk_hi = -1;
+    int n_shards = 1, shard = 0;
+    // split step with peer memory (ob_set_peer_words): every shard's worker
+    // rows and server words, as this process addresses them
+    bool peer = false;
+    std::vector<uint32_t *> peer_bits;
+    std::vector<const uint32_t *> peer_sbits;
     // profiling
     bool profiling = false;
     std::vector<cudaEvent_t> event_pool;
@@ -624,14 +631,35 @@ ob_status launch_pack(ob_ctx *c, const float *const *g, int64_t g_offset, int ti
     return fail_cuda(c, launch(onebit::ob_pack_kernel, pack_geometry(tile_hi - tile_lo), P, c->stream));
 }
 
+int shard_tile_end(const Plan &pl, int G, int q);
+
+// In the split step with peer memory, the update reads each chunk's server
+// words from the process serving it and copies them into this context's.
+void add_peer_sources(const ob_ctx *c, onebit::ApplyParams *A) {
+    if (!c->peer || c->split_stage != 2) return;
+    A->n_shards = c->n_shards;
+    for (int q = 0; q < c->n_shards; ++q) {
+        A->shard_end[q] = shard_tile_end(c->plan, c->n_shards, q);
+        A->src_sbits[q] = c->peer_sbits[q];
+    }
+    A->sbits_copy = c->sbits();
+}
+
 // The gather and update (1-bit LAMB's with layerwise rates when on; then
 // its new ||p||^2 summed per tensor for the next step).
 ob_status launch_apply(ob_ctx *c) {
     if (c->n_tiles() == 0) return OB_OK;
     KernelTimer k(c, OB_K_APPLY);
-    cudaError_t e =
-        c->lamb ? launch(onebit::ob_lamb_apply_kernel, apply_geometry(c), lamb_apply_params(c), c->stream)
-                : launch(onebit::ob_apply_kernel, apply_geometry(c), apply_params(c), c->stream);
+    cudaError_t e;
+    if (c->lamb) {
+        onebit::LambApplyParams L = lamb_apply_params(c);
+        add_peer_sources(c, &L.a);
+        e = launch(onebit::ob_lamb_apply_kernel, apply_geometry(c), L, c->stream);
+    } else {
+        onebit::ApplyParams A = apply_params(c);
+        add_peer_sources(c, &A);
+        e = launch(onebit::ob_apply_kernel, apply_geometry(c), A, c->stream);
+    }
     if (e == cudaSuccess && c->lamb)
         e = launch(onebit::ob_scale_kernel, range_sum_geometry(c->plan.T, 1, c->plan.tensor_max_seg),
                    tensor_sum_params(c, c->partial_w(), 1, c->pnorm()), c->stream);
@@ -909,6 +937,13 @@ void shard_chunks(const Plan &pl, int G, int r, int *lo, int *hi) {
     };
     *lo = cut(r);
     *hi = cut(r + 1);
+}
+
+// One past the last tile of shard q of G (the tiles of its chunks).
+int shard_tile_end(const Plan &pl, int G, int q) {
+    int lo, hi;
+    shard_chunks(pl, G, q, &lo, &hi);
+    return pl.chunk_tile_begin[hi];
 }
 
 // First server word of flat chunk c (n_pad/32 for c == T*W): chunk j of a
@@ -1271,6 +1306,13 @@ ob_status ob_worker_stage(ob_ctx *c, const float *const *d_grads, int w_begin, i
         P.s_prev = c->s_prev() + (size_t)w_begin * T;
         P.partial = c->partial_w() + (size_t)w_begin * nt;
         P.W = w_count;
+        if (c->peer) {  // every chunk's words straight to the process serving it
+            P.n_shards = c->n_shards;
+            for (int q = 0; q < c->n_shards; ++q) {
+                P.shard_end[q] = shard_tile_end(c->plan, c->n_shards, q);
+                P.dest[q] = c->peer_bits[q] + (size_t)w_begin * (n / 32);
+            }
+        }
         KernelTimer k(c, OB_K_PACK);
         const cudaError_t e = launch(onebit::ob_pack_kernel, pack_geometry((int)nt), P, c->stream);
         k.stop();
@@ -1310,7 +1352,36 @@ ob_status ob_set_server_shard(ob_ctx *c, int n_shards, int shard) {
     if (st != OB_OK) return st;
     if (n_shards < 1 || shard < 0 || shard >= n_shards) return OB_ERR_INVALID_ARG;
     if (c->split_stage != 0) return OB_ERR_PHASE;
+    if (c->peer && n_shards != c->n_shards) return OB_ERR_PHASE;  // peers were set for the old split
     shard_chunks(c->plan, n_shards, shard, &c->chunk_lo, &c->chunk_hi);
+    c->n_shards = n_shards;
+    c->shard = shard;
+    return OB_OK;
+}
+
+ob_status ob_set_peer_words(ob_ctx *c, int n_shards, uint32_t *const *d_worker_bits,
+                            const uint32_t *const *d_server_bits) {
+    ob_status st = check_ctx(c);
+    if (st != OB_OK) return st;
+    if (c->split_stage != 0) return OB_ERR_PHASE;
+    if (n_shards == 0) {
+        c->peer = false;
+        return OB_OK;
+    }
+    if (n_shards != c->n_shards || n_shards > OB_MAX_WORKERS || !d_worker_bits || !d_server_bits)
+        return OB_ERR_INVALID_ARG;
+    for (int q = 0; q < n_shards; ++q) {
+        if (!d_worker_bits[q] || !d_server_bits[q]) return OB_ERR_INVALID_ARG;
+        if (!aligned(d_worker_bits[q], 16) || !aligned(d_server_bits[q], 16)) return OB_ERR_ALIGN;
+    }
+    try {
+        host_alloc_point();
+        c->peer_bits.assign(d_worker_bits, d_worker_bits + n_shards);
+        c->peer_sbits.assign(d_server_bits, d_server_bits + n_shards);
+    } catch (const std::bad_alloc &) {
+        return OB_ERR_OOM;
+    }
+    c->peer = true;
     return OB_OK;
 }
 

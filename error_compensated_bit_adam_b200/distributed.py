@@ -20,6 +20,14 @@ whose words are one contiguous range [wb_r, we_r) of the padded layout
     chunks' scales to every other process and receives theirs (about n/8
     bytes in per process).
 
+With peer_words (ob_set_peer_words) the two word exchanges move into the
+kernels instead: the worker stage stores each chunk's words straight into
+the serving process's rows, and the update reads each chunk's server words
+from the serving process (copying them locally); only the worker scales
+and the server scales are still exchanged, and those exchanges also order
+the stages across processes.  The other processes' buffers are mapped into
+each process with CUDA IPC.
+
 Every process ends the step with the same parameters, bit for bit equal to
 one ob_compressed_step over all W workers.  A process's rows of the other
 workers hold only the words of the chunks it serves (the rest is stale),
@@ -131,7 +139,8 @@ class DistributedOneBitAdam:
     (a TorchExchange by default) between the library calls."""
 
     def __init__(self, numel: Sequence[int], W: int, *, rank: int, world: int, exchange=None,
-                 device=None, stream: Optional[torch.cuda.Stream] = None, **hyper):
+                 device=None, stream: Optional[torch.cuda.Stream] = None, peer_words: bool = False,
+                 **hyper):
         if world < 1 or W % world != 0 or not 0 <= rank < world:
             raise ValueError(f"W = {W} workers cannot be split over {world} processes")
         self.rank, self.world = int(rank), int(world)
@@ -152,6 +161,34 @@ class DistributedOneBitAdam:
         sbits, sbits_bytes, sp, sp_bytes = B.ob_server_exchange_buffers(ctx)
         self.server_bits = _view(ws, sbits, sbits_bytes, torch.int32)
         self.server_scales = _view(ws, sp, sp_bytes, torch.float32)
+        self.peer_words = False
+        self._peer_workspaces: List[torch.Tensor] = []
+        if peer_words:
+            self.connect_peers()
+
+    def set_peer_words(self, worker_bits: Sequence[int], server_bits: Sequence[int]) -> None:
+        """Fused word exchanges with the given per-shard buffer addresses
+        (every process's worker_bits and server_bits, as this process
+        addresses them)."""
+        B.ob_set_peer_words(self.opt.ctx, list(worker_bits), list(server_bits))
+        self.peer_words = True
+
+    def connect_peers(self) -> None:
+        """Map every process's workspace into this one with CUDA IPC (the
+        handles travel over the default process group) and turn on the
+        fused word exchanges.  Processes on one node whose GPUs reach each
+        other's memory; not run on more than one GPU here."""
+        import torch.distributed as dist
+        from torch.multiprocessing.reductions import reduce_tensor
+        ws = self.opt.workspace
+        handles = [None] * self.world
+        dist.all_gather_object(handles, reduce_tensor(ws) if self.world > 1 else None)
+        peers = [ws if q == self.rank else h[0](*h[1]) for q, h in enumerate(handles)]
+        self._peer_workspaces = peers                  # keeps the mappings alive
+        bits_off = self.worker_bits.data_ptr() - ws.data_ptr()
+        sbits_off = self.server_bits.data_ptr() - ws.data_ptr()
+        self.set_peer_words([p.data_ptr() + bits_off for p in peers],
+                            [p.data_ptr() + sbits_off for p in peers])
 
     @property
     def params(self) -> torch.Tensor:
@@ -226,14 +263,18 @@ class DistributedOneBitAdam:
 
     def exchange_worker_stage(self, ex) -> None:
         """The worker stage's exchange: each rank's chunks of every worker's
-        words, and all worker scales."""
-        ex.send_worker_chunks(self.worker_bits, self.w_local, self.word_ranges)
+        words (unless the kernel stored them already), and all worker
+        scales."""
+        if not self.peer_words:
+            ex.send_worker_chunks(self.worker_bits, self.w_local, self.word_ranges)
         ex.gather_rows(self.worker_scales, self.w_begin, self.w_local)
 
     def exchange_server_stage(self, ex) -> None:
-        """The server stage's exchange: every rank's server words and chunk
-        scales to every rank."""
-        ex.gather_ranges(self.server_bits, self.word_ranges)
+        """The server stage's exchange: every rank's server words (unless the
+        update reads them from their server) and chunk scales to every
+        rank."""
+        if not self.peer_words:
+            ex.gather_ranges(self.server_bits, self.word_ranges)
         ex.gather_ranges(self.server_scales, self.chunk_ranges)
 
     def step(self, local_grads: Sequence[torch.Tensor]) -> None:
@@ -248,7 +289,9 @@ class DistributedOneBitAdam:
             self.apply_update()
 
     def exchange_bytes(self) -> dict:
-        """Bytes each exchange brings into this process per step."""
+        """Bytes each exchange brings into this process per step (with
+        peer_words the words move inside the kernels: stored by the other
+        processes' worker stages, loaded by this process's update)."""
         others = self.W - self.w_local
         wb, we = self.word_ranges[self.rank]
         T = self.worker_scales.shape[1]
@@ -257,7 +300,8 @@ class DistributedOneBitAdam:
                 "worker_scales": others * T * 4,
                 "server_words": sum(self.word_ranges[q][1] - self.word_ranges[q][0] for q in theirs) * 4,
                 "server_scales": sum(self.chunk_ranges[q][1] - self.chunk_ranges[q][0]
-                                     for q in theirs) * 4}
+                                     for q in theirs) * 4,
+                "words_in_kernels": self.peer_words}
 
     def read(self, kind: int, index: int = 0):
         return self.opt.read(kind, index)
@@ -272,13 +316,20 @@ class LocalRanks:
     rank waits for another's: the ranks' launches are queued one after
     another on the same stream."""
 
-    def __init__(self, numel: Sequence[int], W: int, G: int, device=None, **hyper):
+    def __init__(self, numel: Sequence[int], W: int, G: int, device=None, peer_words: bool = False,
+                 **hyper):
         self.G, self.W = int(G), int(W)
         stream = torch.cuda.current_stream(device)
         self.ranks: List[DistributedOneBitAdam] = [
             DistributedOneBitAdam(numel, W, rank=r, world=G, device=device, stream=stream, **hyper)
             for r in range(G)]
         self.w_local = self.ranks[0].w_local
+        self.peer_words = bool(peer_words)
+        if self.peer_words:  # the "peers" are the other contexts' buffers on this GPU
+            bits = [r.worker_bits.data_ptr() for r in self.ranks]
+            sbits = [r.server_bits.data_ptr() for r in self.ranks]
+            for r in self.ranks:
+                r.set_peer_words(bits, sbits)
 
     def warmup_step(self, all_grads: torch.Tensor) -> None:
         for r in self.ranks:
@@ -333,12 +384,14 @@ class LocalRanks:
         for r in self.ranks:
             r.worker_stage([all_grads[r.w_begin + i] for i in range(r.w_local)])
         if self.G > 1:
-            self._send_worker_chunks()
+            if not self.peer_words:
+                self._send_worker_chunks()
             self._gather_rows("worker_scales")
         for r in self.ranks:
             r.server_stage()
         if self.G > 1:
-            self._gather_ranges("server_bits", "word_ranges")
+            if not self.peer_words:
+                self._gather_ranges("server_bits", "word_ranges")
             self._gather_ranges("server_scales", "chunk_ranges")
         for r in self.ranks:
             r.apply_update()

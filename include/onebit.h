@@ -286,6 +286,33 @@ OB_API ob_status ob_server_exchange_buffers(ob_ctx *ctx, uint32_t **d_sbits, siz
  * unless ob_server_stage came before. */
 OB_API ob_status ob_apply_update(ob_ctx *ctx);
 
+/* The split step with the word exchanges fused into the kernels: the
+ * worker stage's sign words of each chunk are stored straight into the
+ * worker rows of the process serving it, and the update reads each chunk's
+ * server words from the process serving it (copying them into this
+ * context's server words, which the next step's momentum decode reads)
+ * -- [1BA, Proposed method, 4]'s worker stage and gather, with the pack
+ * and the unpack doing the transfers.  d_worker_bits[q] / d_server_bits[q]:
+ * the buffers ob_worker_exchange_buffers / ob_server_exchange_buffers
+ * return in the context serving shard q, as device addresses this process
+ * can store to and load from (the same device, or another GPU's memory
+ * mapped here, e.g. through CUDA IPC, reached with plain loads and
+ * stores); the entry of this context's own shard may be its own buffers.
+ * n_shards must be the shard count given to ob_set_server_shard (0 turns
+ * this off).  With
+ * it on, the caller exchanges only the worker scales (all-gather) and the
+ * server scales (every process's chunk range to every process), each after
+ * the stage that produced them: those exchanges also order the stages
+ * across processes (a process's server stage must start after every
+ * process's worker stage has finished storing into it, and the servers'
+ * words must be complete before any update reads them).  OB_ERR_PHASE while
+ * a split step is open; OB_ERR_INVALID_ARG for a shard count that differs
+ * from the context's or a NULL buffer; OB_ERR_ALIGN for a buffer that is
+ * not 16-byte aligned.  The library cannot check that the addresses point
+ * at the right buffers. */
+OB_API ob_status ob_set_peer_words(ob_ctx *ctx, int n_shards, uint32_t *const *d_worker_bits,
+                                   const uint32_t *const *d_server_bits);
+
 /* Copy one piece of state to host memory.  kind: ob_state_kind.  index:
  * the worker for OB_STATE_E_WORKER / OB_STATE_BITS_WORKER, else 0.  bytes:
  * must equal the size listed with the kind.  Waits for the stream first.

@@ -35,14 +35,14 @@ CASES = {
 }
 
 
-def _run(sizes, W, G, warmup=2, compressed=4, seed=31, orc=False):
+def _run(sizes, W, G, warmup=2, compressed=4, seed=31, orc=False, peer_words=False):
     wl = WL.Workload(f"split-{W}-{G}", tuple((n,) for n in sizes), W, warmup, compressed, seed=seed,
                      zero_fraction=0.2)
     offsets, n_pad = B.ob_layout(wl.numels)
     params = WL.make_params(wl, offsets, n_pad, device="cuda")
     scale = WL.grad_scale_vector(wl, offsets, n_pad, device="cuda")
     ref = OneBitAdam(wl.numels, W, params=params.clone(), **WL.HYPER)
-    ranks = LocalRanks(wl.numels, W, G, **WL.HYPER)
+    ranks = LocalRanks(wl.numels, W, G, peer_words=peer_words, **WL.HYPER)
     run = (oracle.OracleRun(WL.split(params.cpu().numpy(), offsets, wl.numels), W, WL.HYPER)
            if orc else None)
     for r in ranks.ranks:
@@ -76,10 +76,16 @@ def _run(sizes, W, G, warmup=2, compressed=4, seed=31, orc=False):
     return (ref, ranks, run) if orc else (ref, ranks)
 
 
+@pytest.mark.parametrize("peer_words", [False, True], ids=["exchange", "peer-words"])
 @pytest.mark.parametrize("name", list(CASES))
-def test_split_step_equals_one_context(name):
+def test_split_step_equals_one_context(name, peer_words):
+    """Both forms of the word exchanges: by the caller (device copies of
+    the ranges, as NCCL moves them between processes), and inside the
+    kernels (the worker stage storing into the serving rank's rows, the
+    update reading the serving rank's words; here the "peers" are the other
+    contexts' buffers on the same GPU)."""
     sizes, W, G = CASES[name]
-    ref, ranks = _run(sizes, W, G)
+    ref, ranks = _run(sizes, W, G, peer_words=peer_words)
     try:
         want = {k: ref.read(k) for k in (B.OB_STATE_P, B.OB_STATE_M, B.OB_STATE_BITS_SERVER,
                                           B.OB_STATE_S_SERVER, B.OB_STATE_S_WORKER, B.OB_STATE_STEP)}

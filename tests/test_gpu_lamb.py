@@ -150,8 +150,9 @@ def test_lamb_graph_mode_equals_direct_launches():
         b.close()
 
 
+@pytest.mark.parametrize("peer_words", [False, True], ids=["exchange", "peer-words"])
 @pytest.mark.parametrize("G", [2, 4])
-def test_lamb_split_step_equals_one_context(G):
+def test_lamb_split_step_equals_one_context(G, peer_words):
     """The split step with layerwise rates: every rank updates all
     parameters with the same ratios, bit for bit one LAMB context."""
     sizes, W = ((100_003,), (31,), (4097,), (70_000,)), 8
@@ -160,7 +161,7 @@ def test_lamb_split_step_equals_one_context(G):
     params = WL.make_params(wl, offs, n_pad, device="cuda")
     scale = WL.grad_scale_vector(wl, offs, n_pad, device="cuda")
     ref = OneBitAdam(wl.numels, W, params=params.clone(), layerwise=True, **WL.HYPER)
-    ranks = LocalRanks(wl.numels, W, G, layerwise=True, **WL.HYPER)
+    ranks = LocalRanks(wl.numels, W, G, layerwise=True, peer_words=peer_words, **WL.HYPER)
     try:
         for r in ranks.ranks:
             r.params.copy_(params)
