@@ -489,7 +489,8 @@ def run_split(args, world: int, rank: int, dev) -> None:
     offsets, n_pad = B.ob_layout(wl.numels)
     params = WL.make_params(wl, offsets, n_pad, device=dev)
     scale = WL.grad_scale_vector(wl, offsets, n_pad, device=dev)
-    D = DistributedOneBitAdam(wl.numels, wl.W, rank=rank, world=world, device=dev, **WL.HYPER)
+    D = DistributedOneBitAdam(wl.numels, wl.W, rank=rank, world=world, device=dev,
+                              peer_words=args.peer_words and world > 1, **WL.HYPER)
     D.params.copy_(params)
     del params
     wl_local, w0 = D.w_local, D.w_begin
@@ -573,7 +574,10 @@ def run_split(args, world: int, rank: int, dev) -> None:
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
             "data": "synthetic",
             "config": workload_config(wl, n_pad, f"dp{world}: split step, {wl_local} of the W={wl.W} "
-                                                 "workers per GPU, per-chunk NCCL exchange",
+                                                 "workers per GPU, "
+                                                 + ("words stored and loaded by the kernels over "
+                                                    "peer memory, scales over NCCL"
+                                                    if D.peer_words else "per-chunk NCCL exchange"),
                                       len(grads)),
             "exchange_bytes_in_per_rank_per_step": D.exchange_bytes(),
             "roofline": {"bound": "hbm", "kernel": "ob_pack_kernel", "achieved": achieved,
@@ -790,6 +794,9 @@ def main(argv=None):
                          "GPUs through the split step and its NCCL exchange; 'replicas' runs N "
                          "independent copies of the one-GPU step.  '--multi split' with one GPU "
                          "runs the split step's calls without an exchange")
+    ap.add_argument("--peer-words", action="store_true",
+                    help="with the split step on N > 1 GPUs: the kernels store and load the sign "
+                         "words over peer memory (CUDA IPC) instead of NCCL moving them")
     ap.add_argument("--lamb", action="store_true",
                     help="time 1-bit LAMB (layerwise trust ratios, ob_set_layerwise) instead of 1-bit Adam")
     ap.add_argument("--overlap", action="store_true",
