@@ -25,8 +25,9 @@ kernels instead: the worker stage stores each chunk's words straight into
 the serving process's rows, and the update reads each chunk's server words
 from the serving process (copying them locally); only the worker scales
 and the server scales are still exchanged, and those exchanges also order
-the stages across processes.  The other processes' buffers are mapped into
-each process with CUDA IPC.
+the stages across processes; a process's worker rows, its own workers'
+included, then hold only the words of the chunks it serves.  The other
+processes' buffers are mapped into each process with CUDA IPC.
 
 Every process ends the step with the same parameters, bit for bit equal to
 one ob_compressed_step over all W workers.  A process's rows of the other

@@ -305,7 +305,9 @@ OB_API ob_status ob_apply_update(ob_ctx *ctx);
  * the stage that produced them: those exchanges also order the stages
  * across processes (a process's server stage must start after every
  * process's worker stage has finished storing into it, and the servers'
- * words must be complete before any update reads them).  OB_ERR_PHASE while
+ * words must be complete before any update reads them).  A context's
+ * worker rows then hold, for every worker including its own, only the
+ * words of the chunks it serves.  OB_ERR_PHASE while
  * a split step is open; OB_ERR_INVALID_ARG for a shard count that differs
  * from the context's or a NULL buffer; OB_ERR_ALIGN for a buffer that is
  * not 16-byte aligned.  The library cannot check that the addresses point
