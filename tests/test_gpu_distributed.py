@@ -236,6 +236,19 @@ def test_split_step_phase_rules():
         with pytest.raises(B.OnebitError) as e:
             B.ob_set_server_shard(ctx, 2, 2)                   # no such shard
         assert e.value.status == B.OB_ERR_INVALID_ARG
+        bits = opt.worker_bits.data_ptr()
+        sbits = opt.server_bits.data_ptr()
+        for bad, status in ((([bits], [sbits]), B.OB_ERR_INVALID_ARG),       # one shard of two
+                            (([bits, 0], [sbits, sbits]), B.OB_ERR_INVALID_ARG),
+                            (([bits, bits + 4], [sbits, sbits]), B.OB_ERR_ALIGN)):
+            with pytest.raises(B.OnebitError) as e:
+                B.ob_set_peer_words(ctx, *bad)
+            assert e.value.status == status
+        B.ob_set_peer_words(ctx, [bits, bits], [sbits, sbits])
+        with pytest.raises(B.OnebitError) as e:
+            B.ob_set_server_shard(ctx, 1, 0)                   # peers were set for two shards
+        assert e.value.status == B.OB_ERR_PHASE
+        B.ob_set_peer_words(ctx, [], [])                       # off again
         B.ob_set_server_shard(ctx, 1, 0)                       # serve everything again
         B.ob_worker_stage(ctx, [0, 0, 0, 0], 0, 0)             # an empty range is a no-op stage
         B.ob_server_stage(ctx)
