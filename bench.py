@@ -109,18 +109,40 @@ def measured_peaks() -> dict:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled while timing."""
+    """nvidia-smi clocks and throttle reasons, sampled while timing.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    start() launches the sampler and waits for its first sample (nvidia-smi
+    needs about a second to start); mark() and stop() bracket the timed
+    region, and only the samples stamped inside it are reported (or, for a
+    region shorter than one interval, the sample nearest its end)."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    N_FIELDS = 10
 
     def __init__(self, interval_ms=50):
         self.proc = None
         self.path = None
         self.interval_ms = interval_ms
+        self.t_start = None
 
-    def start(self):
+    def _rows(self):
+        import datetime
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) != self.N_FIELDS:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    continue
+                rows.append((ts, parts[1:]))
+        return rows
+
+    def start(self, ready_timeout_s=5.0):
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -128,38 +150,46 @@ class ClockSampler:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  f"-lms", str(self.interval_ms)], stdout=self.out, stderr=subprocess.DEVNULL)
+            t_end = time.time() + ready_timeout_s
+            while time.time() < t_end and self.proc.poll() is None and not self._rows():
+                time.sleep(0.02)
         except Exception:
             self.proc = None
+
+    def mark(self):
+        self.t_start = time.time()
 
     def stop(self):
         if self.proc is None:
             return None
+        t_stop = time.time()
+        time.sleep(2 * self.interval_ms / 1000.0)  # the sample that covers the region's end
         try:
             self.proc.terminate()
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
         self.out.close()
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) == 9:
-                    rows.append(parts)
+        rows = self._rows()
         os.unlink(self.path)
-        if not rows:
+        t_start = self.t_start if self.t_start is not None else t_stop
+        inside = [r for ts, r in rows if t_start <= ts <= t_stop]
+        if not inside:
+            before = [r for ts, r in rows if ts <= t_stop]
+            inside = before[-1:] or [r for _, r in rows][:1]
+        if not inside:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        sm = [float(r[1]) for r in inside if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in inside if r[2].replace(".", "").isdigit()]
         reasons = set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
+        for r in inside:
             for name, val in zip(names, r[5:9]):
                 if val.strip().lower() == "active":
                     reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
-                "samples": len(rows)}
+                "samples": len(inside)}
 
 
 def pick_workload(args) -> WL.Workload:
@@ -523,6 +553,7 @@ def run_split(args, world: int, rank: int, dev) -> None:
         sampler.start()
     barrier(world)
     torch.cuda.synchronize(dev)
+    sampler.mark()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for k in range(args.steps):
@@ -654,6 +685,7 @@ def run_b200(args) -> None:
             sampler.start()
         barrier(world)
         torch.cuda.synchronize(dev)
+        sampler.mark()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for k in range(steps):

@@ -33,6 +33,48 @@ def test_reference_arm_prints_one_line_with_the_contract_keys():
                         "d2h_bytes_per_step": 0}
 
 
+FAKE_SMI = """#!/usr/bin/env python3
+import datetime, sys, time
+while True:
+    ts = datetime.datetime.now().strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+    clk = 1500 if time.time() < float(sys.argv[-1]) else 1965
+    print(f"{ts}, 0, {clk}, 1965, 700.00, 0x4, Not Active, Not Active, Not Active, Active", flush=True)
+    time.sleep(0.02)
+"""
+
+
+def test_clock_sampler_reports_only_the_timed_region(tmp_path, monkeypatch):
+    """The sampler waits for nvidia-smi's first sample, then keeps only the
+    samples stamped between mark() and stop() (a fake nvidia-smi reports
+    1500 MHz before a switch time and 1965 MHz after it)."""
+    import importlib.util
+    import time
+
+    switch = time.time() + 0.6
+    fake = tmp_path / "nvidia-smi"
+    fake.write_text(FAKE_SMI.replace("sys.argv[-1]", repr(str(switch))))
+    fake.chmod(0o755)
+    monkeypatch.setenv("PATH", str(tmp_path) + os.pathsep + os.environ["PATH"])
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+
+    s = bench.ClockSampler(interval_ms=20)
+    s.start()
+    time.sleep(max(0.0, switch - time.time()) + 0.1)
+    s.mark()
+    time.sleep(0.4)
+    c = s.stop()
+    assert c["samples"] >= 5 and c["sm_mhz"] == 1965.0 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"]
+
+    s = bench.ClockSampler(interval_ms=20)       # a region shorter than one interval
+    s.start()
+    s.mark()
+    c = s.stop()
+    assert c["samples"] >= 1
+
+
 def test_reference_arm_other_ranks_exit_without_work():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr
