@@ -349,6 +349,16 @@ class OracleRun:
         return self.o.worker_compress(self.hp["beta1"], self.m[t], g, self.e_w[w][t])
 
     def compressed_step(self, grads: Sequence[Sequence[np.ndarray]]) -> None:
+        """grads[w][t]: worker w's gradient of tensor t."""
+        self.begin_compressed_step()
+        self.worker_stages(lambda w: grads[w], range(self.W))
+        self.end_compressed_step()
+
+    # The compressed step in its phases, for callers that cannot hold every
+    # worker's gradient at once: begin, then the worker stages of any
+    # subsets of the workers (each worker exactly once), then the end (the
+    # server stage and the update).  Same calls, same results.
+    def begin_compressed_step(self) -> None:
         assert self.d is not None, "not frozen"
         T, W = self.T, self.W
         self.bits_w = [[None] * T for _ in range(W)]
@@ -356,10 +366,21 @@ class OracleRun:
         self.sbits = [None] * T
         self.s_srv = np.zeros((T, W), np.float32)
 
+    def worker_stages(self, grads_of, workers) -> None:
+        """Worker stage of each worker w in `workers`, grads_of(w)[t] being
+        its gradient of tensor t."""
+        rows = {w: grads_of(w) for w in workers}
+
         def worker_job(t, w):
-            b, s = self.worker_stage(w, t, grads[w][t])
+            b, s = self.worker_stage(w, t, rows[w][t])
             self.bits_w[w][t] = b
             self.s_w[w, t] = s
+
+        self._run([lambda t=t, w=w: worker_job(t, w) for t in range(self.T) for w in rows])
+
+    def end_compressed_step(self) -> None:
+        T, W = self.T, self.W
+        assert all(b is not None for row in self.bits_w for b in row), "a worker stage is missing"
 
         def server_job(t):
             sb, ss = self.o.server_compress([self.bits_w[w][t] for w in range(W)], self.s_w[:, t],
@@ -375,7 +396,6 @@ class OracleRun:
             self.o.apply_chunk(j, W, self.hp["lr"], self.sbits[t], self.s_srv[t, j], self.d[t],
                                self.p[t], self.m[t])
 
-        self._run([lambda t=t, w=w: worker_job(t, w) for t in range(T) for w in range(W)])
         if self.lamb:  # server stage of every chunk, then each tensor's ratio, then the update
             def srv_job(t, j):
                 bits = [self.bits_w[w][t] for w in range(W)]

@@ -36,12 +36,40 @@ def words_of(flat_words: np.ndarray, offsets, numels):
     return out
 
 
+class DeviceSlices:
+    """One worker's gradient of one tensor as the oracle reads it, copied
+    from the device buffer that the seeded generator filled, slice by slice
+    when sliced (a[a:b]) or whole (np.asarray)."""
+
+    def __init__(self, row: torch.Tensor, offset: int, numel: int):
+        self.row, self.offset, self.numel = row, offset, numel
+
+    def __len__(self):
+        return self.numel
+
+    def __getitem__(self, sl):
+        a, b, step = sl.indices(self.numel)
+        assert step == 1
+        return self.row[self.offset + a:self.offset + b].cpu().numpy()
+
+    def __array__(self, dtype=None, copy=None):
+        a = self[0:self.numel]
+        return a if dtype is None else a.astype(dtype, copy=False)
+
+
 class Pair:
-    """A GPU context and an oracle run over the same workload."""
+    """A GPU context and an oracle run over the same workload.
+
+    stream_workers=K keeps the host from holding every worker's gradient at
+    once (for the largest workloads): the oracle's warmup reads the
+    gradients slice by slice from the device buffer, and its compressed
+    step runs the worker stages K workers at a time, each group's
+    gradients copied to the host just before."""
 
     def __init__(self, wl: WL.Workload, device="cuda", threads: int = 1, hp: Optional[dict] = None,
-                 lamb: bool = False):
+                 lamb: bool = False, stream_workers: Optional[int] = None):
         self.wl = wl
+        self.stream = stream_workers
         self.lamb = lamb
         self.hp = dict(hp or WL.HYPER)
         self.W = wl.W
@@ -61,15 +89,26 @@ class Pair:
         self.gpu.close()
 
     # ------------------------------------------------------------- inputs
-    def next_grads(self):
+    def fill_grads(self):
         WL.fill_grads(self.wl, self.step_index, self.scale, self.grads)
         self.step_index += 1
+
+    def next_grads(self):
+        self.fill_grads()
         host = self.grads.cpu().numpy()
         return [WL.split(host[w], self.offsets, self.numels) for w in range(self.W)]
 
+    def host_row(self, w: int):
+        return WL.split(self.grads[w].cpu().numpy(), self.offsets, self.numels)
+
     # ------------------------------------------------------------- phases
     def warmup_step(self):
-        g = self.next_grads()
+        if self.stream:
+            self.fill_grads()
+            g = [[DeviceSlices(self.grads[w], o, n) for o, n in zip(self.offsets, self.numels)]
+                 for w in range(self.W)]
+        else:
+            g = self.next_grads()
         self.gpu.warmup_step(self.grads)
         self.orc.warmup_step(g)
 
@@ -78,6 +117,14 @@ class Pair:
         self.orc.freeze()
 
     def compressed_step(self):
+        if self.stream:
+            self.fill_grads()
+            self.gpu.step(self.grads)
+            self.orc.begin_compressed_step()
+            for w0 in range(0, self.W, self.stream):
+                self.orc.worker_stages(self.host_row, range(w0, min(self.W, w0 + self.stream)))
+            self.orc.end_compressed_step()
+            return
         g = self.next_grads()
         self.gpu.step(self.grads)
         self.orc.compressed_step(g)
@@ -162,13 +209,14 @@ class Pair:
 
 
 def run_schedule(wl: WL.Workload, synced: bool, warmup: Optional[int] = None,
-                 compressed: Optional[int] = None, threads: int = 1, hp: Optional[dict] = None):
+                 compressed: Optional[int] = None, threads: int = 1, hp: Optional[dict] = None,
+                 stream_workers: Optional[int] = None):
     """Warmup (checked bit for bit every step), freeze (bit for bit), then
     compressed steps: re-synced from the oracle before each step, or left to
     run free.  Returns (pair, list of per-step 'scales exact' flags)."""
     warmup = wl.warmup_steps if warmup is None else warmup
     compressed = wl.compressed_steps if compressed is None else compressed
-    pr = Pair(wl, threads=threads, hp=hp)
+    pr = Pair(wl, threads=threads, hp=hp, stream_workers=stream_workers)
     for _ in range(warmup):
         pr.warmup_step()
         pr.check_warmup_exact()

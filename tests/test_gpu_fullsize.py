@@ -3,8 +3,10 @@ bench.py times (the library chooses tiles and grids from the sizes alone).
 
 Each workload runs at its real size with a shortened schedule.  When the
 host has the RAM for the oracle's whole state, the oracle runs the same
-schedule (its independent per-tensor / per-worker calls run concurrently)
-and every step is compared: warmup and freeze state bit for bit, packed
+schedule (its independent per-tensor / per-worker calls run concurrently;
+where every worker's gradient would not fit on the host at once, the
+oracle reads them from the device buffer a few workers, or a slice, at a
+time) and every step is compared: warmup and freeze state bit for bit, packed
 worker and server words bit for bit, scales within 1e-6, parameters within
 1e-5 relative L2.  Otherwise (the largest sweep points on a small host) the
 run is checked on sampled elements the oracle computes one by one (warmup,
@@ -15,6 +17,8 @@ compresses; words are the signs of x = e + C(x)).
 import gc
 import math
 import os
+
+from typing import Optional
 
 import numpy as np
 import pytest
@@ -40,10 +44,16 @@ def host_available() -> int:
         return 0
 
 
-def oracle_host_bytes(wl: WL.Workload) -> int:
-    # oracle: p, m, v, d, e_s + W errors; gradients of one step (W) on the
-    # host; the GPU read-backs and temporaries: ~4 more vectors
-    return 4 * wl.n * (2 * wl.W + 9)
+def oracle_host_bytes(wl: WL.Workload, stream_workers: Optional[int] = None) -> int:
+    # oracle: p, m, v, d, e_s + W errors; gradients of one step (W, or K
+    # when streamed K workers at a time) on the host; the GPU read-backs and
+    # temporaries: ~4 more vectors
+    held = wl.W if stream_workers is None else min(wl.W, stream_workers)
+    return 4 * wl.n * (wl.W + held + 9)
+
+
+# workers whose gradients the streamed oracle holds at once
+STREAM_WORKERS = 8
 
 
 def shortened(wl: WL.Workload, warmup: int, compressed: int) -> WL.Workload:
@@ -66,8 +76,8 @@ for _w in WL.sweep():
     FULL[_w.name] = shortened(_w, 1, 2)
 
 
-def run_with_oracle(wl: WL.Workload):
-    pr, flags = run_schedule(wl, synced=False, threads=THREADS)
+def run_with_oracle(wl: WL.Workload, stream_workers: Optional[int] = None):
+    pr, flags = run_schedule(wl, synced=False, threads=THREADS, stream_workers=stream_workers)
     try:
         rel = pr.params_rel_l2()
         assert rel <= PARAM_TOL, rel
@@ -156,13 +166,16 @@ def device_room(wl: WL.Workload):
 
 @pytest.mark.parametrize("name", list(FULL))
 def test_full_size_against_oracle(name):
-    """The whole oracle when the host has 1.25x the RAM it needs (every
-    sweep point but (2^29, 32) on a host of about 200 GB), else the
-    sampled check for a flat vector."""
+    """The whole oracle when the host has 1.25x the RAM it needs, with the
+    gradients streamed from the device a few workers at a time when they
+    would not fit all at once ((2^29, 32) on a host of about 200 GB), else
+    the sampled check for a flat vector."""
     wl = FULL[name]
     device_room(wl)
     if host_available() >= 1.25 * oracle_host_bytes(wl):
         run_with_oracle(wl)
+    elif host_available() >= 1.25 * oracle_host_bytes(wl, STREAM_WORKERS):
+        run_with_oracle(wl, stream_workers=STREAM_WORKERS)
     elif wl.n_tensors == 1:
         print(f"{name}: host RAM {host_available() / 1e9:.0f} GB < 1.25 x the oracle's "
               f"{oracle_host_bytes(wl) / 1e9:.0f} GB; sampled check")
