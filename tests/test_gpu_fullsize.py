@@ -172,9 +172,13 @@ def test_full_size_against_oracle(name):
     the sampled check for a flat vector."""
     wl = FULL[name]
     device_room(wl)
-    if host_available() >= 1.25 * oracle_host_bytes(wl):
+    avail = host_available()
+    if avail >= 1.25 * oracle_host_bytes(wl):
+        print(f"{name}: whole oracle, gradients of all workers on the host")
         run_with_oracle(wl)
-    elif host_available() >= 1.25 * oracle_host_bytes(wl, STREAM_WORKERS):
+    elif avail >= 1.25 * oracle_host_bytes(wl, STREAM_WORKERS):
+        print(f"{name}: whole oracle, gradients streamed {STREAM_WORKERS} workers at a time "
+              f"(host RAM {avail / 1e9:.0f} GB)")
         run_with_oracle(wl, stream_workers=STREAM_WORKERS)
     elif wl.n_tensors == 1:
         print(f"{name}: host RAM {host_available() / 1e9:.0f} GB < 1.25 x the oracle's "
@@ -182,3 +186,22 @@ def test_full_size_against_oracle(name):
         run_sampled(wl)
     else:
         pytest.skip(f"host RAM: the oracle needs ~{oracle_host_bytes(wl) / 1e9:.0f} GB")
+
+
+def test_streamed_oracle_equals_whole_oracle():
+    """The streamed mode (the oracle reading the gradients slice by slice in
+    the warmup and a group of workers at a time in the compressed steps; 3
+    workers a group, so the groups do not divide W) on a small workload:
+    the same per-step checks as above, and the same oracle parameters as
+    the whole mode's, bit for bit."""
+    wl = WL.Workload("streamed", ((300_001,), (4_097,)), 16, 2, 3, seed=71)
+    a, _ = run_schedule(wl, synced=False, threads=4, stream_workers=3)
+    b, _ = run_schedule(wl, synced=False, threads=4)
+    try:
+        for t in range(len(wl.numels)):
+            np.testing.assert_array_equal(a.orc.p[t], b.orc.p[t])
+            np.testing.assert_array_equal(a.orc.sbits[t], b.orc.sbits[t])
+        assert a.params_rel_l2() <= PARAM_TOL
+    finally:
+        a.close()
+        b.close()

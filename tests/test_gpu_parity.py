@@ -36,6 +36,11 @@ CASES = {
     "flat-ragged-tail-W3": WL.flat(100_003, 3, 3, 5, seed=23),
     "flat-W5": WL.flat(40_000, 5, 2, 4, seed=24),
     "flat-W1": WL.flat(70_001, 1, 2, 4, seed=25),
+    # W past the 8 tabulated workers, not a power of two (the server stage
+    # adds workers 8.. one by one and divides by W)
+    "flat-W9": WL.flat(90_001, 9, 2, 4, seed=30),
+    "ragged-W12": WL.Workload("ragged-W12", ((50_000,), (4_097,), (0,), (33,)), 12, 2, 4, seed=31,
+                              zero_fraction=0.1),
     # > 2048 tiles per tensor and per server chunk: multi-segment scale sums
     "flat-multi-segment-W2": WL.flat((1 << 24) + 12_345, 2, 1, 2, seed=29),
 }
@@ -59,7 +64,7 @@ def test_free_running_steps_stay_within_tolerance(name):
         pr.close()
 
 
-@pytest.mark.parametrize("W", [2, 8, 32, 64])
+@pytest.mark.parametrize("W", [2, 8, 24, 32, 48, 64])
 def test_sweep_small_n(W):
     wl = WL.flat(1 << 20, W, 2, 3, seed=26, name=f"sweep-small-W{W}")
     pr, flags = run_schedule(wl, synced=False)
