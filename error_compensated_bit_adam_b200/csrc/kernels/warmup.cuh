@@ -84,16 +84,23 @@ __global__ void __launch_bounds__(kThreads) ob_warmup_kernel(const __grid_consta
 __global__ void __launch_bounds__(kThreads) ob_freeze_kernel(const Tile *tiles, float *v, float bc2,
                                                              float eps) {
     const Tile tile = tiles[blockIdx.x];
+    // every slot's load first, so that the four are in flight together
+    // while the divides and square roots run
+    float4 x[kUnroll];
+    int real[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
         const int off = 4 * ((int)threadIdx.x + kThreads * u);
-        const int real = slot_real(tile.count, off);
-        if (real == 0) continue;
-        float4 x = ld_stream(v + tile.begin + off);
+        real[u] = slot_real(tile.count, off);
+        x[u] = real[u] > 0 ? ld_stream(v + tile.begin + off) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        if (real[u] == 0) continue;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
-            if (k < real) set(x, k, __fadd_rn(__fsqrt_rn(__fdiv_rn(get(x, k), bc2)), eps));
-        st_stream(v + tile.begin + off, x);
+            if (k < real[u]) set(x[u], k, __fadd_rn(__fsqrt_rn(__fdiv_rn(get(x[u], k), bc2)), eps));
+        st_stream(v + tile.begin + 4 * ((int)threadIdx.x + kThreads * u), x[u]);
     }
 }
 
