@@ -441,14 +441,14 @@ dim3 grid1(int n) { return dim3((unsigned)n); }
 
 // ---------------------------------------------------------------- launches
 //
-// The three kernels of a compressed step, each with its parameters built by
+// The five launches of a compressed step (worker stage, worker scales,
+// server stage, server scales, update), each with its parameters built by
 // one function, so direct launches and the CUDA-graph nodes of graph mode
 // are the same launches.
 
-// Worker scales, finished by the worker-stage kernel: ranges = tensors,
-// one row per worker, scale (t, w) at s_prev[w * T + t].
 // Range sums of per-tile partial sums (ob_scale_kernel): the worker and
-// server scales, and plain sums for 1-bit LAMB's norms.
+// server scales, and plain sums for 1-bit LAMB's norms.  Worker scales:
+// ranges = tensors, one row per worker, scale (t, w) at s_prev[w * T + t].
 onebit::ScaleParams worker_scale_params(const ob_ctx *c) {
     onebit::ScaleParams P{};  // zeroed, padding too: compared bytewise in graph mode
     P.partial = c->partial_w();

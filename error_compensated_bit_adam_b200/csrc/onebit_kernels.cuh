@@ -2,21 +2,22 @@
 //
 // The compression-phase step of 1-bit Adam ("1-bit Adam: Communication
 // Efficient Large-Scale Training with Adam's Convergence Speed", review
-// page, sections "Abstract" and "Proposed method") as three HBM-streaming
-// kernels over a list of 4096-element tiles, each launched so that it may
+// page, sections "Abstract" and "Proposed method") as five HBM-streaming
+// launches over a list of 4096-element tiles, each launched so that it may
 // start while the one before it finishes (programmatic dependent launch):
 //
-//   ob_pack_kernel          worker stage, all W workers of a tile per CTA;
-//                           its last CTAs per tensor finish the worker scales
-//   ob_server_kernel        server stage of a tile; its last CTAs per chunk
-//                           finish the server scales
+//   ob_pack_kernel          worker stage, all W workers of a tile per CTA
+//   ob_scale_kernel         the worker scales from the per-tile sums
+//   ob_server_kernel        server stage of a tile (the first 8 workers'
+//                           sequential sums from a per-tile table)
+//   ob_scale_kernel         the server scales from the per-tile sums
 //   ob_apply_kernel         gather, decode, preconditioned update
 //
 // plus the warmup Adam step, the freeze and an error decoder used when the
 // host reads state, and the 1-bit LAMB variants (kernels/lamb.cuh: the
-// warmup in two passes, the norms, the update with layerwise rates).  No step is a dense contraction, so no tensor cores:
-// every kernel is a stream of coalesced 16-byte loads and stores, bound by
-// HBM bandwidth.
+// warmup in two passes, the norms, the update with layerwise rates).  No
+// step is a dense contraction, so no tensor cores: every kernel is a stream
+// of coalesced 16- or 32-byte loads and stores, bound by HBM bandwidth.
 //
 // Numerics.  Every fp32 operation is written with an explicit
 // round-to-nearest intrinsic (__fmul_rn, __fadd_rn, __fsub_rn, __fdiv_rn,
