@@ -83,6 +83,10 @@ EDGE = {
     "fewer-words-than-servers": ((100,), 8),
     "many-workers-tiny": ((300, 7), 64),
     "tile-boundaries": ((4095, 4096, 4097, 8192 + 1), 2),
+    # the server stage's table and 55 workers added one by one, W not a
+    # power of two; and 17 workers over ragged tensors
+    "workers-63": ((5_000, 33), 63),
+    "workers-17-ragged": ((12_345, 4_097, 1, 0), 17),
 }
 
 
