@@ -51,14 +51,17 @@ GRAD_SETS = 2
 
 # ----------------------------------------------------------------- helpers
 
-def algorithmic_bytes(n_real: int, W: int) -> dict:
+def algorithmic_bytes(n_real: int, W: int, lamb: bool = False) -> dict:
     """Bytes each kernel of a steady-state compressed step must move, per
     real parameter, in this formulation (errors stored as (x, s) and the
     momentum as last step's server words and scales):
       pack    1/8 (server words -> m) + W (4 g + 4 x_prev + 4 x) + W/8 (words)
       server  W/8 (words) + 4 (y_prev) + 4 (y) + 1/8 (words)
-      apply   1/8 (words) + 4 (d) + 8 (p read and write)
+      apply   1/8 (words) + 4 (d) + 8 (p read and write)   (1-bit LAMB's
+              update the same, plus per-tile sums of ~0)
       warmup  4W (g) + 24 (m, v, p read and write)   [pre-path]
+              1-bit LAMB: 4W + 20 (moments: g, m, v, p read; m, v
+              written) + 16 (step: m, v, p read; p written)
       freeze  8 (v read, d written)                  [pre-path]
     The scale kernels move ~0.  'model' is the dense-momentum byte model
     12W + W/4 + 28.25 (126.25 B at W=8) the effective-bandwidth target is
@@ -70,7 +73,16 @@ def algorithmic_bytes(n_real: int, W: int) -> dict:
             "step": pack + server + apply, "model": n_real * (12 * W + W / 4 + 28.25),
             # the untimed pre-path: Adam reads W gradients and reads and
             # writes m, v and p; the freeze reads v and writes d in its place
-            "ob_warmup_kernel": n_real * (4 * W + 24), "ob_freeze_kernel": n_real * 8}
+            "ob_warmup_kernel": n_real * (4 * W + (36 if lamb else 24)), "ob_freeze_kernel": n_real * 8}
+
+
+# With 1-bit LAMB the warmup and update slots of the profiling counters time
+# LAMB's kernels: their DRAM traffic is looked up under LAMB's own entries.
+LAMB_TRAFFIC_KEYS = {"ob_warmup_kernel": "ob_lamb_warmup", "ob_apply_kernel": "ob_lamb_apply_kernel"}
+
+
+def traffic_key(name: str, lamb: bool) -> str:
+    return LAMB_TRAFFIC_KEYS.get(name, name) if lamb else name
 
 
 def kernel_sources_sha256(files) -> str:
@@ -714,7 +726,7 @@ def run_b200(args) -> None:
 
     # roofline of the dominant kernel, from its own events over the timed region
     peak = measured_peaks()
-    algo = algorithmic_bytes(wl.n, wl.W)
+    algo = algorithmic_bytes(wl.n, wl.W, lamb=args.lamb)
     pack_ms, pack_n = prof["ob_pack_kernel"]
     pack_avg_s = pack_ms / 1e3 / max(1, pack_n)
     achieved = algo["ob_pack_kernel"] / pack_avg_s / 1e9
@@ -730,7 +742,7 @@ def run_b200(args) -> None:
             if name in algo:
                 entry["gbs"] = algo[name] / (kms / args.steps / 1e3) / 1e9
                 entry["algorithmic_bytes_per_launch"] = algo[name]
-                entry["traffic"] = measured_traffic(name, wl.n, wl.W)
+                entry["traffic"] = measured_traffic(traffic_key(name, args.lamb), wl.n, wl.W)
             per_kernel[name] = entry
 
     # the pre-path (full-precision Adam warmup and the freeze), timed by the
@@ -744,7 +756,7 @@ def run_b200(args) -> None:
             pre_path[name] = {"launches": cnt, "avg_launch_ms": kms / cnt, "gbs": gbs,
                               "frac_of_measured_hbm": gbs / peak["hbm_gbs"],
                               "algorithmic_bytes_per_launch": algo[name],
-                              "traffic": measured_traffic(name, wl.n, wl.W)}
+                              "traffic": measured_traffic(traffic_key(name, args.lamb), wl.n, wl.W)}
 
     # end to end: host gradients in pinned memory, copied in every step, and
     # the step's server scales read back, through ob_compressed_step_host
