@@ -70,6 +70,7 @@ __all__ = [name for name in EXPORTS] + [
     "OB_STATE_P", "OB_STATE_M", "OB_STATE_V", "OB_STATE_D", "OB_STATE_E_WORKER",
     "OB_STATE_E_SERVER", "OB_STATE_S_WORKER", "OB_STATE_S_SERVER", "OB_STATE_BITS_WORKER",
     "OB_STATE_BITS_SERVER", "OB_STATE_STEP", "OB_STATE_RATIO",
+    "OB_LAYERWISE_OFF", "OB_LAYERWISE_STEP", "OB_LAYERWISE_FROZEN", "layerwise_mode",
     "OB_K_WARMUP", "OB_K_FREEZE", "OB_K_PACK", "OB_K_PACK_SCALE", "OB_K_SERVER",
     "OB_K_SERVER_SCALE", "OB_K_APPLY", "OB_NUM_KERNELS",
 ]
@@ -271,8 +272,25 @@ def ob_set_lr(ctx: int, lr: float) -> None:
     _check(lib().ob_set_lr(ctx, float(lr)), "ob_set_lr")
 
 
-def ob_set_layerwise(ctx: int, on: bool) -> None:
-    _check(lib().ob_set_layerwise(ctx, 1 if on else 0), "ob_set_layerwise")
+# ob_set_layerwise modes (include/onebit.h)
+OB_LAYERWISE_OFF, OB_LAYERWISE_STEP, OB_LAYERWISE_FROZEN = 0, 1, 2
+
+
+def layerwise_mode(mode) -> int:
+    """An OB_LAYERWISE_* mode from an int, a bool (True: per-step ratios) or
+    a name ("off", "step", "frozen")."""
+    if isinstance(mode, bool) or mode is None:
+        return OB_LAYERWISE_STEP if mode else OB_LAYERWISE_OFF
+    if isinstance(mode, str):
+        names = {"off": OB_LAYERWISE_OFF, "step": OB_LAYERWISE_STEP, "frozen": OB_LAYERWISE_FROZEN}
+        if mode not in names:
+            raise ValueError(f"layerwise mode {mode!r}: one of {sorted(names)}")
+        return names[mode]
+    return int(mode)
+
+
+def ob_set_layerwise(ctx: int, mode) -> None:
+    _check(lib().ob_set_layerwise(ctx, layerwise_mode(mode)), "ob_set_layerwise")
 
 
 def ob_graph_enable(ctx: int, on: bool) -> None:

@@ -11,6 +11,9 @@
 // u being Adam's direction in the warmup and m_hat / d in the compression
 // phase (m_hat the decoded averaged momentum every worker holds after the
 // gather, d the frozen denominator); the ratio is recomputed every step.
+// The other reading, the ratios of the last warmup step kept at the freeze
+// like the variance, makes the compressed update read the stored ratio
+// (LambApplyParams::fixed_ratio) and needs none of the norms below.
 //
 // In the compression phase ||u||^2 = sum_j s'_j^2 D_j over the tensor's
 // server chunks j, with D_j = sum over the chunk of (1/d)^2: d is frozen,
@@ -178,8 +181,9 @@ struct LambApplyParams {
     const int *tensor_tile_begin;  // [T+1]
     const double *pnorm;  // [T]: ||p||^2 before this step
     const double *dnorm;  // [T][W]: D_j
-    float *ratio;         // [T] out
+    float *ratio;         // [T] out (in, when fixed_ratio)
     double *partial;      // [n_tiles]: per tile, sum of the new p^2 (the next step's ||p||^2)
+    int fixed_ratio;      // the ratios kept at the freeze: read ratio, no norms, no partial
 };
 
 // [1BA, Proposed method, 1-2] with the 1-bit LAMB page's layerwise rates:
@@ -196,6 +200,17 @@ __global__ void __launch_bounds__(kThreads) ob_lamb_apply_kernel(const __grid_co
     grid_dependency_wait();
     allow_dependent_launch();
     const int t = tile.tensor, W = P.a.W;
+    const bool peer = P.a.n_shards > 0;
+    const uint32_t *sbits = peer ? P.a.src_sbits[shard_of(tile_id, P.a.n_shards, P.a.shard_end)] : P.a.sbits;
+    uint32_t *copy = peer ? P.a.sbits_copy : nullptr;
+    if (P.fixed_ratio) {  // the ratio kept at the freeze
+        const float lr_t = __fmul_rn(P.a.lr, P.ratio[t]);
+        if (tile.count == kTile)
+            apply_tile<true, false>(P.a, tile, sd, spp, lr_t, sbits, copy);
+        else
+            apply_tile<false, false>(P.a, tile, sd, spp, lr_t, sbits, copy);
+        return;
+    }
     double u_sq = 0.0;
     for (int j = 0; j < W; ++j) {
         const double s = (double)P.a.sp[t * W + j];
@@ -205,9 +220,6 @@ __global__ void __launch_bounds__(kThreads) ob_lamb_apply_kernel(const __grid_co
     if (threadIdx.x == 0 && tile_id == P.tensor_tile_begin[t]) P.ratio[t] = ratio;
     const float lr_t = __fmul_rn(P.a.lr, ratio);
     double pp;
-    const bool peer = P.a.n_shards > 0;
-    const uint32_t *sbits = peer ? P.a.src_sbits[shard_of(tile_id, P.a.n_shards, P.a.shard_end)] : P.a.sbits;
-    uint32_t *copy = peer ? P.a.sbits_copy : nullptr;
     if (tile.count == kTile)
         pp = apply_tile<true, true>(P.a, tile, sd, spp, lr_t, sbits, copy);
     else

@@ -312,9 +312,11 @@ struct ob_ctx {
     bool m_dense = true;
     bool use_graph = true;  // graph mode (ob_graph_enable); used while the stream is not captured
     StepGraph graph;
-    // 1-bit LAMB (ob_set_layerwise): layerwise trust ratios; the norms the
+    // 1-bit LAMB (ob_set_layerwise): layerwise trust ratios, recomputed every
+    // step or (lamb_frozen) kept from the last warmup step; the norms the
     // compressed update needs are valid unless p or d changed otherwise
     bool lamb = false;
+    bool lamb_frozen = false;
     bool pnorm_valid = false, dnorm_valid = false;
     bool broken = false;
     // split step: 0 idle, 1 after ob_worker_stage, 2 after ob_server_stage
@@ -582,6 +584,7 @@ onebit::LambApplyParams lamb_apply_params(const ob_ctx *c) {
     P.dnorm = c->dnorm();
     P.ratio = c->ratio();
     P.partial = c->partial_w();
+    P.fixed_ratio = c->lamb_frozen ? 1 : 0;
     return P;
 }
 
@@ -660,7 +663,7 @@ ob_status launch_apply(ob_ctx *c) {
         add_peer_sources(c, &A);
         e = launch(onebit::ob_apply_kernel, apply_geometry(c), A, c->stream);
     }
-    if (e == cudaSuccess && c->lamb)
+    if (e == cudaSuccess && c->lamb && !c->lamb_frozen)
         e = launch(onebit::ob_scale_kernel, range_sum_geometry(c->plan.T, 1, c->plan.tensor_max_seg),
                    tensor_sum_params(c, c->partial_w(), 1, c->pnorm()), c->stream);
     k.stop();
@@ -699,7 +702,7 @@ ob_status launch_lamb_norms(ob_ctx *c, bool want_d, bool want_p) {
 
 // Before a 1-bit LAMB compressed step: the norms its update reads.
 ob_status ensure_lamb_norms(ob_ctx *c) {
-    if (!c->lamb) return OB_OK;
+    if (!c->lamb || c->lamb_frozen) return OB_OK;  // kept ratios need no norms
     return launch_lamb_norms(c, !c->dnorm_valid, !c->pnorm_valid);
 }
 
@@ -784,8 +787,9 @@ ob_status build_graph(ob_ctx *c, const float *const *g) {
     if (nt > 0) {
         if (sg.lamb) {
             add((void *)onebit::ob_lamb_apply_kernel, apply_geometry(c), &sg.lamb_apply, &sg.apply_node);
-            add((void *)onebit::ob_scale_kernel, range_sum_geometry(c->plan.T, 1, c->plan.tensor_max_seg),
-                &pn, &n_pn);
+            if (!c->lamb_frozen)
+                add((void *)onebit::ob_scale_kernel, range_sum_geometry(c->plan.T, 1, c->plan.tensor_max_seg),
+                    &pn, &n_pn);
         } else {
             add((void *)onebit::ob_apply_kernel, apply_geometry(c), &sg.apply, &sg.apply_node);
         }
@@ -1241,7 +1245,7 @@ ob_status ob_freeze_variance(ob_ctx *c) {
     if ((st = fail_cuda(c, e)) != OB_OK) return st;
     c->frozen = true;
     c->dnorm_valid = false;
-    if (c->lamb && (st = launch_lamb_norms(c, true, true)) != OB_OK) return st;
+    if (c->lamb && !c->lamb_frozen && (st = launch_lamb_norms(c, true, true)) != OB_OK) return st;
     return OB_OK;
 }
 
@@ -1491,9 +1495,11 @@ ob_status ob_apply_update(ob_ctx *c) {
     return OB_OK;
 }
 
-ob_status ob_set_layerwise(ob_ctx *c, int on) {
+ob_status ob_set_layerwise(ob_ctx *c, int mode) {
     ob_status st = check_ctx(c);
     if (st != OB_OK) return st;
+    if (mode != OB_LAYERWISE_OFF && mode != OB_LAYERWISE_STEP && mode != OB_LAYERWISE_FROZEN)
+        return OB_ERR_INVALID_ARG;
     if (c->t_warmup != 0 || c->t_compressed != 0 || c->frozen || c->split_stage != 0)
         return OB_ERR_PHASE;
     DeviceGuard dg(c->device);
@@ -1508,7 +1514,8 @@ ob_status ob_set_layerwise(ob_ctx *c, int on) {
     } catch (const std::bad_alloc &) {
         return OB_ERR_OOM;
     }
-    c->lamb = on != 0;
+    c->lamb = mode != OB_LAYERWISE_OFF;
+    c->lamb_frozen = mode == OB_LAYERWISE_FROZEN;
     c->pnorm_valid = c->dnorm_valid = false;
     return OB_OK;
 }
@@ -1676,6 +1683,10 @@ ob_status ob_write_state(ob_ctx *c, int kind, int index, const void *host_src, s
     case OB_STATE_E_SERVER:
         dst = c->y();
         e = cudaMemsetAsync(c->sp_prev(), 0, (size_t)c->plan.T * c->plan.W * 4, c->stream);
+        break;
+    case OB_STATE_RATIO:  // state only when the ratios are kept at the freeze
+        if (!c->lamb_frozen) return OB_ERR_INVALID_ARG;
+        dst = c->ratio();
         break;
     default:
         return OB_ERR_INVALID_ARG;

@@ -30,14 +30,16 @@ class OneBitAdam:
     n_padded elements in the padded layout (see ``layout``), updated in
     place; a zero tensor is made if omitted.  Gradients are passed as a
     [W, n_padded] float32 CUDA tensor or a list of W such vectors.
-    layerwise=True runs 1-bit LAMB instead (ob_set_layerwise): every
-    tensor's step scaled by its trust ratio ||p|| / ||u||.
+    layerwise=True (or "step") runs 1-bit LAMB instead (ob_set_layerwise):
+    every tensor's step scaled by its trust ratio ||p|| / ||u||, recomputed
+    every step; layerwise="frozen" keeps the last warmup step's ratios from
+    the freeze on.
     """
 
     def __init__(self, numel: Sequence[int], W: int, *, beta1: float = 0.9, beta2: float = 0.999,
                  eps: float = 1e-8, lr: float = 1e-4, params: Optional[torch.Tensor] = None,
                  device: Union[str, torch.device, None] = None,
-                 stream: Optional[torch.cuda.Stream] = None, layerwise: bool = False):
+                 stream: Optional[torch.cuda.Stream] = None, layerwise: Union[bool, str] = False):
         self.numel = [int(n) for n in numel]
         self.W = int(W)
         self.offsets, self.n_padded = B.ob_layout(self.numel)
@@ -60,8 +62,8 @@ class OneBitAdam:
             self.ctx = B.ob_create(self.numel, self.W, beta1, beta2, eps, lr, params.data_ptr(),
                                    self.workspace.data_ptr(), self.workspace_bytes,
                                    self.stream.cuda_stream)
-            if layerwise:
-                B.ob_set_layerwise(self.ctx, True)
+            if B.layerwise_mode(layerwise) != B.OB_LAYERWISE_OFF:
+                B.ob_set_layerwise(self.ctx, layerwise)
 
     # ------------------------------------------------------------ helpers
     def layout(self):

@@ -96,7 +96,8 @@ typedef enum ob_state_kind {
     OB_STATE_STEP = 10,       /* int64[3]: {warmup steps taken, compressed steps taken, frozen} rw */
     OB_STATE_RATIO = 11       /* last step's 1-bit LAMB trust ratios, float[n_tensors] (1 while
                                  layerwise rates are off, before the first step, for empty
-                                 tensors)                                                       r  */
+                                 tensors); written only in OB_LAYERWISE_FROZEN, where they
+                                 are state (the ratios kept at the freeze)                     r  */
 } ob_state_kind;
 
 /* Kernels timed by the profiling counters (ob_profile_read). */
@@ -330,23 +331,33 @@ OB_API ob_status ob_read_state(ob_ctx *ctx, int kind, int index, void *host_dst,
  * Waits for the copy to finish. */
 OB_API ob_status ob_write_state(ob_ctx *ctx, int kind, int index, const void *host_src, size_t bytes);
 
-/* 1-bit LAMB: layerwise adaptive learning rates on (on != 0) or off (the
- * default, 1-bit Adam).  The 1-bit LAMB review page ("1-bit LAMB:
- * Communication Efficient Large-Scale Large-Batch Training with LAMB's
- * Convergence Speed", Abstract) keeps LAMB's layerwise rates while the
- * momentum is exchanged compressed; it prints no update rule, and the
- * reading taken is LAMB's trust ratio per tensor,
+/* 1-bit LAMB: layerwise adaptive learning rates.  The 1-bit LAMB review
+ * page ("1-bit LAMB: Communication Efficient Large-Scale Large-Batch
+ * Training with LAMB's Convergence Speed", Abstract) keeps LAMB's
+ * layerwise rates while the momentum is exchanged compressed; it prints no
+ * update rule.  The rate taken is LAMB's trust ratio per tensor,
  *   ratio_t = ||p_t|| / ||u_t||   (1 when either norm is 0),
- * recomputed every step, scaling that tensor's step: p -= (lr ratio_t) u.
- * In the warmup u is Adam's direction m_hat / (sqrt(v_hat) + eps); in the
- * compression phase u = m_hat / d, m_hat the momentum decoded from the
- * compressed exchange (the same on every worker) and d the frozen
- * denominator.  Everything else (the compressed exchange, the errors, the
- * freeze) is 1-bit Adam's.  The trust ratios are read as OB_STATE_RATIO.
- * Only before the first step: OB_ERR_PHASE afterwards.  The ratios are
- * rounded from fp64 sums of squares taken in an order of the GPU's own, so
- * they can differ from a sequential evaluation in the last place. */
-OB_API ob_status ob_set_layerwise(ob_ctx *ctx, int on);
+ * scaling that tensor's step: p -= (lr ratio_t) u.  In the warmup u is
+ * Adam's direction m_hat / (sqrt(v_hat) + eps), the ratio recomputed every
+ * step.  In the compression phase, mode
+ *   OB_LAYERWISE_STEP    recomputes it every step with u = m_hat / d, m_hat
+ *                        the momentum decoded from the compressed exchange
+ *                        (the same on every worker), d the frozen
+ *                        denominator;
+ *   OB_LAYERWISE_FROZEN  keeps the last warmup step's ratios from the
+ *                        freeze on, as the variance is kept (they are then
+ *                        state: OB_STATE_RATIO can be written, for resume);
+ *   OB_LAYERWISE_OFF     (the default) is 1-bit Adam.
+ * Everything else (the compressed exchange, the errors, the freeze) is
+ * 1-bit Adam's.  The trust ratios are read as OB_STATE_RATIO.  Only before
+ * the first step: OB_ERR_PHASE afterwards; another mode OB_ERR_INVALID_ARG.
+ * The ratios are rounded from fp64 sums of squares taken in an order of
+ * the GPU's own, so they can differ from a sequential evaluation in the
+ * last place. */
+#define OB_LAYERWISE_OFF 0
+#define OB_LAYERWISE_STEP 1
+#define OB_LAYERWISE_FROZEN 2
+OB_API ob_status ob_set_layerwise(ob_ctx *ctx, int mode);
 
 /* Set the learning rate used by the following warmup and compressed steps
  * (learning-rate schedules).  OB_ERR_INVALID_ARG for a non-finite lr. */

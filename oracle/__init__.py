@@ -263,14 +263,22 @@ class OracleRun:
     lamb=True runs 1-bit LAMB: the warmup and the update scale each
     tensor's step by its trust ratio (kept in ``ratio`` after each step);
     the warmup then runs one call per tensor, the compressed step the
-    server stage of every chunk before any update.
+    server stage of every chunk before any update.  With lamb_frozen=True
+    (the other reading of the 1-bit LAMB page) the ratios are those of the
+    last warmup step, kept at the freeze like the variance, and the
+    compressed steps use them instead of recomputing them.
     """
 
     SLICE = 1 << 22  # elements per warmup/freeze call when threaded
 
     def __init__(self, params: Sequence[np.ndarray], W: int, hp: dict,
-                 oracle: Optional[Oracle] = None, threads: int = 1, lamb: bool = False):
+                 oracle: Optional[Oracle] = None, threads: int = 1, lamb: bool = False,
+                 lamb_frozen: bool = False):
+        if lamb_frozen and not lamb:
+            raise ValueError("lamb_frozen needs lamb")
         self.lamb = bool(lamb)
+        self.lamb_frozen = bool(lamb_frozen)
+        self.frozen_ratio: Optional[np.ndarray] = None  # [T] the ratios kept at the freeze
         self.ratio: Optional[np.ndarray] = None  # [T] trust ratios of the last step (LAMB)
         self.threads = max(1, int(threads))
         self.o = oracle or default()
@@ -339,6 +347,8 @@ class OracleRun:
             self.d[t][a:b] = self.o.freeze(self.t_warmup, self.hp, self.v[t][a:b])
         self._run([lambda t=t, a=a, b=b: job(t, a, b)
                    for t in range(self.T) for a, b in self._slices(self.numel[t])])
+        if self.lamb_frozen:  # the last warmup step's trust ratios, kept
+            self.frozen_ratio = np.array(self.ratio, np.float32, copy=True)
         # e_w = 0, e_s = 0 (fresh zero arrays: their pages are only touched
         # when the first compressed step writes them)
         self.e_w = [[np.zeros(n, np.float32) for n in self.numel] for _ in range(self.W)]
@@ -405,12 +415,15 @@ class OracleRun:
             for t in range(T):
                 self.sbits[t] = np.zeros(self.o.num_words(self.numel[t]), np.uint32)
             self._run([lambda t=t, j=j: srv_job(t, j) for t in range(T) for j in range(W)])
-            self.ratio = np.zeros(T, np.float32)
+            if self.lamb_frozen:
+                self.ratio = self.frozen_ratio.copy()
+            else:
+                self.ratio = np.zeros(T, np.float32)
 
-            def ratio_job(t):
-                self.ratio[t] = self.o.lamb_compressed_ratio(W, self.sbits[t], self.s_srv[t],
-                                                             self.d[t], self.p[t])
-            self._run([lambda t=t: ratio_job(t) for t in range(T)])
+                def ratio_job(t):
+                    self.ratio[t] = self.o.lamb_compressed_ratio(W, self.sbits[t], self.s_srv[t],
+                                                                 self.d[t], self.p[t])
+                self._run([lambda t=t: ratio_job(t) for t in range(T)])
             self._run([lambda t=t, j=j: self.o.lamb_apply_chunk(
                 j, W, self.hp["lr"], self.ratio[t], self.sbits[t], self.s_srv[t, j], self.d[t],
                 self.p[t], self.m[t]) for t in range(T) for j in range(W)])

@@ -67,7 +67,7 @@ class Pair:
     gradients copied to the host just before."""
 
     def __init__(self, wl: WL.Workload, device="cuda", threads: int = 1, hp: Optional[dict] = None,
-                 lamb: bool = False, stream_workers: Optional[int] = None):
+                 lamb=False, stream_workers: Optional[int] = None):
         self.wl = wl
         self.stream = stream_workers
         self.lamb = lamb
@@ -78,9 +78,12 @@ class Pair:
         self.dev = torch.device(device)
         params = WL.make_params(wl, self.offsets, self.n_pad, device=self.dev)
         self.scale = WL.grad_scale_vector(wl, self.offsets, self.n_pad, device=self.dev)
+        # lamb: False (1-bit Adam), True or "step" (1-bit LAMB, ratios every
+        # step) or "frozen" (1-bit LAMB, ratios kept at the freeze)
         self.gpu = OneBitAdam(self.numels, wl.W, params=params.clone(), layerwise=lamb, **self.hp)
         self.orc = oracle.OracleRun(WL.split(params.cpu().numpy(), self.offsets, self.numels), wl.W,
-                                    self.hp, threads=threads, lamb=lamb)
+                                    self.hp, threads=threads, lamb=bool(lamb),
+                                    lamb_frozen=lamb == "frozen")
         del params
         self.grads = torch.empty((wl.W, self.n_pad), dtype=torch.float32, device=self.dev)
         self.step_index = 0
@@ -139,6 +142,8 @@ class Pair:
         for w in range(self.W):
             self.gpu.write(B.OB_STATE_E_WORKER, w, pad(o.e_w[w]))
         self.gpu.write(B.OB_STATE_E_SERVER, 0, pad(o.e_s))
+        if o.lamb_frozen and o.frozen_ratio is not None:   # the kept ratios are state
+            self.gpu.write(B.OB_STATE_RATIO, 0, o.frozen_ratio)
 
     # ------------------------------------------------------------ readers
     def read_tensors(self, kind, index=0):

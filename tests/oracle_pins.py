@@ -363,11 +363,12 @@ def _unpack_bytes(buf: bytes, count: int) -> np.ndarray:
     return np.array(codes, F64)
 
 
-def brute_force_step(W, m, d, p, grads, e_w, e_s, lamb=False, lr=None):
+def brute_force_step(W, m, d, p, grads, e_w, e_s, lamb=False, lr=None, ratio=None):
     """One compressed step as W workers and W servers exchanging byte
     messages, in float64.  Returns a dict of results and the bytes sent.
     lamb: the update is 1-bit LAMB's, scaled by the trust ratio
-    ||p|| / ||m_hat / d|| (1 when a norm is 0)."""
+    ||p|| / ||m_hat / d|| (1 when a norm is 0), or by `ratio` when given
+    (the ratio kept at the freeze)."""
     n = m.size
     b1 = F64(F32(HP["beta1"]))
     lr = F64(F32(HP["lr"] if lr is None else lr))
@@ -406,8 +407,10 @@ def brute_force_step(W, m, d, p, grads, e_w, e_s, lamb=False, lr=None):
         buf, s2 = bcast[j]
         m_hat[b:e] = s2 * _unpack_bytes(buf, e - b)
     u = m_hat / d
-    ratio = 1.0
-    if lamb and np.linalg.norm(p) > 0 and np.linalg.norm(u) > 0:
+    given, ratio = ratio, 1.0
+    if lamb and given is not None:
+        ratio = F64(given)
+    elif lamb and np.linalg.norm(p) > 0 and np.linalg.norm(u) > 0:
         ratio = np.linalg.norm(p) / np.linalg.norm(u)
     res["ratio"] = ratio
     res["p"] = p - lr * ratio * u
@@ -595,6 +598,58 @@ def pin_lamb_brute_force_message_passing(o, seed=24):
                 np.testing.assert_allclose(p, ref["p"], rtol=1e-5, atol=1e-8)
 
 
+def pin_lamb_frozen_ratio_run(o, seed=25):
+    """The frozen-ratio reading of 1-bit LAMB, end to end on OracleRun:
+    LAMB warmup steps, then the freeze keeping the last warmup step's trust
+    ratios (like the variance), then compressed steps that scale each
+    tensor's update by the kept ratio.  Against float64: a LAMB warmup run
+    beside it (numpy's ||p|| / ||r||, the step -lr ratio r), whose last
+    ratios are the kept ones, and for each compressed step the
+    message-passing brute force with those ratios from the run's state."""
+    from oracle import OracleRun
+
+    rng = np.random.default_rng(seed)
+    W, sizes, Tw = 3, (200, 33, 0), 3
+    hp = dict(HP, lr=LAMB_LR)
+    lr = F64(F32(LAMB_LR))
+    b1, b2, eps = F64(F32(HP["beta1"])), F64(F32(HP["beta2"])), F64(F32(HP["eps"]))
+    params = [rng.normal(0, 0.02, n).astype(F32) for n in sizes]
+    run = OracleRun(params, W, hp, oracle=o, lamb=True, lamb_frozen=True)
+    P = [a.astype(F64) for a in params]
+    M = [np.zeros(n) for n in sizes]
+    V = [np.zeros(n) for n in sizes]
+    kept = np.ones(len(sizes))
+    for t in range(1, Tw + 1):
+        g = [[rng.normal(0, 1e-3, n).astype(F32) for n in sizes] for _ in range(W)]
+        run.warmup_step(g)
+        for k, n in enumerate(sizes):
+            gbar = sum(g[w][k].astype(F64) for w in range(W)) / W
+            M[k] = b1 * M[k] + (1 - b1) * gbar
+            V[k] = b2 * V[k] + (1 - b2) * gbar * gbar
+            r = (M[k] / (1 - b1 ** t)) / (np.sqrt(V[k] / (1 - b2 ** t)) + eps)
+            if n and np.linalg.norm(P[k]) > 0 and np.linalg.norm(r) > 0:
+                kept[k] = np.linalg.norm(P[k]) / np.linalg.norm(r)
+            else:
+                kept[k] = 1.0
+            P[k] = P[k] - lr * kept[k] * r
+            assert abs(F64(run.ratio[k]) - kept[k]) <= 1e-5 * kept[k], (t, k)
+    run.freeze()
+    assert np.array_equal(run.frozen_ratio, run.ratio)
+    for _ in range(3):
+        g = [[rng.normal(0, 1e-3, n).astype(F32) for n in sizes] for _ in range(W)]
+        before = [(run.m[k].astype(F64), run.d[k].astype(F64), run.p[k].astype(F64),
+                   [run.e_w[w][k].astype(F64) for w in range(W)], run.e_s[k].astype(F64))
+                  for k in range(len(sizes))]
+        run.compressed_step(g)
+        assert np.array_equal(run.ratio, run.frozen_ratio)   # not recomputed
+        for k, n in enumerate(sizes):
+            m, d, p, e_w, e_s = before[k]
+            ref = brute_force_step(W, m, d, p, [g[w][k].astype(F64) for w in range(W)], e_w, e_s,
+                                   lamb=True, lr=LAMB_LR, ratio=kept[k])
+            np.testing.assert_allclose(run.m[k], ref["m"], rtol=1e-5, atol=1e-12)
+            np.testing.assert_allclose(run.p[k], ref["p"], rtol=1e-5, atol=1e-8)
+
+
 # ---------------------------------------------------------------------------
 # communication volume                              [1BA, Abstract]
 # ---------------------------------------------------------------------------
@@ -652,4 +707,5 @@ ALL_PINS = [
     pin_lamb_warmup_layerwise_step,
     pin_lamb_compressed_update,
     pin_lamb_brute_force_message_passing,
+    pin_lamb_frozen_ratio_run,
 ]

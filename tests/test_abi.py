@@ -147,3 +147,17 @@ def test_product_package_does_not_touch_the_oracle():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".c")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"\boracle\b", text.replace("the oracle", "")), f
+
+
+def test_binding_constants_match_the_header_defines():
+    """Every integer #define of include/onebit.h has the binding's value."""
+    text = open(HEADER).read()
+    defines = re.findall(r"^#define\s+(OB_\w+)\s+\(?\(?(?:int64_t\))?\s*([0-9x]+)\s*(?:<<\s*(\d+))?\)?", text, re.M)
+    assert defines
+    for name, value, shift in defines:
+        v = int(value, 0) << (int(shift) if shift else 0)
+        assert getattr(B, name) == v, name
+    assert {"OB_LAYERWISE_OFF", "OB_LAYERWISE_STEP", "OB_LAYERWISE_FROZEN"} <= {d[0] for d in defines}
+    assert [B.layerwise_mode(m) for m in (False, True, "off", "step", "frozen", 2)] == [0, 1, 0, 1, 2, 2]
+    with pytest.raises(ValueError):
+        B.layerwise_mode("sometimes")

@@ -114,3 +114,39 @@ def test_pins_catch_planted_mistake(name, old, new, source, tmp_path):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"no pin catches the planted mistake {name}"
+
+
+# Mistakes in the runner's frozen-ratio bookkeeping (the 1-bit LAMB
+# reading whose ratios are kept at the freeze): planted by wrapping
+# OracleRun's methods; pin_lamb_frozen_ratio_run must fail on each.
+def _recompute_after_freeze(run_cls):
+    freeze = run_cls.freeze
+
+    def patched(self):
+        freeze(self)
+        self.lamb_frozen = False          # the ratios recomputed after all
+    return {"freeze": patched}
+
+
+def _keep_first_warmup_ratio(run_cls):
+    warmup_step, freeze = run_cls.warmup_step, run_cls.freeze
+
+    def warm(self, grads):
+        warmup_step(self, grads)
+        if self.t_warmup == 1:
+            self._first_ratio = self.ratio.copy()
+
+    def frz(self):
+        freeze(self)
+        if self.lamb_frozen:
+            self.frozen_ratio = self._first_ratio.copy()   # the first step's, not the last
+    return {"warmup_step": warm, "freeze": frz}
+
+
+@pytest.mark.parametrize("plant", [_recompute_after_freeze, _keep_first_warmup_ratio],
+                         ids=["recomputed_after_freeze", "first_warmup_ratio_kept"])
+def test_frozen_ratio_pin_catches_runner_mistakes(plant, monkeypatch):
+    for name, fn in plant(oracle.OracleRun).items():
+        monkeypatch.setattr(oracle.OracleRun, name, fn)
+    with pytest.raises(AssertionError):
+        oracle_pins.pin_lamb_frozen_ratio_run(oracle.default())
