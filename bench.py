@@ -664,7 +664,7 @@ def run_b200(args) -> None:
     offsets, n_pad = B.ob_layout(wl.numels)
     params = WL.make_params(wl, offsets, n_pad, device=dev)
     scale = WL.grad_scale_vector(wl, offsets, n_pad, device=dev)
-    opt = OneBitAdam(wl.numels, wl.W, params=params, device=dev, layerwise=args.lamb, **WL.HYPER)
+    opt = OneBitAdam(wl.numels, wl.W, params=params, device=dev, layerwise=args.lamb or False, **WL.HYPER)
     set_bytes = 4 * wl.W * n_pad
     free_bytes = torch.cuda.mem_get_info(dev)[0]
     n_sets = GRAD_SETS if free_bytes > GRAD_SETS * set_bytes + 2 * 4 * n_pad + (1 << 30) else 1
@@ -726,7 +726,7 @@ def run_b200(args) -> None:
 
     # roofline of the dominant kernel, from its own events over the timed region
     peak = measured_peaks()
-    algo = algorithmic_bytes(wl.n, wl.W, lamb=args.lamb)
+    algo = algorithmic_bytes(wl.n, wl.W, lamb=bool(args.lamb))
     pack_ms, pack_n = prof["ob_pack_kernel"]
     pack_avg_s = pack_ms / 1e3 / max(1, pack_n)
     achieved = algo["ob_pack_kernel"] / pack_avg_s / 1e9
@@ -742,7 +742,7 @@ def run_b200(args) -> None:
             if name in algo:
                 entry["gbs"] = algo[name] / (kms / args.steps / 1e3) / 1e9
                 entry["algorithmic_bytes_per_launch"] = algo[name]
-                entry["traffic"] = measured_traffic(traffic_key(name, args.lamb), wl.n, wl.W)
+                entry["traffic"] = measured_traffic(traffic_key(name, bool(args.lamb)), wl.n, wl.W)
             per_kernel[name] = entry
 
     # the pre-path (full-precision Adam warmup and the freeze), timed by the
@@ -756,7 +756,7 @@ def run_b200(args) -> None:
             pre_path[name] = {"launches": cnt, "avg_launch_ms": kms / cnt, "gbs": gbs,
                               "frac_of_measured_hbm": gbs / peak["hbm_gbs"],
                               "algorithmic_bytes_per_launch": algo[name],
-                              "traffic": measured_traffic(traffic_key(name, args.lamb), wl.n, wl.W)}
+                              "traffic": measured_traffic(traffic_key(name, bool(args.lamb)), wl.n, wl.W)}
 
     # end to end: host gradients in pinned memory, copied in every step, and
     # the step's server scales read back, through ob_compressed_step_host
@@ -789,7 +789,8 @@ def run_b200(args) -> None:
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": dict(workload_config(wl, n_pad, f"replicas{world}" if world > 1 else "single GPU",
                                            n_sets),
-                           optimizer="1-bit LAMB (layerwise trust ratios)" if args.lamb else "1-bit Adam"),
+                           optimizer=(f"1-bit LAMB (layerwise trust ratios, {args.lamb})" if args.lamb
+                                      else "1-bit Adam")),
             "params_per_s_aggregate_all_workers": value * wl.W,
             "hbm_gbs_step": step_gbs,
             "hbm_frac_of_measured_peak_step": step_gbs / peak["hbm_gbs"],
@@ -841,8 +842,10 @@ def main(argv=None):
     ap.add_argument("--peer-words", action="store_true",
                     help="with the split step on N > 1 GPUs: the kernels store and load the sign "
                          "words over peer memory (CUDA IPC) instead of NCCL moving them")
-    ap.add_argument("--lamb", action="store_true",
-                    help="time 1-bit LAMB (layerwise trust ratios, ob_set_layerwise) instead of 1-bit Adam")
+    ap.add_argument("--lamb", nargs="?", const="step", default=None, choices=["step", "frozen"],
+                    help="time 1-bit LAMB (layerwise trust ratios, ob_set_layerwise) instead of 1-bit "
+                         "Adam: ratios recomputed every step (step, the default) or kept at the "
+                         "freeze (frozen)")
     ap.add_argument("--overlap", action="store_true",
                     help="also measure bucketed steps overlapping a synthetic backward pass")
     ap.add_argument("--split-ranks", type=int, default=0,
